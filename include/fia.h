@@ -1,0 +1,205 @@
+/*
+ * fia.h -- C ABI of the B200 paged fused-inference-attention library (libfia.so).
+ *
+ * Operation (aclnnFusedInferAttentionScoreV4 "Formula"; V3 "Formula"):
+ *
+ *     attnOut = Softmax(qkScale * Q K^T + bias) V
+ *
+ * over a paged K/V cache (V4/V3 paged-attention bullets: the blocks that
+ * blockTables lists for a sequence form one logically contiguous K/V run),
+ * with GQA head grouping, an internally generated causal mask, an ALiBi bias
+ * from per-head slopes, an optional full pse-shift bias, an optional lse
+ * output, an optional per-head learnable sink and an optional int8 K/V cache
+ * with per-channel dequantisation.  One call covers both the prefill /
+ * prefix-encoder case (several new tokens per sequence attending to the cached
+ * prefix and to themselves) and single-token decode.
+ *
+ * Call pattern (the two-phase convention of the aclnn API and of the ATB
+ * PrefixEncoder interface, "Definition"):
+ *
+ *     fia_get_workspace_size(...)  -> validates everything, plans the launch,
+ *                                     reports the workspace size, returns an op
+ *     fia_run(workspace, size, op, stream)
+ *                                  -> enqueues the kernels on the stream
+ *     fia_op_destroy(op)
+ *
+ * Conventions that hold for every entry point:
+ *  - Every tensor is dense, row-major and contiguous.  `data` is a DEVICE
+ *    pointer unless a parameter says "host".  The caller owns every buffer;
+ *    the op keeps pointers, not copies, so the tensors and the workspace must
+ *    stay alive and unchanged until the stream has finished fia_run.
+ *  - Phase 1 launches nothing and reads or writes no device memory.  It does
+ *    query the current device's attributes and encodes TMA descriptors, so it
+ *    needs a CUDA device (it returns FIA_ERR_CUDA without one).
+ *  - fia_run is asynchronous on `stream`, allocates nothing and does not
+ *    synchronise.  It may be called any number of times on the same op.
+ *  - Block ids in blockTables are not validated on the device (the pages say
+ *    the same: "the validity of block IDs is not verified").  Entries past
+ *    ceil(kvSeqLen[b] / blockSize) are never read.
+ *  - Errors are returned as fia_status; nothing is printed and nothing aborts.
+ */
+#ifndef FIA_H
+#define FIA_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FIA_API __attribute__((visibility("default")))
+#else
+#define FIA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FIA_OK = 0,
+    FIA_ERR_NULLPTR = 1,     /* a required pointer is NULL                        */
+    FIA_ERR_PARAM = 2,       /* a scalar parameter is out of range                */
+    FIA_ERR_DTYPE = 3,       /* a tensor has a dtype the operation does not take  */
+    FIA_ERR_SHAPE = 4,       /* tensor ranks / extents are inconsistent           */
+    FIA_ERR_UNSUPPORTED = 5, /* valid per the pages but not built (e.g. D=96)     */
+    FIA_ERR_WORKSPACE = 6,   /* workspace NULL, misaligned or smaller than needed */
+    FIA_ERR_CUDA = 7         /* a CUDA runtime / driver call failed               */
+} fia_status;
+
+typedef enum { FIA_F16 = 0, FIA_BF16 = 1, FIA_F32 = 2, FIA_I8 = 3, FIA_I32 = 4 } fia_dtype;
+
+/* A dense row-major tensor: dims[0] is the slowest axis.  ndim <= 4. */
+typedef struct {
+    void *data;
+    fia_dtype dtype;
+    int32_t ndim;
+    int64_t dims[4];
+} fia_tensor;
+
+/* maskType codes of the ATB PrefixEncoder table ("maskType" row). */
+typedef enum {
+    FIA_MASK_NONE = 0,   /* no mask: every key t < kvSeqLen[b] is visible              */
+    FIA_MASK_ALIBI = 3,  /* MASK_TYPE_ALIBI_COMPRESS: causal mask plus the ALiBi bias
+                            slope_h * (t - qpos), generated in registers from `slopes` */
+    FIA_MASK_CAUSAL = 9  /* MASK_TYPE_CAUSAL_MASK: internally generated causal mask     */
+} fia_mask_type;
+
+/* Optional extensions; the struct pointer and every field may be NULL. */
+typedef struct {
+    /* pse-shift bias [batch, headNum, maxQ, maxKV], the query's dtype, added to
+       the scaled scores: s += pse[b][h][i][t] for new token i and key position t
+       (V4 "alibi fullmask" restrictions: shape [B, N, maxQ, maxKV]).  Needs
+       maxQ >= max seqLen and maxKV >= max kvSeqLen.  Not combinable with
+       FIA_MASK_ALIBI. */
+    const fia_tensor *pse;
+    /* learnable sink [headNum] f32 (V4 learnableSinkOptional): a raw logit,
+       not scaled by qkScale, that joins the softmax denominator with no value
+       row.  lse includes it. */
+    const fia_tensor *sink;
+    /* int8 K/V dequantisation, per (kvHead, channel): [kvHeadNum, headSize] f32
+       (V3 fake-quantization bullets, per-channel mode).  The cache value x
+       stands for scale * (x + offset).  kScale and vScale are required when
+       key/value are FIA_I8; a NULL offset means 0 (symmetric). */
+    const fia_tensor *kScale;
+    const fia_tensor *kOffset;
+    const fia_tensor *vScale;
+    const fia_tensor *vOffset;
+    /* lse output [nTokens, headNum] f32 (V3 "lse" bullet): m + log(sum exp(s - m)).
+       Rows with no visible key get +inf. */
+    fia_tensor *lse;
+} fia_ext;
+
+typedef struct fia_op fia_op;
+
+/*
+ * Phase 1 (ATB AtbSelfAttentionPrefixEncoderGetWorkspaceSize; aclnn
+ * ...GetWorkspaceSize "implements input parameter verification").
+ *
+ *  query        [nTokens, headNum, headSize] or [nTokens, headNum*headSize], f16|bf16.
+ *               The new tokens of all sequences, concatenated in batch order.
+ *  key, value   [numBlocks, blockSize, kvHeadNum, headSize] or
+ *               [numBlocks, blockSize, kvHeadNum*headSize]; the query's dtype, or
+ *               FIA_I8 with ext->kScale/vScale.  Same shape.
+ *  blockTables  [batch, maxBlockNum] int32, device.  maxBlockNum must cover
+ *               ceil(kvSeqLen[b] / blockSize) for every b.
+ *  seqLen       host int32[batch]: new tokens per sequence; sum == nTokens.
+ *  kvSeqLen     host int32[batch]: cached tokens per sequence INCLUDING the new
+ *               ones (the new tokens' K/V are already in the cache); new token
+ *               i of sequence b sits at position qpos = kvSeqLen[b]-seqLen[b]+i.
+ *               seqLen[b] <= kvSeqLen[b] unless kvSeqLen[b] == 0 (rows with no
+ *               keys: out 0, lse +inf).
+ *  batch        number of sequences, >= 0.
+ *  slopes       [headNum] f32 device, required for FIA_MASK_ALIBI, else NULL.
+ *  maskType     FIA_MASK_NONE | FIA_MASK_ALIBI | FIA_MASK_CAUSAL.
+ *  headNum      > 0;  kvHeadNum > 0 and headNum % kvHeadNum == 0; query head h
+ *               reads KV head h / (headNum / kvHeadNum).
+ *  qkScale      multiplies Q K^T before the bias is added (PrefixEncoder
+ *               "post-multiplied by Q*K^T").
+ *  ext          optional extensions (see fia_ext), may be NULL.
+ *  attnOut      [nTokens, headNum, headSize] (or 2-D), the query's dtype.
+ *  workspaceSize  out: bytes of device workspace fia_run needs (0 if none).
+ *  op           out: the planned operation; free with fia_op_destroy.
+ *
+ * Supported build limits: headSize in {64, 128}; blockSize a multiple of 16,
+ * 16 <= blockSize <= 256; headNum <= 1024.  Everything else the pages allow
+ * returns FIA_ERR_UNSUPPORTED.
+ * nTokens == 0 returns FIA_OK with workspaceSize 0 and an op whose run is a no-op.
+ */
+FIA_API fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key,
+                                  const fia_tensor *value, const fia_tensor *blockTables,
+                                  const int32_t *seqLen, const int32_t *kvSeqLen, int32_t batch,
+                                  const fia_tensor *slopes, int32_t maskType, int32_t headNum,
+                                  int32_t kvHeadNum, float qkScale, const fia_ext *ext,
+                                  fia_tensor *attnOut, uint64_t *workspaceSize, fia_op **op);
+
+/*
+ * Phase 2 (ATB AtbSelfAttentionPrefixEncoder; aclnn second-phase call).
+ *  workspace      device buffer of at least workspaceSize bytes, 256-byte aligned
+ *                 (may be NULL only when workspaceSize was 0).  Its contents
+ *                 are scratch: fia_run overwrites them.
+ *  stream         a cudaStream_t (0 = legacy default stream), passed as void*.
+ * Returns FIA_ERR_WORKSPACE for a NULL/misaligned/too-small workspace and
+ * FIA_ERR_CUDA when a copy or launch fails (the op stays usable).
+ */
+FIA_API fia_status fia_run(void *workspace, uint64_t workspaceSize, fia_op *op, void *stream);
+
+/* Frees the op (host memory only).  NULL is a no-op. */
+FIA_API void fia_op_destroy(fia_op *op);
+
+/* Static, human-readable text for a status code. */
+FIA_API const char *fia_status_string(fia_status s);
+
+/*
+ * Measurement hook: when both events are non-NULL, fia_run records `start`
+ * immediately before its main attention kernel and `stop` immediately after
+ * its last kernel, on the run's stream, so that cudaEventElapsedTime gives the
+ * device time of the kernels alone (the plan upload is excluded).  Pass NULLs
+ * to switch it off.  Events are cudaEvent_t handles passed as void*, owned by
+ * the caller.
+ */
+FIA_API fia_status fia_op_set_timing_events(fia_op *op, void *start, void *stop);
+
+/*
+ * Introspection of the plan phase 1 chose (for tests and reports).
+ *   path            0 = no-op, 1 = decode (split-KV + combine), 2 = prefill (tcgen05)
+ *   kernels_per_run number of kernel launches one fia_run makes
+ *   work_items      decode: split units; prefill: (q-tile, head) items
+ *   grid            CTAs of the main kernel
+ *   (NULL op or info -> FIA_ERR_NULLPTR)
+ */
+typedef struct {
+    int32_t path;
+    int32_t kernels_per_run;
+    int64_t work_items;
+    int32_t grid;
+    int32_t split_tokens;     /* decode: keys per split unit (0 otherwise)            */
+    int64_t error_word_offset;/* byte offset in the workspace of a uint32 that a kernel
+                                 sets non-zero when a bounded internal wait runs out;
+                                 fia_run clears it                                     */
+} fia_plan_info;
+
+FIA_API fia_status fia_op_get_plan_info(const fia_op *op, fia_plan_info *info);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FIA_H */

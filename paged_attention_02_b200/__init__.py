@@ -1,0 +1,157 @@
+"""B200-native paged fused inference attention.
+
+    out = Softmax(qkScale * Q K^T + bias) V
+
+over a paged K/V cache, for prefill / prefix-encoder and decode, on sm_100a
+kernels behind the C ABI of ``include/fia.h`` (libfia.so).  This module is the
+thin Python face of that ABI: it turns torch CUDA tensors into ``fia_tensor``
+descriptors, allocates the workspace phase 1 asks for, and calls the two
+phases.  All arithmetic runs in the CUDA kernels; nothing here computes
+attention, and a missing libfia.so raises at import.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Sequence
+
+import torch
+
+from . import _lib
+from ._lib import (FIA_MASK_ALIBI, FIA_MASK_CAUSAL, FIA_MASK_NONE, FiaError, fia_ext,
+                   fia_plan_info, fia_tensor)
+
+__all__ = ["FiaOp", "fused_infer_attention", "FIA_MASK_NONE", "FIA_MASK_ALIBI",
+           "FIA_MASK_CAUSAL", "FiaError", "tensor_desc"]
+
+_DT = {torch.float16: _lib.FIA_F16, torch.bfloat16: _lib.FIA_BF16, torch.float32: _lib.FIA_F32,
+       torch.int8: _lib.FIA_I8, torch.int32: _lib.FIA_I32}
+
+
+def tensor_desc(t: Optional[torch.Tensor]) -> Optional[fia_tensor]:
+    """fia_tensor describing a contiguous torch tensor (None -> None)."""
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("fia tensors must be contiguous")
+    if t.dim() > 4:
+        raise ValueError("fia tensors have at most 4 dims")
+    d = fia_tensor()
+    d.data = ctypes.c_void_p(t.data_ptr()) if t.numel() > 0 else ctypes.c_void_p(t.data_ptr() or None)
+    d.dtype = _DT[t.dtype]
+    d.ndim = t.dim()
+    for i, n in enumerate(t.shape):
+        d.dims[i] = int(n)
+    return d
+
+
+def _ptr(d: Optional[fia_tensor]):
+    return ctypes.pointer(d) if d is not None else None
+
+
+class FiaOp:
+    """One planned call (phase 1 done); ``run()`` enqueues phase 2.
+
+    Arguments follow ``fia_get_workspace_size``: query ``[nTokens, H, D]``,
+    key/value caches ``[numBlocks, blockSize, kvHeadNum, D]``, block table
+    ``[batch, maxBlockNum]`` int32 (all on the same CUDA device), host
+    sequence lengths.  ``out`` / ``lse`` are allocated when not given
+    (``want_lse=False`` skips lse).  Tensors are referenced, not copied: keep
+    them unchanged while runs are in flight.
+    """
+
+    def __init__(self, query, key, value, block_tables, seq_len: Sequence[int],
+                 kv_seq_len: Sequence[int], head_num: int, kv_head_num: int, qk_scale: float,
+                 mask_type: int = FIA_MASK_NONE, slopes=None, pse=None, sink=None, k_scale=None,
+                 k_offset=None, v_scale=None, v_offset=None, out=None, lse=None,
+                 want_lse: bool = True):
+        dev = query.device
+        self.out = out if out is not None else torch.empty_like(query)
+        if lse is None and want_lse:
+            lse = torch.empty((query.shape[0], head_num), dtype=torch.float32, device=dev)
+        self.lse = lse
+        self._keep = [query, key, value, block_tables, slopes, pse, sink, k_scale, k_offset,
+                      v_scale, v_offset, self.out, self.lse]
+        self._d = {n: tensor_desc(t) for n, t in
+                   dict(q=query, k=key, v=value, bt=block_tables, slopes=slopes, pse=pse,
+                        sink=sink, ks=k_scale, ko=k_offset, vs=v_scale, vo=v_offset,
+                        out=self.out, lse=self.lse).items()}
+        self._ext = fia_ext(_ptr(self._d["pse"]), _ptr(self._d["sink"]), _ptr(self._d["ks"]),
+                            _ptr(self._d["ko"]), _ptr(self._d["vs"]), _ptr(self._d["vo"]),
+                            _ptr(self._d["lse"]))
+        b = len(seq_len)
+        self._sl = (ctypes.c_int32 * max(b, 1))(*[int(x) for x in seq_len])
+        self._kl = (ctypes.c_int32 * max(b, 1))(*[int(x) for x in kv_seq_len])
+        self._op = ctypes.c_void_p()
+        ws = ctypes.c_uint64(0)
+        with torch.cuda.device(dev):
+            st = _lib.fia_get_workspace_size(
+                _ptr(self._d["q"]), _ptr(self._d["k"]), _ptr(self._d["v"]), _ptr(self._d["bt"]),
+                self._sl, self._kl, b, _ptr(self._d["slopes"]), int(mask_type), int(head_num),
+                int(kv_head_num), float(qk_scale), ctypes.pointer(self._ext), _ptr(self._d["out"]),
+                ctypes.byref(ws), ctypes.byref(self._op))
+        if st != _lib.FIA_OK:
+            raise FiaError(st, "fia_get_workspace_size")
+        self.workspace_size = int(ws.value)
+        # 256-byte aligned device workspace (torch's allocator aligns to 512 B)
+        self.workspace = torch.empty(max(self.workspace_size, 1), dtype=torch.uint8, device=dev)
+        self._timing = None
+
+    def run(self, stream: Optional[torch.cuda.Stream] = None):
+        s = stream if stream is not None else torch.cuda.current_stream(self.out.device)
+        st = _lib.fia_run(ctypes.c_void_p(self.workspace.data_ptr()), self.workspace_size,
+                          self._op, ctypes.c_void_p(s.cuda_stream))
+        if st != _lib.FIA_OK:
+            raise FiaError(st, "fia_run")
+        return self.out, self.lse
+
+    def plan_info(self) -> dict:
+        info = fia_plan_info()
+        st = _lib.fia_op_get_plan_info(self._op, ctypes.byref(info))
+        if st != _lib.FIA_OK:
+            raise FiaError(st, "fia_op_get_plan_info")
+        return {f: getattr(info, f) for f, _ in fia_plan_info._fields_}
+
+    def error_word(self) -> int:
+        """Value of the kernels' error word after the last run (syncs the device)."""
+        off = self.plan_info()["error_word_offset"]
+        if self.workspace_size == 0:
+            return 0
+        return int(self.workspace[off:off + 4].view(torch.int32).item())
+
+    def set_timing_events(self, start: Optional[torch.cuda.Event], stop: Optional[torch.cuda.Event]):
+        """Have run() record ``start``/``stop`` around its kernels only."""
+        if start is None:
+            st = _lib.fia_op_set_timing_events(self._op, None, None)
+        else:
+            s = torch.cuda.current_stream(self.out.device)
+            start.record(s)    # make sure the events exist before taking their handles
+            stop.record(s)
+            st = _lib.fia_op_set_timing_events(self._op, ctypes.c_void_p(start.cuda_event),
+                                               ctypes.c_void_p(stop.cuda_event))
+        if st != _lib.FIA_OK:
+            raise FiaError(st, "fia_op_set_timing_events")
+        self._timing = (start, stop)
+
+    def close(self):
+        if getattr(self, "_op", None) is not None and self._op.value:
+            _lib.fia_op_destroy(self._op)
+            self._op = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def fused_infer_attention(query, key, value, block_tables, seq_len, kv_seq_len, head_num,
+                          kv_head_num, qk_scale, mask_type=FIA_MASK_NONE, slopes=None, pse=None,
+                          sink=None, k_scale=None, k_offset=None, v_scale=None, v_offset=None,
+                          want_lse=True):
+    """One-shot call: plan, run on the current stream, return (out, lse)."""
+    op = FiaOp(query, key, value, block_tables, seq_len, kv_seq_len, head_num, kv_head_num,
+               qk_scale, mask_type, slopes, pse, sink, k_scale, k_offset, v_scale, v_offset,
+               want_lse=want_lse)
+    out, lse = op.run()
+    op._keep.append(op.workspace)
+    return out, lse

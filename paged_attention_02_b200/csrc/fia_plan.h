@@ -1,0 +1,91 @@
+// fia_plan.h -- launch parameters shared by the host planner and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <stdint.h>
+
+namespace fia {
+
+// Per-sequence facts, uploaded to the workspace by fia_run.
+struct SeqInfo {
+    int32_t cu_q;    // first token of the sequence inside query / attnOut
+    int32_t qlen;    // seqLen[b]
+    int32_t kvlen;   // kvSeqLen[b]
+    int32_t pad;
+};
+
+// Decode work unit: one (sequence, kv head, key range) split.
+struct DecodeUnit {
+    int32_t b, kvh, t_begin, t_end;
+    int32_t slot;    // partial-result slot (logical split order within (b, kvh))
+    int32_t pad[3];
+};
+
+// Decode combine item: the splits of one (sequence, kv head).
+struct CombineItem {
+    int32_t slot0, nsplit, b, kvh;
+};
+
+// Prefill work item: 128 new tokens of one sequence for one query head.
+struct PrefillItem {
+    int32_t b, q0, h, pad;
+};
+
+constexpr int kDecodeRows = 16;      // rows (new token x head-in-group) per decode unit
+constexpr int kDecodeTile = 64;      // keys per decode pipeline stage
+constexpr int kPrefillBM = 128;      // new tokens per prefill item
+constexpr int kPrefillBN = 128;      // keys per prefill tile
+
+struct CommonArgs {
+    const void *q;          // [nTokens, H, D]
+    void *out;              // [nTokens, H, D]
+    float *lse;             // [nTokens, H] or null
+    const int32_t *bt;      // [B, bt_stride]
+    const SeqInfo *seq;     // workspace
+    const float *slopes;    // [H] (mask 3) or null
+    const void *pse;        // [B, H, pse_q, pse_kv] or null
+    const float *sink;      // [H] or null
+    uint32_t *err;          // workspace error word
+    int64_t pse_q, pse_kv;
+    int32_t bt_stride;
+    int32_t H, KVH, g, D, bs, box_rows;
+    int32_t mask_type;
+    int32_t pse_vec;        // pse rows 16-byte aligned (vector loads allowed)
+    float scale_log2;       // qkScale * log2(e)
+};
+
+struct DecodeArgs {
+    CommonArgs c;
+    const DecodeUnit *units;
+    float *part_o;          // [slots][16][D]
+    float2 *part_ml;        // [slots][16] (m in log2 units, l)
+    const float *k_scale, *k_offset;   // int8 only
+    int32_t n_units;
+};
+
+struct CombineArgs {
+    CommonArgs c;
+    const CombineItem *items;
+    const float *part_o;
+    const float2 *part_ml;
+    const float *v_scale, *v_offset;   // int8 only
+    int32_t n_items;
+};
+
+struct PrefillArgs {
+    CommonArgs c;
+    const int32_t *cta_off;        // [grid + 1]
+    const PrefillItem *items;
+};
+
+// Kernel launchers (defined in the .cu files).
+cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap &tk, const CUtensorMap &tv,
+                          int q_dtype, bool kv_int8, int grid, cudaStream_t s);
+cudaError_t launch_combine(const CombineArgs &a, int q_dtype, bool kv_int8, int grid,
+                           cudaStream_t s);
+cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tq, const CUtensorMap &tk,
+                           const CUtensorMap &tv, int q_dtype, int grid, cudaStream_t s);
+int decode_smem_bytes(int D, bool kv_int8);
+int prefill_smem_bytes(int D);
+
+}  // namespace fia

@@ -1,0 +1,482 @@
+// prefill_kernel.cu -- paged prefill / prefix-encoder attention on sm_100a
+// tensor cores (tcgen05 UMMA, TMEM accumulators, TMA-staged paged K/V).
+//
+// Computes, for 128 new tokens of one sequence and one query head at a time,
+//     O = Softmax(qkScale * Q K^T + bias) V
+// (aclnnFusedInferAttentionScoreV4 / V3 "Formula"; ATB PrefixEncoder: new
+// tokens attend to the cached prefix and to themselves, maskType 9 causal
+// generated internally, maskType 3 ALiBi from per-head slopes; V4 alibi
+// fullmask = pse tensor; V4 learnable sink; V3 lse bullet).
+//
+// One persistent CTA per SM walks a host-planned, longest-first list of
+// (sequence, 128-token tile, head) items.  Warp roles:
+//   warp 0   TMA producer: Q tile once per item, then K and V tiles of 128
+//            keys, each tile gathered block by block through the block table
+//            into a 2-stage ring (128-byte swizzled, K-major rows).
+//   warp 1   UMMA issuer (one elected lane): S_j = Q K_j^T into one of two
+//            TMEM S buffers, then O += P_{j-1} V_{j-1} into the TMEM O buffer,
+//            so the next QK^T overlaps the softmax of the previous tile.
+//            It also zeroes the V rows past kvSeqLen in a ragged last tile.
+//   warps 2-5 softmax + epilogue, one query row per thread (TMEM lane):
+//            tcgen05.ld the S row, scale / mask / bias in registers, online
+//            softmax in fp32 (log2 domain, rescale of O in TMEM only when the
+//            running max grows by more than 2^8), P rounded to the input dtype
+//            into shared memory for the PV MMA; at the end O / l, the sink
+//            term and lse.
+// Every mbarrier wait is bounded in time (see fia_device.cuh).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "fia_device.cuh"
+#include "fia_plan.h"
+
+namespace fia {
+
+template <int D>
+struct PrefillCfg {
+    static constexpr int kHalves = D / 64;                 // 128-byte column groups
+    static constexpr int kTileBytes = 128 * D * 2;         // Q, K or V tile (128 rows)
+    static constexpr int kGroupBytes = 128 * 128;          // one 128-row x 128-byte group
+    static constexpr int kStages = 2;
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kOffQ + kTileBytes;       // K[s] = kOffK + s * 2 * kTileBytes
+    static constexpr int kOffP = kOffK + kStages * 2 * kTileBytes;
+    static constexpr int kPBytes = 128 * 128 * 2;
+    static constexpr int kOffBar = kOffP + kPBytes;
+    static constexpr int kNumBar = 14;
+    static constexpr int kUsed = kOffBar + kNumBar * 8 + 16;
+    // Keep one CTA per SM (each CTA holds all 512 TMEM columns).
+    static constexpr int kSmem = 1024 + (kUsed > 118 * 1024 ? kUsed : 118 * 1024);
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+};
+
+int prefill_smem_bytes(int D) {
+    if (D == 64) return PrefillCfg<64>::kSmem;
+    if (D == 128) return PrefillCfg<128>::kSmem;
+    return -1;
+}
+
+struct ItemGeom {
+    int b, q0, h, kvh, cu_q, qlen, kvlen, rows, kv_end, n;
+};
+
+__device__ __forceinline__ ItemGeom item_geom(const PrefillArgs &a, int idx) {
+    const PrefillItem it = a.items[idx];
+    const SeqInfo si = a.c.seq[it.b];
+    ItemGeom g;
+    g.b = it.b; g.q0 = it.q0; g.h = it.h; g.kvh = it.h / a.c.g;
+    g.cu_q = si.cu_q; g.qlen = si.qlen; g.kvlen = si.kvlen;
+    g.rows = min(kPrefillBM, si.qlen - it.q0);
+    const bool causal = (a.c.mask_type == 9 || a.c.mask_type == 3);
+    g.kv_end = causal ? min(si.kvlen, si.kvlen - si.qlen + it.q0 + g.rows) : si.kvlen;
+    if (g.kv_end < 0) g.kv_end = 0;
+    g.n = (g.kv_end + kPrefillBN - 1) / kPrefillBN;
+    return g;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(192, 1)
+fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tq,
+                   const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
+    using Cfg = PrefillCfg<D>;
+    constexpr bool BF = MmaType<T>::bf16;
+    constexpr uint32_t IDESC_QK = umma_idesc_f16(BF, false, false, 128, kPrefillBN);
+    constexpr uint32_t IDESC_PV = umma_idesc_f16(BF, false, true, 128, D);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
+    uint64_t *q_full = bars + 0;
+    uint64_t *q_empty = bars + 1;
+    uint64_t *k_full = bars + 2;      // [2]
+    uint64_t *v_full = bars + 4;      // [2]
+    uint64_t *kv_empty = bars + 6;    // [2]
+    uint64_t *s_full = bars + 8;      // [2]
+    uint64_t *s_empty = bars + 10;    // [2]
+    uint64_t *p_full = bars + 12;
+    uint64_t *pv_done = bars + 13;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + Cfg::kNumBar);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    // o_full shares the pv_done phase sequence: a separate barrier keeps the
+    // epilogue wait independent of the per-tile waits.
+    __shared__ uint64_t o_full_bar;
+    uint64_t *o_full = &o_full_bar;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+
+    if (tid == 0) {
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+            mbar_init(&s_full[s], 1);
+            mbar_init(&s_empty[s], 4);
+        }
+        mbar_init(p_full, 4);
+        mbar_init(pv_done, 1);
+        mbar_init(o_full, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tq);
+        tma_prefetch_desc(&tk);
+        tma_prefetch_desc(&tv);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, Cfg::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const int it_begin = a.cta_off[blockIdx.x];
+    const int it_end = a.cta_off[blockIdx.x + 1];
+    const uint32_t sm_q = smem_u32(smem + Cfg::kOffQ);
+    const uint32_t sm_k0 = smem_u32(smem + Cfg::kOffK);
+    const uint32_t sm_p = smem_u32(smem + Cfg::kOffP);
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            uint32_t q_it = 0, kv_it = 0;
+            const int br = a.c.box_rows;
+            for (int idx = it_begin; idx < it_end; ++idx) {
+                const ItemGeom gm = item_geom(a, idx);
+                if (gm.n == 0) continue;
+                if (!mbar_wait(q_empty, (q_it & 1) ^ 1, abort_flag, a.c.err, 10)) goto done;
+                mbar_arrive_expect_tx(q_full, Cfg::kTileBytes);
+                for (int hv = 0; hv < Cfg::kHalves; ++hv)
+                    tma_load_3d(smem + Cfg::kOffQ + hv * Cfg::kGroupBytes, &tq, q_full, hv * 64,
+                                gm.h, gm.cu_q + gm.q0);
+                ++q_it;
+                const int32_t *bt_row = a.c.bt + (int64_t)gm.b * a.c.bt_stride;
+                for (int j = 0; j < gm.n; ++j, ++kv_it) {
+                    const int st = kv_it & 1;
+                    if (!mbar_wait(&kv_empty[st], ((kv_it >> 1) & 1) ^ 1, abort_flag, a.c.err, 11))
+                        goto done;
+                    const int t0 = j * kPrefillBN;
+                    const int t1 = min(t0 + kPrefillBN, gm.kvlen);
+                    const int nbox = (t1 - t0 + br - 1) / br;
+                    const uint32_t bytes = (uint32_t)(nbox * br * 128 * Cfg::kHalves);
+                    uint8_t *ks = smem + Cfg::kOffK + st * 2 * Cfg::kTileBytes;
+                    uint8_t *vs = ks + Cfg::kTileBytes;
+                    mbar_arrive_expect_tx(&k_full[st], bytes);
+                    for (int bi = 0; bi < nbox; ++bi) {
+                        const int t = t0 + bi * br;
+                        const int prow = bt_row[t / a.c.bs] * a.c.bs + (t % a.c.bs);
+                        for (int hv = 0; hv < Cfg::kHalves; ++hv)
+                            tma_load_3d(ks + hv * Cfg::kGroupBytes + bi * br * 128, &tk, &k_full[st],
+                                        hv * 64, gm.kvh, prow);
+                    }
+                    mbar_arrive_expect_tx(&v_full[st], bytes);
+                    for (int bi = 0; bi < nbox; ++bi) {
+                        const int t = t0 + bi * br;
+                        const int prow = bt_row[t / a.c.bs] * a.c.bs + (t % a.c.bs);
+                        for (int hv = 0; hv < Cfg::kHalves; ++hv)
+                            tma_load_3d(vs + hv * Cfg::kGroupBytes + bi * br * 128, &tv, &v_full[st],
+                                        hv * 64, gm.kvh, prow);
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ UMMA issuer
+        uint32_t q_it = 0, kv_it = 0, s_it = 0, p_it = 0;
+        for (int idx = it_begin; idx < it_end; ++idx) {
+            const ItemGeom gm = item_geom(a, idx);
+            if (gm.n == 0) continue;
+            if (!mbar_wait(q_full, q_it & 1, abort_flag, a.c.err, 20)) goto done;
+            ++q_it;
+            const uint32_t kv_base = kv_it;
+            for (int j = 0; j <= gm.n; ++j) {
+                if (j < gm.n) {
+                    // S_j = Q K_j^T
+                    const uint32_t kvi = kv_base + j;
+                    const int st = kvi & 1;
+                    if (!mbar_wait(&k_full[st], (kvi >> 1) & 1, abort_flag, a.c.err, 21)) goto done;
+                    const int sb = s_it & 1;
+                    if (!mbar_wait(&s_empty[sb], ((s_it >> 1) & 1) ^ 1, abort_flag, a.c.err, 22))
+                        goto done;
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t kbase = sm_k0 + st * 2 * Cfg::kTileBytes;
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t off = (kk >> 2) * Cfg::kGroupBytes + (kk & 3) * 32;
+                            umma_ss(tmem + (sb ? Cfg::kColS1 : Cfg::kColS0),
+                                    umma_desc_sw128(sm_q + off, 16, 1024),
+                                    umma_desc_sw128(kbase + off, 16, 1024), IDESC_QK, kk > 0);
+                        }
+                        umma_commit(&s_full[sb]);
+                        if (j == gm.n - 1) umma_commit(q_empty);
+                    }
+                    __syncwarp();
+                    ++s_it;
+                }
+                if (j >= 1) {
+                    // O += P_{j-1} V_{j-1}
+                    const int jj = j - 1;
+                    const uint32_t kvi = kv_base + jj;
+                    const int st = kvi & 1;
+                    if (!mbar_wait(p_full, p_it & 1, abort_flag, a.c.err, 23)) goto done;
+                    if (!mbar_wait(&v_full[st], (kvi >> 1) & 1, abort_flag, a.c.err, 24)) goto done;
+                    const uint32_t vbase = sm_k0 + st * 2 * Cfg::kTileBytes + Cfg::kTileBytes;
+                    const int valid = gm.kvlen - jj * kPrefillBN;
+                    if (valid < kPrefillBN) {
+                        // rows past kvSeqLen: P is 0 there, but the slots may
+                        // hold anything (NaN * 0 = NaN in the MMA) -> zero them.
+                        uint8_t *vs = smem + Cfg::kOffK + st * 2 * Cfg::kTileBytes + Cfg::kTileBytes;
+                        const int nbytes = (kPrefillBN - valid) * 128;
+                        for (int hv = 0; hv < Cfg::kHalves; ++hv) {
+                            uint4 *p = reinterpret_cast<uint4 *>(vs + hv * Cfg::kGroupBytes + valid * 128);
+                            for (int x = lane; x < nbytes / 16; x += 32) p[x] = make_uint4(0, 0, 0, 0);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                    }
+                    tc_fence_after();
+                    if (lane == 0) {
+#pragma unroll
+                        for (int kk = 0; kk < kPrefillBN / 16; ++kk) {
+                            const uint32_t poff = (kk >> 2) * Cfg::kGroupBytes + (kk & 3) * 32;
+                            umma_ss(tmem + Cfg::kColO, umma_desc_sw128(sm_p + poff, 16, 1024),
+                                    umma_desc_sw128(vbase + kk * 2048, Cfg::kGroupBytes, 1024),
+                                    IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit(pv_done);
+                        umma_commit(&kv_empty[st]);
+                        if (jj == gm.n - 1) umma_commit(o_full);
+                    }
+                    __syncwarp();
+                    ++p_it;
+                }
+            }
+            kv_it = kv_base + gm.n;
+        }
+    } else {
+        // ------------------------------------------------------------ softmax + epilogue
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;
+        const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
+        const bool causal = (a.c.mask_type == 9 || a.c.mask_type == 3);
+        const bool alibi = (a.c.mask_type == 3);
+        const float sl2 = a.c.scale_log2;
+        uint32_t s_it = 0, p_it = 0, o_it = 0;
+        T *outp = reinterpret_cast<T *>(a.c.out);
+        for (int idx = it_begin; idx < it_end; ++idx) {
+            const ItemGeom gm = item_geom(a, idx);
+            const int i = gm.q0 + row;
+            const bool valid = i < gm.qlen;
+            const int qpos = gm.kvlen - gm.qlen + i;
+            const int64_t orow = ((int64_t)(gm.cu_q + i) * a.c.H + gm.h);
+            if (gm.n == 0) {
+                if (valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(outp + orow * D);
+                    for (int x = 0; x < D * 2 / 16; ++x) dst[x] = make_uint4(0, 0, 0, 0);
+                    if (a.c.lse) a.c.lse[orow] = INFINITY;
+                }
+                continue;
+            }
+            const float slope2 = alibi ? a.c.slopes[gm.h] * kLog2e : 0.f;
+            const T *pse_row = nullptr;
+            if (a.c.pse && valid)
+                pse_row = reinterpret_cast<const T *>(a.c.pse) +
+                          (((int64_t)gm.b * a.c.H + gm.h) * a.c.pse_q + i) * a.c.pse_kv;
+            float m = -INFINITY, l = 0.f;
+            for (int j = 0; j < gm.n; ++j) {
+                const int sb = s_it & 1;
+                if (!mbar_wait(&s_full[sb], (s_it >> 1) & 1, abort_flag, a.c.err, 30)) goto done;
+                tc_fence_after();
+                uint32_t sr[4][32];
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc)
+                    tmem_ld32(t_lane + (sb ? Cfg::kColS1 : Cfg::kColS0) + cc * 32, sr[cc]);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_empty[sb]);
+                ++s_it;
+
+                // scores in log2 units, masks, bias
+                const int tb = j * kPrefillBN;
+                const bool edge = (tb + kPrefillBN > gm.kvlen) || (causal && tb + kPrefillBN - 1 > qpos);
+                float mx = -INFINITY;
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) {
+                        const int t = tb + cc * 32 + x;
+                        float v = __uint_as_float(sr[cc][x]) * sl2;
+                        if (alibi) v = fmaf(slope2, (float)(t - qpos), v);
+                        if (edge) {
+                            const bool keep = (t < gm.kvlen) && !(causal && t > qpos);
+                            v = keep ? v : -INFINITY;
+                        }
+                        sr[cc][x] = __float_as_uint(v);
+                    }
+                }
+                if (pse_row) {
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll
+                        for (int x8 = 0; x8 < 4; ++x8) {
+                            const int t = tb + cc * 32 + x8 * 8;
+                            if (a.c.pse_vec && t + 8 <= gm.kvlen) {
+                                const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(pse_row + t));
+                                const T *pv = reinterpret_cast<const T *>(&raw);
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) {
+                                    float v = __uint_as_float(sr[cc][x8 * 8 + e]);
+                                    sr[cc][x8 * 8 + e] = __float_as_uint(fmaf(to_f32<T>(pv[e]), kLog2e, v));
+                                }
+                            } else {
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) {
+                                    if (t + e < gm.kvlen) {
+                                        float v = __uint_as_float(sr[cc][x8 * 8 + e]);
+                                        sr[cc][x8 * 8 + e] =
+                                            __float_as_uint(fmaf(to_f32<T>(pse_row[t + e]), kLog2e, v));
+                                    }
+                                }
+                            }
+                        }
+                    }
+                }
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) mx = fmaxf(mx, __uint_as_float(sr[cc][x]));
+
+                // the previous PV must be complete before O or P is touched
+                if (j > 0) {
+                    if (!mbar_wait(pv_done, (p_it - 1) & 1, abort_flag, a.c.err, 31)) goto done;
+                    tc_fence_after();
+                }
+                const float m_new = fmaxf(m, mx);
+                if (j == 0) {
+                    m = m_new;
+                } else {
+                    const bool need = (m_new > m + 8.0f);
+                    if (__any_sync(0xffffffffu, need)) {
+                        const float alpha = need ? ex2(m - m_new) : 1.0f;
+                        if (need) { l *= alpha; m = m_new; }
+#pragma unroll
+                        for (int cc = 0; cc < D / 32; ++cc) {
+                            uint32_t orr[32];
+                            tmem_ld32(t_lane + Cfg::kColO + cc * 32, orr);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int x = 0; x < 32; ++x)
+                                orr[x] = __float_as_uint(__uint_as_float(orr[x]) * alpha);
+                            tmem_st32(t_lane + Cfg::kColO + cc * 32, orr);
+                        }
+                        tmem_st_wait();
+                    }
+                }
+                const float mu = (m == -INFINITY) ? 0.f : m;
+                // P = 2^(s - m) -> input dtype -> shared memory (K-major, swizzled)
+                float ls = 0.f;
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) {
+                        const float p0 = ex2(__uint_as_float(sr[cc][2 * x]) - mu);
+                        const float p1 = ex2(__uint_as_float(sr[cc][2 * x + 1]) - mu);
+                        ls += p0 + p1;
+                        pk[x] = pack2<T>(p0, p1);
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int chunk = cc * 4 + q;          // 16-byte chunk over 128 keys
+                        const uint32_t addr = sm_p + (chunk >> 3) * Cfg::kGroupBytes + swz128(row, chunk & 7);
+                        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr),
+                                     "r"(pk[4 * q]), "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]),
+                                     "r"(pk[4 * q + 3]) : "memory");
+                    }
+                }
+                l += ls;
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(p_full);
+                ++p_it;
+            }
+
+            // ---- epilogue: O / l (+ sink), lse ----
+            if (!mbar_wait(o_full, o_it & 1, abort_flag, a.c.err, 32)) goto done;
+            ++o_it;
+            tc_fence_after();
+            const float mu = (m == -INFINITY) ? 0.f : m;
+            float M = mu, lt = l;
+            if (a.c.sink) {
+                const float s2 = a.c.sink[gm.h] * kLog2e;
+                M = fmaxf(mu, s2);
+                lt = l * ex2(mu - M) + ex2(s2 - M);
+            }
+            const float oscale = ex2(mu - M) / lt;
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t orr[32];
+                tmem_ld32(t_lane + Cfg::kColO + cc * 32, orr);
+                tmem_ld_wait();
+                if (valid) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int x = 0; x < 16; ++x)
+                        pk[x] = pack2<T>(__uint_as_float(orr[2 * x]) * oscale,
+                                         __uint_as_float(orr[2 * x + 1]) * oscale);
+                    uint4 *dst = reinterpret_cast<uint4 *>(outp + orow * D + cc * 32);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                }
+            }
+            if (valid && a.c.lse) a.c.lse[orow] = (M + log2f(lt)) * kLn2;
+            tc_fence_before();
+        }
+    }
+done:
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, Cfg::kTmemCols);
+    }
+}
+
+template <typename T, int D>
+static cudaError_t launch_prefill_t(const PrefillArgs &a, const CUtensorMap &tq,
+                                    const CUtensorMap &tk, const CUtensorMap &tv, int grid,
+                                    cudaStream_t s) {
+    auto kern = fia_prefill_kernel<T, D>;
+    const int smem = PrefillCfg<D>::kSmem;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, 192, smem, s>>>(a, tq, tk, tv);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tq, const CUtensorMap &tk,
+                           const CUtensorMap &tv, int q_dtype, int grid, cudaStream_t s) {
+    const bool bf = (q_dtype == 1);
+    if (a.c.D == 128)
+        return bf ? launch_prefill_t<__nv_bfloat16, 128>(a, tq, tk, tv, grid, s)
+                  : launch_prefill_t<__half, 128>(a, tq, tk, tv, grid, s);
+    if (a.c.D == 64)
+        return bf ? launch_prefill_t<__nv_bfloat16, 64>(a, tq, tk, tv, grid, s)
+                  : launch_prefill_t<__half, 64>(a, tq, tk, tv, grid, s);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace fia

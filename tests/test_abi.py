@@ -1,0 +1,136 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/fia.h declares, and phase 1 rejects bad inputs with
+the documented status codes before touching any device (aclnn
+GetWorkspaceSize "implements input parameter verification")."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for f in sorted(os.listdir(inc)):
+        if f.endswith(".h"):
+            src = open(os.path.join(inc, f)).read()
+            names += re.findall(r"FIA_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+    return names
+
+
+def test_library_builds_and_exports_every_declared_symbol():
+    from paged_attention_02_b200 import build
+    build.build()
+    lib = ctypes.CDLL(build.LIB_PATH)
+    names = _declared_functions()
+    assert len(names) >= 6
+    for n in names:
+        assert hasattr(lib, n), "missing export %s" % n
+
+
+def test_status_strings():
+    import paged_attention_02_b200 as fia
+    from paged_attention_02_b200 import _lib
+    for s in range(8):
+        assert fia._lib.fia_status_string(s)
+    assert _lib.fia_status_string(99) == "unknown status"
+
+
+def _call(**kw):
+    """Phase 1 on CPU tensors (only shapes and dtypes are read)."""
+    from paged_attention_02_b200 import _lib, tensor_desc
+    from paged_attention_02_b200._lib import fia_ext
+    B, H, KVH, D, bs = 2, 4, 2, 128, 16
+    t = dict(q=torch.zeros(3, H, D, dtype=torch.bfloat16),
+             k=torch.zeros(8, bs, KVH, D, dtype=torch.bfloat16),
+             v=torch.zeros(8, bs, KVH, D, dtype=torch.bfloat16),
+             bt=torch.zeros(B, 4, dtype=torch.int32),
+             out=torch.zeros(3, H, D, dtype=torch.bfloat16),
+             slopes=None, pse=None, sink=None, lse=None, ks=None, vs=None)
+    args = dict(seq=[1, 2], kv=[20, 33], batch=B, mask=9, H=H, KVH=KVH, scale=0.1)
+    for k, v in kw.items():
+        if k in t:
+            t[k] = v
+        else:
+            args[k] = v
+    d = {k: tensor_desc(v) for k, v in t.items()}
+    P = lambda x: ctypes.pointer(x) if x is not None else None
+    ext = fia_ext(P(d["pse"]), P(d["sink"]), P(d["ks"]), None, P(d["vs"]), None, P(d["lse"]))
+    n = max(len(args["seq"]), 1)
+    sl = (ctypes.c_int32 * n)(*args["seq"])
+    kl = (ctypes.c_int32 * n)(*args["kv"])
+    ws = ctypes.c_uint64(123)
+    op = ctypes.c_void_p()
+    st = _lib.fia_get_workspace_size(P(d["q"]), P(d["k"]), P(d["v"]), P(d["bt"]), sl, kl,
+                                     args["batch"], P(d["slopes"]), args["mask"], args["H"],
+                                     args["KVH"], args["scale"], ctypes.pointer(ext), P(d["out"]),
+                                     ctypes.byref(ws), ctypes.byref(op))
+    if op.value:
+        _lib.fia_op_destroy(op)
+    return st
+
+
+def test_phase1_rejects_bad_inputs():
+    from paged_attention_02_b200 import _lib as L
+    assert _call(H=6, KVH=4) == L.FIA_ERR_PARAM                                   # H % KVH
+    assert _call(mask=5) == L.FIA_ERR_PARAM                                       # mask code
+    assert _call(seq=[2, 2]) == L.FIA_ERR_SHAPE                                   # sum != nTokens
+    assert _call(seq=[1, 2], kv=[20, 1]) == L.FIA_ERR_PARAM                       # seqLen > kvSeqLen
+    assert _call(kv=[20, 80]) == L.FIA_ERR_SHAPE                                  # table too short
+    assert _call(k=torch.zeros(8, 16, 2, 128, dtype=torch.float16),
+                 v=torch.zeros(8, 16, 2, 128, dtype=torch.float16)) == L.FIA_ERR_DTYPE
+    assert _call(out=torch.zeros(3, 4, 128, dtype=torch.float16)) == L.FIA_ERR_DTYPE
+    assert _call(bt=torch.zeros(2, 4, dtype=torch.float32)) == L.FIA_ERR_DTYPE
+    assert _call(v=torch.zeros(9, 16, 2, 128, dtype=torch.bfloat16)) == L.FIA_ERR_SHAPE
+    assert _call(mask=3) == L.FIA_ERR_NULLPTR                                     # ALiBi w/o slopes
+    assert _call(mask=9, slopes=torch.zeros(4)) == L.FIA_ERR_PARAM                # slopes w/o ALiBi
+    assert _call(sink=torch.zeros(3)) == L.FIA_ERR_SHAPE
+    assert _call(lse=torch.zeros(3, 4, dtype=torch.float16)) == L.FIA_ERR_DTYPE
+    assert _call(pse=torch.zeros(2, 4, 2, 16, dtype=torch.bfloat16)) == L.FIA_ERR_SHAPE
+    assert _call(scale=float("nan")) == L.FIA_ERR_PARAM
+    assert _call(batch=-1) == L.FIA_ERR_PARAM
+
+
+def test_phase1_int8_rules():
+    from paged_attention_02_b200 import _lib as L
+    k8 = torch.zeros(8, 16, 2, 128, dtype=torch.int8)
+    assert _call(k=k8, v=k8) == L.FIA_ERR_NULLPTR                                 # scales missing
+    ks = torch.ones(2, 128)
+    # scales on a bf16 cache are a parameter error
+    assert _call(ks=ks, vs=ks) == L.FIA_ERR_PARAM
+    # int8 needs the decode path (seqLen * g <= 16): 9 new tokens x g=2 is too many
+    q = torch.zeros(10, 4, 128, dtype=torch.bfloat16)
+    assert _call(k=k8, v=k8, ks=ks, vs=ks, q=q, out=q.clone(), seq=[1, 9]) == L.FIA_ERR_UNSUPPORTED
+
+
+def test_phase1_build_limits():
+    from paged_attention_02_b200 import _lib as L
+    q = torch.zeros(3, 4, 96, dtype=torch.bfloat16)
+    k = torch.zeros(8, 16, 2, 96, dtype=torch.bfloat16)
+    assert _call(q=q, out=q.clone(), k=k, v=k.clone()) == L.FIA_ERR_UNSUPPORTED   # D=96
+    k = torch.zeros(8, 24, 2, 128, dtype=torch.bfloat16)
+    assert _call(k=k, v=k.clone(), bt=torch.zeros(2, 8, dtype=torch.int32)) == L.FIA_ERR_UNSUPPORTED
+
+
+def test_phase1_without_gpu_reports_cuda_error():
+    from paged_attention_02_b200 import _lib as L
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert _call() == L.FIA_ERR_CUDA
+
+
+def test_empty_query_is_a_noop_op():
+    from paged_attention_02_b200 import _lib as L
+    q = torch.zeros(0, 4, 128, dtype=torch.bfloat16)
+    assert _call(q=q, out=q.clone(), seq=[0, 0], kv=[0, 0]) == L.FIA_OK
+
+
+def test_run_rejects_null_op_and_missing_workspace():
+    from paged_attention_02_b200 import _lib as L
+    assert L.fia_run(None, 0, None, None) == L.FIA_ERR_NULLPTR
+    assert L.fia_op_set_timing_events(None, None, None) == L.FIA_ERR_NULLPTR
+    assert L.fia_op_get_plan_info(None, None) == L.FIA_ERR_NULLPTR

@@ -1,0 +1,222 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.  Tolerances: max |err| <= 2e-2 and mean |err| <= 2e-3 on
+the fp16/bf16 output, |err| <= 5e-3 on the fp32 lse; gather/index work is
+checked bit-exactly (single key, dominant key, block permutation)."""
+import dataclasses
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from fia_testlib import compare, run_gpu, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+# ---------------------------------------------------------------------------
+# Small cases, full comparison.  Sizes span several tiles and a ragged tail.
+# ---------------------------------------------------------------------------
+DECODE_CASES = {
+    "mha_d64_bs16_f16": dict(seq_len=[1, 1, 1], kv_seq_len=[37, 64, 1], head_num=4, kv_head_num=4,
+                             head_size=64, block_size=16, dtype="f16", qk_scale=0.125),
+    "gqa4_bs16_ragged_bf16": dict(seq_len=[1] * 5, kv_seq_len=[1, 15, 129, 700, 1000],
+                                  head_num=16, kv_head_num=4, head_size=128, block_size=16),
+    "gqa8_bs128_bf16": dict(seq_len=[1] * 3, kv_seq_len=[300, 1025, 2049], head_num=32,
+                            kv_head_num=4, head_size=128, block_size=128),
+    "gqa16_bs64_f16_sink": dict(seq_len=[1, 1], kv_seq_len=[513, 77], head_num=16, kv_head_num=1,
+                                head_size=128, block_size=64, dtype="f16", sink=True),
+    "mtp_causal_q3_g4": dict(seq_len=[3, 4, 1], kv_seq_len=[45, 260, 9], head_num=8,
+                             kv_head_num=2, head_size=128, block_size=32, mask_type=W.MASK_CAUSAL),
+    "mtp_alibi_q2_g4": dict(seq_len=[2, 2], kv_seq_len=[100, 333], head_num=8, kv_head_num=2,
+                            head_size=128, block_size=16, mask_type=W.MASK_ALIBI,
+                            alibi_slopes=True, dtype="f16"),
+    "decode_pse": dict(seq_len=[1, 2], kv_seq_len=[90, 200], head_num=4, kv_head_num=2,
+                       head_size=64, block_size=16, mask_type=W.MASK_CAUSAL, pse=True, dtype="f16"),
+    "nan_tail_slots": dict(seq_len=[1, 1], kv_seq_len=[70, 131], head_num=8, kv_head_num=2,
+                           head_size=128, block_size=64, tail_fill=float("nan"), pad_value=-1),
+    "int8_sink_offsets": dict(seq_len=[1, 1, 1], kv_seq_len=[200, 1500, 65], head_num=16,
+                              kv_head_num=2, head_size=128, block_size=128, kv_dtype="i8",
+                              sink=True),
+    "int8_symmetric_f16": dict(seq_len=[1, 1], kv_seq_len=[333, 64], head_num=8, kv_head_num=8,
+                               head_size=128, block_size=32, dtype="f16", kv_dtype="i8",
+                               int8_offsets=False),
+    "int8_mtp_causal": dict(seq_len=[2, 3], kv_seq_len=[50, 700], head_num=8, kv_head_num=2,
+                            head_size=128, block_size=64, kv_dtype="i8",
+                            mask_type=W.MASK_CAUSAL),
+}
+
+PREFILL_CASES = {
+    "causal_gqa_prefix_bs16": dict(seq_len=[37, 130], kv_seq_len=[100, 300], head_num=8,
+                                   kv_head_num=2, head_size=128, block_size=16,
+                                   mask_type=W.MASK_CAUSAL),
+    "causal_bs128_f16": dict(seq_len=[256, 129], kv_seq_len=[256, 400], head_num=4, kv_head_num=4,
+                             head_size=128, block_size=128, dtype="f16", mask_type=W.MASK_CAUSAL),
+    "nomask_d64_bs32": dict(seq_len=[70, 200], kv_seq_len=[70, 333], head_num=4, kv_head_num=2,
+                            head_size=64, block_size=32),
+    "alibi_causal": dict(seq_len=[200, 64], kv_seq_len=[200, 300], head_num=4, kv_head_num=4,
+                         head_size=128, block_size=64, mask_type=W.MASK_ALIBI, alibi_slopes=True,
+                         dtype="f16"),
+    "pse_causal": dict(seq_len=[150, 40], kv_seq_len=[150, 260], head_num=4, kv_head_num=4,
+                       head_size=128, block_size=64, mask_type=W.MASK_CAUSAL, pse=True,
+                       dtype="f16"),
+    "sink_gqa": dict(seq_len=[140, 30], kv_seq_len=[300, 30], head_num=8, kv_head_num=2,
+                     head_size=128, block_size=32, mask_type=W.MASK_CAUSAL, sink=True),
+    "nan_tail_slots_prefill": dict(seq_len=[100, 50], kv_seq_len=[150, 50], head_num=4,
+                                   kv_head_num=1, head_size=128, block_size=64,
+                                   mask_type=W.MASK_CAUSAL, tail_fill=float("nan")),
+    "wide_group_decode_shape": dict(seq_len=[1, 1], kv_seq_len=[300, 129], head_num=32,
+                                    kv_head_num=1, head_size=128, block_size=16),
+}
+
+
+@pytest.mark.parametrize("name", sorted(DECODE_CASES))
+def test_decode_small(name):
+    p = W.make_problem(name=name, seed=zlib.crc32(name.encode()) % 10000, spare_blocks=2, **DECODE_CASES[name])
+    op, out, lse = run_gpu(p)
+    assert op.plan_info()["path"] == 1
+    ref_out, ref_lse = oracle.attention(p)
+    compare(out, lse, ref_out, ref_lse, name)
+
+
+@pytest.mark.parametrize("name", sorted(PREFILL_CASES))
+def test_prefill_small(name):
+    p = W.make_problem(name=name, seed=zlib.crc32(name.encode()) % 10000, spare_blocks=2, **PREFILL_CASES[name])
+    op, out, lse = run_gpu(p)
+    assert op.plan_info()["path"] == 2
+    ref_out, ref_lse = oracle.attention(p)
+    compare(out, lse, ref_out, ref_lse, name)
+
+
+def test_tiny_decode_config():
+    p = W.tiny_decode()
+    _, out, lse = run_gpu(p)
+    ref_out, ref_lse = oracle.attention(p)
+    compare(out, lse, ref_out, ref_lse, "tiny_decode")
+
+
+# ---------------------------------------------------------------------------
+# Bit-exact gather checks through the real kernels.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("kind", ["decode", "prefill"])
+def test_single_key_returns_value_row_bitwise(kind):
+    if kind == "decode":
+        p = W.make_problem(seed=31, seq_len=[1, 1], kv_seq_len=[1, 1], head_num=8, kv_head_num=2,
+                           head_size=128, block_size=16)
+    else:
+        p = W.make_problem(seed=31, seq_len=[1, 1], kv_seq_len=[1, 1], head_num=32,
+                           kv_head_num=1, head_size=128, block_size=16)
+    _, out, _ = run_gpu(p)
+    for b in range(2):
+        blk = int(p.block_tables[b, 0])
+        for h in range(p.head_num):
+            v = p.value_cache[blk, 0, h // (p.head_num // p.kv_head_num)].double().numpy()
+            assert np.array_equal(out[b, h], v)
+
+
+@pytest.mark.parametrize("kind", ["decode", "prefill"])
+def test_dominant_key_bit_exact_gather(kind):
+    """For every logical position t, make key t dominate (score margin > 110)
+    and check the output equals V[t] bit for bit: the block-table resolve
+    reached the right physical row."""
+    kv = 48
+    if kind == "decode":
+        p = W.make_problem(seed=32, seq_len=[1], kv_seq_len=[kv], head_num=4, kv_head_num=1,
+                           head_size=128, block_size=16, dtype="f16", qk_scale=1.0)
+    else:
+        p = W.make_problem(seed=32, seq_len=[1], kv_seq_len=[kv], head_num=32, kv_head_num=1,
+                           head_size=128, block_size=16, dtype="f16", qk_scale=1.0)
+    q = p.query[0, 0].double()
+    qs = p.query.clone()
+    qs[0, :] = p.query[0, 0]              # every head asks the same question
+    for target in range(0, kv, 5):
+        kc = p.key_cache.clone()
+        blk = int(p.block_tables[0, target // 16])
+        kc[blk, target % 16, 0] = (q * 200.0 / float(q.norm() ** 2)).to(torch.float16)
+        pp = dataclasses.replace(p, key_cache=kc, query=qs)
+        _, out, _ = run_gpu(pp)
+        v = p.value_cache[blk, target % 16, 0].double().numpy()
+        for h in range(p.head_num):
+            assert np.array_equal(out[0, h], v), (target, h)
+
+
+@pytest.mark.parametrize("kind", ["decode", "prefill"])
+def test_block_permutation_bitwise_invariant(kind):
+    if kind == "decode":
+        base = dict(seq_len=[1, 1, 1], kv_seq_len=[100, 513, 64], head_num=8, kv_head_num=2,
+                    head_size=128, block_size=16)
+    else:
+        base = dict(seq_len=[70, 128], kv_seq_len=[170, 128], head_num=4, kv_head_num=2,
+                    head_size=128, block_size=16, mask_type=W.MASK_CAUSAL)
+    p = W.make_problem(seed=33, spare_blocks=5, **base)
+    _, out, lse = run_gpu(p)
+    _, out2, lse2 = run_gpu(W.permute_blocks(p, 7))
+    assert np.array_equal(out, out2) and np.array_equal(lse, lse2)
+
+
+@pytest.mark.parametrize("kind", ["decode", "prefill"])
+def test_run_to_run_determinism(kind):
+    if kind == "decode":
+        p = W.make_problem(seed=34, seq_len=[1] * 4, kv_seq_len=[3000, 20, 900, 4097],
+                           head_num=16, kv_head_num=2, head_size=128, block_size=64, sink=True)
+    else:
+        p = W.make_problem(seed=34, seq_len=[300, 20], kv_seq_len=[500, 20], head_num=8,
+                           kv_head_num=2, head_size=128, block_size=64, mask_type=W.MASK_CAUSAL)
+    op, out, lse = run_gpu(p)
+    for _ in range(3):
+        o2, l2 = op.run()
+        torch.cuda.synchronize()
+        assert np.array_equal(o2.float().double().cpu().numpy(), out)
+        assert np.array_equal(l2.double().cpu().numpy(), lse)
+
+
+def test_empty_kv_rows_and_empty_query():
+    p = W.make_problem(seed=35, seq_len=[1, 1], kv_seq_len=[0, 40], head_num=4, kv_head_num=2,
+                       head_size=128, block_size=16)
+    _, out, lse = run_gpu(p)
+    assert np.all(out[0] == 0) and np.all(np.isposinf(lse[0]))
+    ref_out, ref_lse = oracle.attention(p)
+    compare(out, lse, ref_out, ref_lse, "empty_kv")
+    e = W.make_problem(seed=35, seq_len=[0, 0], kv_seq_len=[0, 0], head_num=4, kv_head_num=2,
+                       head_size=128, block_size=16)
+    op, out, _ = run_gpu(e)
+    assert op.plan_info()["path"] == 0 and out.size == 0
+
+
+# ---------------------------------------------------------------------------
+# The five named workloads at full size: sampled rows against the oracle.
+# ---------------------------------------------------------------------------
+def _full_size(p, n_rows, seed):
+    op, out, lse = run_gpu(p)
+    rows = sample_rows(p, n_rows, seed)
+    ref_o, ref_l = oracle.attention(p, rows=rows)
+    got_o = np.stack([out[t, h] for t, h in rows])
+    got_l = np.array([lse[t, h] for t, h in rows])
+    compare(got_o, got_l, ref_o, ref_l, p.name)
+    return op, out, lse
+
+
+def test_config_prefill_prefix_full():
+    _full_size(W.prefill_prefix(), 384, 1)
+
+
+def test_config_decode_large_batch_full():
+    p = W.decode_large_batch()
+    op, out, lse = _full_size(p, 512, 2)
+    assert op.plan_info()["path"] == 1
+
+
+def test_config_alibi_prefill_and_pse_agree():
+    a = W.alibi_prefill(False)
+    _, oa, la = _full_size(a, 256, 3)
+    b = W.alibi_prefill(True)
+    _, ob, lb = _full_size(b, 256, 3)
+    # same bias in two forms: slope generated in registers vs fp16 pse tensor
+    assert float(np.abs(oa - ob).max()) <= 2e-2
+
+
+def test_config_int8_long_decode_full():
+    p = W.int8_long_decode()
+    _full_size(p, 256, 4)
