@@ -118,6 +118,22 @@ class FiaOp:
             return 0
         return int(self.workspace[off:off + 4].view(torch.int32).item())
 
+    def error_trail(self) -> list:
+        """Records the kernels left when a bounded wait ran out (syncs the device):
+        dicts with the wait site, block, thread, three site values and the
+        barrier's raw state."""
+        if self.workspace_size == 0:
+            return []
+        off = self.plan_info()["error_word_offset"]
+        words = self.workspace[off:off + (4 + 8 * 31) * 4].view(torch.int32).cpu().tolist()
+        n = min(words[1] & 0xffffffff, 31)
+        out = []
+        for k in range(n):
+            r = [w & 0xffffffff for w in words[4 + 8 * k: 12 + 8 * k]]
+            out.append(dict(where=r[0], block=r[1], thread=r[2], x0=r[3], x1=r[4], x2=r[5],
+                            bar=(r[7] << 32) | r[6]))
+        return out
+
     def set_timing_events(self, start: Optional[torch.cuda.Event], stop: Optional[torch.cuda.Event]):
         """Have run() record ``start``/``stop`` around its kernels only."""
         if start is None:

@@ -215,6 +215,7 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
     for (int j = 0; j < n_tiles; ++j) {
         const int s = j % STAGES;
         if (!mbar_wait(&full[s], (j / STAGES) & 1, abort_flag, a.c.err, 1)) { ok = false; break; }
+        __syncwarp();      // ldmatrix / mma.sync below are warp-collective (.aligned)
         const uint32_t kst = smem_u32(smem + s * Cfg::kStageBytes);
         const uint32_t vst = kst + Cfg::kTileBytes;
         const int tw = u.t_begin + j * kDecodeTile + warp * 16;   // first key of this warp
@@ -363,6 +364,7 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
             if (!mbar_wait(&empty[s], (j / STAGES) & 1, abort_flag, a.c.err, 2)) { ok = false; break; }
             issue(j + STAGES);
         }
+        __syncwarp();
     }
     (void)ok;
 

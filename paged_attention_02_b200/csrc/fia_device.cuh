@@ -83,6 +83,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// Error region layout (uint32 words): [0] error word, [1] trail count,
+// [4 + 8k .. 4 + 8k + 7] trail record k (k < kTrailMax): where, block, thread,
+// three caller values, the waited barrier's raw 64-bit state.
+constexpr uint32_t kTrailMax = 31;
+constexpr uint32_t kErrRegionBytes = (4 + 8 * kTrailMax) * 4;
+
+static __device__ __noinline__ void fail_trail(uint32_t *err, uint32_t where, uint32_t x0, uint32_t x1,
+                                        uint32_t x2, const uint64_t *bar) {
+    if (!err) return;
+    const uint32_t k = atomicAdd(err + 1, 1u);
+    if (k >= kTrailMax) return;
+    uint64_t st = 0;
+    if (bar) asm volatile("ld.shared.b64 %0, [%1];" : "=l"(st) : "r"(smem_u32(bar)));
+    uint32_t *r = err + 4 + 8 * k;
+    r[0] = where; r[1] = blockIdx.x; r[2] = threadIdx.x;
+    r[3] = x0; r[4] = x1; r[5] = x2;
+    r[6] = (uint32_t)st; r[7] = (uint32_t)(st >> 32);
+}
+
 // ---------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), no multicast.
 // ---------------------------------------------------------------------------
@@ -136,6 +155,17 @@ __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64
                  : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem], kind::f16, one CTA.  A is 128 lanes (rows)
+// x K 16-bit elements packed two per 32-bit column.
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+                 ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+
 // Arrive (once) on `bar` when every tcgen05 op this thread issued so far is done.
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -170,8 +200,34 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+          "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
+          "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// tcgen05.ld writes its destination registers asynchronously; they are only
+// defined after tcgen05.wait::ld.  The compiler does not know that, so after
+// the wait every loaded register is passed through an empty volatile asm:
+// no use of it can then be scheduled above the wait.
+__device__ __forceinline__ void reg_fence32(uint32_t (&r)[32]) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                   "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                   "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                   "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");

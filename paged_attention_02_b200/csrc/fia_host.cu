@@ -27,6 +27,7 @@
 #include <vector>
 
 #include "../../include/fia.h"
+#include "fia_device.cuh"
 #include "fia_plan.h"
 
 using namespace fia;
@@ -335,7 +336,7 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
     o->off_seq = off;
     off = align_up(off + sizeof(SeqInfo) * std::max(batch, 1), 256);
     o->off_err = off;
-    off = align_up(off + 16, 256);
+    off = align_up(off + kErrRegionBytes, 256);
     std::vector<uint8_t> host;
     if (decode) {
         o->path = 1;

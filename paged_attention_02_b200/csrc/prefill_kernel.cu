@@ -40,13 +40,15 @@ struct PrefillCfg {
     static constexpr int kHalves = D / 64;                 // 128-byte column groups
     static constexpr int kTileBytes = 128 * D * 2;         // Q, K or V tile (128 rows)
     static constexpr int kGroupBytes = 128 * 128;          // one 128-row x 128-byte group
-    static constexpr int kStages = 2;
+    static constexpr int kKStages = 3;
+    static constexpr int kVStages = 3;
     static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + kTileBytes;       // K[s] = kOffK + s * 2 * kTileBytes
-    static constexpr int kOffP = kOffK + kStages * 2 * kTileBytes;
-    static constexpr int kPBytes = 128 * 128 * 2;
-    static constexpr int kOffBar = kOffP + kPBytes;
-    static constexpr int kNumBar = 14;
+    static constexpr int kOffK = kOffQ + kTileBytes;                   // K[s]
+    static constexpr int kOffV = kOffK + kKStages * kTileBytes;        // V[s]
+    static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
+    // q_full, q_empty, k_full[3], k_empty[3], v_full[3], v_empty[3],
+    // s_full[2], s_empty[2], p_full, pv_done, o_full
+    static constexpr int kNumBar = 2 + 4 * 3 + 4 + 3;
     static constexpr int kUsed = kOffBar + kNumBar * 8 + 16;
     // Keep one CTA per SM (each CTA holds all 512 TMEM columns).
     static constexpr int kSmem = 1024 + (kUsed > 118 * 1024 ? kUsed : 118 * 1024);
@@ -78,11 +80,23 @@ __device__ __forceinline__ ItemGeom item_geom(const PrefillArgs &a, int idx) {
     return g;
 }
 
+// Bounded wait; on failure lane 0 leaves a trail record (item, tile, parity).
+#define FIA_WAIT(bar, parity, where)                                                      \
+    do {                                                                                  \
+        const uint32_t _par = (parity);                                                   \
+        if (!mbar_wait((bar), _par, abort_flag, a.c.err, (where))) {                      \
+            if (lane == 0) fail_trail(a.c.err, (where), (uint32_t)idx, (uint32_t)dbg_j,   \
+                                      _par, (bar));                                       \
+            goto done;                                                                    \
+        }                                                                                 \
+    } while (0)
+
 template <typename T, int D>
 __global__ void __launch_bounds__(192, 1)
 fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tq,
                    const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
     using Cfg = PrefillCfg<D>;
+    constexpr int KS = Cfg::kKStages, VS = Cfg::kVStages;
     constexpr bool BF = MmaType<T>::bf16;
     constexpr uint32_t IDESC_QK = umma_idesc_f16(BF, false, false, 128, kPrefillBN);
     constexpr uint32_t IDESC_PV = umma_idesc_f16(BF, false, true, 128, D);
@@ -93,19 +107,17 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
     uint64_t *q_full = bars + 0;
     uint64_t *q_empty = bars + 1;
-    uint64_t *k_full = bars + 2;      // [2]
-    uint64_t *v_full = bars + 4;      // [2]
-    uint64_t *kv_empty = bars + 6;    // [2]
-    uint64_t *s_full = bars + 8;      // [2]
-    uint64_t *s_empty = bars + 10;    // [2]
-    uint64_t *p_full = bars + 12;
-    uint64_t *pv_done = bars + 13;
+    uint64_t *k_full = bars + 2;            // [KS]
+    uint64_t *k_empty = k_full + KS;        // [KS]
+    uint64_t *v_full = k_empty + KS;        // [VS]
+    uint64_t *v_empty = v_full + VS;        // [VS]
+    uint64_t *s_full = v_empty + VS;        // [2]
+    uint64_t *s_empty = s_full + 2;         // [2]  (released by the PV that read P from it)
+    uint64_t *p_full = s_empty + 2;
+    uint64_t *pv_done = p_full + 1;
+    uint64_t *o_full = pv_done + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + Cfg::kNumBar);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    // o_full shares the pv_done phase sequence: a separate barrier keeps the
-    // epilogue wait independent of the per-tile waits.
-    __shared__ uint64_t o_full_bar;
-    uint64_t *o_full = &o_full_bar;
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -114,13 +126,9 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     if (tid == 0) {
         mbar_init(q_full, 1);
         mbar_init(q_empty, 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&k_full[s], 1);
-            mbar_init(&v_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
-            mbar_init(&s_full[s], 1);
-            mbar_init(&s_empty[s], 4);
-        }
+        for (int s = 0; s < KS; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
+        for (int s = 0; s < VS; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
+        for (int s = 0; s < 2; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], 1); }
         mbar_init(p_full, 4);
         mbar_init(pv_done, 1);
         mbar_init(o_full, 1);
@@ -138,12 +146,13 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    int dbg_j = -1;     // tile index recorded in failure trails
 
     const int it_begin = a.cta_off[blockIdx.x];
     const int it_end = a.cta_off[blockIdx.x + 1];
     const uint32_t sm_q = smem_u32(smem + Cfg::kOffQ);
     const uint32_t sm_k0 = smem_u32(smem + Cfg::kOffK);
-    const uint32_t sm_p = smem_u32(smem + Cfg::kOffP);
+    const uint32_t sm_v0 = smem_u32(smem + Cfg::kOffV);
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -153,7 +162,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             for (int idx = it_begin; idx < it_end; ++idx) {
                 const ItemGeom gm = item_geom(a, idx);
                 if (gm.n == 0) continue;
-                if (!mbar_wait(q_empty, (q_it & 1) ^ 1, abort_flag, a.c.err, 10)) goto done;
+                FIA_WAIT(q_empty, (q_it & 1) ^ 1, 10);
                 mbar_arrive_expect_tx(q_full, Cfg::kTileBytes);
                 for (int hv = 0; hv < Cfg::kHalves; ++hv)
                     tma_load_3d(smem + Cfg::kOffQ + hv * Cfg::kGroupBytes, &tq, q_full, hv * 64,
@@ -161,29 +170,30 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 ++q_it;
                 const int32_t *bt_row = a.c.bt + (int64_t)gm.b * a.c.bt_stride;
                 for (int j = 0; j < gm.n; ++j, ++kv_it) {
-                    const int st = kv_it & 1;
-                    if (!mbar_wait(&kv_empty[st], ((kv_it >> 1) & 1) ^ 1, abort_flag, a.c.err, 11))
-                        goto done;
+                    dbg_j = j;
                     const int t0 = j * kPrefillBN;
                     const int t1 = min(t0 + kPrefillBN, gm.kvlen);
                     const int nbox = (t1 - t0 + br - 1) / br;
                     const uint32_t bytes = (uint32_t)(nbox * br * 128 * Cfg::kHalves);
-                    uint8_t *ks = smem + Cfg::kOffK + st * 2 * Cfg::kTileBytes;
-                    uint8_t *vs = ks + Cfg::kTileBytes;
-                    mbar_arrive_expect_tx(&k_full[st], bytes);
+                    const int ks = kv_it % KS, vs = kv_it % VS;
+                    FIA_WAIT(&k_empty[ks], ((kv_it / KS) & 1) ^ 1, 11);
+                    uint8_t *kd = smem + Cfg::kOffK + ks * Cfg::kTileBytes;
+                    mbar_arrive_expect_tx(&k_full[ks], bytes);
                     for (int bi = 0; bi < nbox; ++bi) {
                         const int t = t0 + bi * br;
                         const int prow = bt_row[t / a.c.bs] * a.c.bs + (t % a.c.bs);
                         for (int hv = 0; hv < Cfg::kHalves; ++hv)
-                            tma_load_3d(ks + hv * Cfg::kGroupBytes + bi * br * 128, &tk, &k_full[st],
+                            tma_load_3d(kd + hv * Cfg::kGroupBytes + bi * br * 128, &tk, &k_full[ks],
                                         hv * 64, gm.kvh, prow);
                     }
-                    mbar_arrive_expect_tx(&v_full[st], bytes);
+                    FIA_WAIT(&v_empty[vs], ((kv_it / VS) & 1) ^ 1, 12);
+                    uint8_t *vd = smem + Cfg::kOffV + vs * Cfg::kTileBytes;
+                    mbar_arrive_expect_tx(&v_full[vs], bytes);
                     for (int bi = 0; bi < nbox; ++bi) {
                         const int t = t0 + bi * br;
                         const int prow = bt_row[t / a.c.bs] * a.c.bs + (t % a.c.bs);
                         for (int hv = 0; hv < Cfg::kHalves; ++hv)
-                            tma_load_3d(vs + hv * Cfg::kGroupBytes + bi * br * 128, &tv, &v_full[st],
+                            tma_load_3d(vd + hv * Cfg::kGroupBytes + bi * br * 128, &tv, &v_full[vs],
                                         hv * 64, gm.kvh, prow);
                     }
                 }
@@ -195,21 +205,23 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         for (int idx = it_begin; idx < it_end; ++idx) {
             const ItemGeom gm = item_geom(a, idx);
             if (gm.n == 0) continue;
-            if (!mbar_wait(q_full, q_it & 1, abort_flag, a.c.err, 20)) goto done;
+            FIA_WAIT(q_full, q_it & 1, 20);
             ++q_it;
             const uint32_t kv_base = kv_it;
+            const uint32_t s_base = s_it;
             for (int j = 0; j <= gm.n; ++j) {
+                dbg_j = j;
                 if (j < gm.n) {
-                    // S_j = Q K_j^T
+                    // S_j = Q K_j^T  into TMEM buffer j % 2
                     const uint32_t kvi = kv_base + j;
-                    const int st = kvi & 1;
-                    if (!mbar_wait(&k_full[st], (kvi >> 1) & 1, abort_flag, a.c.err, 21)) goto done;
+                    const int ks = kvi % KS;
+                    FIA_WAIT(&k_full[ks], (kvi / KS) & 1, 21);
                     const int sb = s_it & 1;
-                    if (!mbar_wait(&s_empty[sb], ((s_it >> 1) & 1) ^ 1, abort_flag, a.c.err, 22))
-                        goto done;
+                    FIA_WAIT(&s_empty[sb], ((s_it >> 1) & 1) ^ 1, 22);
+                    __syncwarp();
                     tc_fence_after();
                     if (lane == 0) {
-                        const uint32_t kbase = sm_k0 + st * 2 * Cfg::kTileBytes;
+                        const uint32_t kbase = sm_k0 + ks * Cfg::kTileBytes;
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const uint32_t off = (kk >> 2) * Cfg::kGroupBytes + (kk & 3) * 32;
@@ -218,27 +230,30 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                                     umma_desc_sw128(kbase + off, 16, 1024), IDESC_QK, kk > 0);
                         }
                         umma_commit(&s_full[sb]);
+                        umma_commit(&k_empty[ks]);
                         if (j == gm.n - 1) umma_commit(q_empty);
                     }
                     __syncwarp();
                     ++s_it;
                 }
                 if (j >= 1) {
-                    // O += P_{j-1} V_{j-1}
+                    // O += P_{j-1} V_{j-1}; P is in TMEM (aliasing S buffer (j-1) % 2)
                     const int jj = j - 1;
                     const uint32_t kvi = kv_base + jj;
-                    const int st = kvi & 1;
-                    if (!mbar_wait(p_full, p_it & 1, abort_flag, a.c.err, 23)) goto done;
-                    if (!mbar_wait(&v_full[st], (kvi >> 1) & 1, abort_flag, a.c.err, 24)) goto done;
-                    const uint32_t vbase = sm_k0 + st * 2 * Cfg::kTileBytes + Cfg::kTileBytes;
+                    const int vs = kvi % VS;
+                    const int sb = (s_base + jj) & 1;
+                    FIA_WAIT(p_full, p_it & 1, 23);
+                    FIA_WAIT(&v_full[vs], (kvi / VS) & 1, 24);
+                    __syncwarp();
+                    const uint32_t vbase = sm_v0 + vs * Cfg::kTileBytes;
                     const int valid = gm.kvlen - jj * kPrefillBN;
                     if (valid < kPrefillBN) {
                         // rows past kvSeqLen: P is 0 there, but the slots may
                         // hold anything (NaN * 0 = NaN in the MMA) -> zero them.
-                        uint8_t *vs = smem + Cfg::kOffK + st * 2 * Cfg::kTileBytes + Cfg::kTileBytes;
+                        uint8_t *vd = smem + Cfg::kOffV + vs * Cfg::kTileBytes;
                         const int nbytes = (kPrefillBN - valid) * 128;
                         for (int hv = 0; hv < Cfg::kHalves; ++hv) {
-                            uint4 *p = reinterpret_cast<uint4 *>(vs + hv * Cfg::kGroupBytes + valid * 128);
+                            uint4 *p = reinterpret_cast<uint4 *>(vd + hv * Cfg::kGroupBytes + valid * 128);
                             for (int x = lane; x < nbytes / 16; x += 32) p[x] = make_uint4(0, 0, 0, 0);
                         }
                         fence_proxy_async_smem();
@@ -246,15 +261,16 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                     }
                     tc_fence_after();
                     if (lane == 0) {
+                        const uint32_t pcol = tmem + (sb ? Cfg::kColS1 : Cfg::kColS0);
 #pragma unroll
                         for (int kk = 0; kk < kPrefillBN / 16; ++kk) {
-                            const uint32_t poff = (kk >> 2) * Cfg::kGroupBytes + (kk & 3) * 32;
-                            umma_ss(tmem + Cfg::kColO, umma_desc_sw128(sm_p + poff, 16, 1024),
+                            umma_ts(tmem + Cfg::kColO, pcol + kk * 8,
                                     umma_desc_sw128(vbase + kk * 2048, Cfg::kGroupBytes, 1024),
                                     IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
                         }
                         umma_commit(pv_done);
-                        umma_commit(&kv_empty[st]);
+                        umma_commit(&v_empty[vs]);
+                        umma_commit(&s_empty[sb]);
                         if (jj == gm.n - 1) umma_commit(o_full);
                     }
                     __syncwarp();
@@ -285,6 +301,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                     for (int x = 0; x < D * 2 / 16; ++x) dst[x] = make_uint4(0, 0, 0, 0);
                     if (a.c.lse) a.c.lse[orow] = INFINITY;
                 }
+                __syncwarp();
                 continue;
             }
             const float slope2 = alibi ? a.c.slopes[gm.h] * kLog2e : 0.f;
@@ -294,17 +311,18 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                           (((int64_t)gm.b * a.c.H + gm.h) * a.c.pse_q + i) * a.c.pse_kv;
             float m = -INFINITY, l = 0.f;
             for (int j = 0; j < gm.n; ++j) {
+                dbg_j = j;
                 const int sb = s_it & 1;
-                if (!mbar_wait(&s_full[sb], (s_it >> 1) & 1, abort_flag, a.c.err, 30)) goto done;
+                const uint32_t scol = t_lane + (sb ? Cfg::kColS1 : Cfg::kColS0);
+                FIA_WAIT(&s_full[sb], (s_it >> 1) & 1, 30);
+                __syncwarp();          // tcgen05.ld/st below are warp-collective (.aligned)
                 tc_fence_after();
                 uint32_t sr[4][32];
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc)
-                    tmem_ld32(t_lane + (sb ? Cfg::kColS1 : Cfg::kColS0) + cc * 32, sr[cc]);
+                for (int cc = 0; cc < 4; ++cc) tmem_ld32(scol + cc * 32, sr[cc]);
                 tmem_ld_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s_empty[sb]);
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) reg_fence32(sr[cc]);
                 ++s_it;
 
                 // scores in log2 units, masks, bias
@@ -352,39 +370,28 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                         }
                     }
                 }
+                __syncwarp();          // reconverge after the per-row pse loads
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
                     for (int x = 0; x < 32; ++x) mx = fmaxf(mx, __uint_as_float(sr[cc][x]));
 
-                // the previous PV must be complete before O or P is touched
-                if (j > 0) {
-                    if (!mbar_wait(pv_done, (p_it - 1) & 1, abort_flag, a.c.err, 31)) goto done;
-                    tc_fence_after();
-                }
+                // running max: exact on the first tile, afterwards raised only
+                // when it grows by more than 2^8 (O and l stay consistent with m)
                 const float m_new = fmaxf(m, mx);
+                bool need = false;
+                float alpha = 1.0f;
                 if (j == 0) {
                     m = m_new;
-                } else {
-                    const bool need = (m_new > m + 8.0f);
-                    if (__any_sync(0xffffffffu, need)) {
-                        const float alpha = need ? ex2(m - m_new) : 1.0f;
-                        if (need) { l *= alpha; m = m_new; }
-#pragma unroll
-                        for (int cc = 0; cc < D / 32; ++cc) {
-                            uint32_t orr[32];
-                            tmem_ld32(t_lane + Cfg::kColO + cc * 32, orr);
-                            tmem_ld_wait();
-#pragma unroll
-                            for (int x = 0; x < 32; ++x)
-                                orr[x] = __float_as_uint(__uint_as_float(orr[x]) * alpha);
-                            tmem_st32(t_lane + Cfg::kColO + cc * 32, orr);
-                        }
-                        tmem_st_wait();
-                    }
+                } else if (m_new > m + 8.0f) {
+                    need = true;
+                    alpha = ex2(m - m_new);
+                    m = m_new;
+                    l *= alpha;
                 }
                 const float mu = (m == -INFINITY) ? 0.f : m;
-                // P = 2^(s - m) -> input dtype -> shared memory (K-major, swizzled)
+
+                // P = 2^(s - m) in the input dtype, stored over S's first 64 columns
                 float ls = 0.f;
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
@@ -396,17 +403,35 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                         ls += p0 + p1;
                         pk[x] = pack2<T>(p0, p1);
                     }
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int chunk = cc * 4 + q;          // 16-byte chunk over 128 keys
-                        const uint32_t addr = sm_p + (chunk >> 3) * Cfg::kGroupBytes + swz128(row, chunk & 7);
-                        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr),
-                                     "r"(pk[4 * q]), "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]),
-                                     "r"(pk[4 * q + 3]) : "memory");
-                    }
+                    tmem_st16(scol + cc * 16, pk);
                 }
                 l += ls;
-                fence_proxy_async_smem();
+
+                // The previous PV must be complete before this warp signals P_j:
+                // (1) O may be rescaled below; (2) it keeps every softmax warp
+                // within one tile of the others, so the 4 arrivals that complete
+                // a p_full phase always belong to the same tile, and pv_done can
+                // never run two phases ahead of this parity wait.
+                if (j > 0) {
+                    FIA_WAIT(pv_done, (p_it - 1) & 1, 31);
+                    __syncwarp();
+                    tc_fence_after();
+                }
+                // rescale O (rare)
+                if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t orr[32];
+                        tmem_ld32(t_lane + Cfg::kColO + cc * 32, orr);
+                        tmem_ld_wait();
+                        reg_fence32(orr);
+#pragma unroll
+                        for (int x = 0; x < 32; ++x)
+                            orr[x] = __float_as_uint(__uint_as_float(orr[x]) * alpha);
+                        tmem_st32(t_lane + Cfg::kColO + cc * 32, orr);
+                    }
+                }
+                tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(p_full);
@@ -414,8 +439,10 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             }
 
             // ---- epilogue: O / l (+ sink), lse ----
-            if (!mbar_wait(o_full, o_it & 1, abort_flag, a.c.err, 32)) goto done;
+            dbg_j = gm.n;
+            FIA_WAIT(o_full, o_it & 1, 32);
             ++o_it;
+            __syncwarp();
             tc_fence_after();
             const float mu = (m == -INFINITY) ? 0.f : m;
             float M = mu, lt = l;
@@ -430,6 +457,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 uint32_t orr[32];
                 tmem_ld32(t_lane + Cfg::kColO + cc * 32, orr);
                 tmem_ld_wait();
+                reg_fence32(orr);
                 if (valid) {
                     uint32_t pk[16];
 #pragma unroll
@@ -441,9 +469,11 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                     for (int q = 0; q < 4; ++q)
                         dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
                 }
+                __syncwarp();
             }
             if (valid && a.c.lse) a.c.lse[orow] = (M + log2f(lt)) * kLn2;
             tc_fence_before();
+            __syncwarp();
         }
     }
 done:

@@ -24,7 +24,8 @@ def run_gpu(p, device="cuda", **overrides):
                    p.kv_head_num, p.qk_scale, **kw)
     out, lse = op.run()
     torch.cuda.synchronize()
-    assert op.error_word() == 0, "kernel error word set: %#x" % op.error_word()
+    ew = op.error_word()
+    assert ew == 0, "kernel error word set: %#x, trail %s" % (ew, op.error_trail())
     o = out.float().double().cpu().numpy()
     l = lse.double().cpu().numpy() if lse is not None else None
     return op, o, l
