@@ -91,7 +91,9 @@ __device__ __forceinline__ ItemGeom item_geom(const PrefillArgs &a, int idx) {
         }                                                                                 \
     } while (0)
 
-template <typename T, int D>
+enum { kModePlain = 0, kModeAlibi = 1, kModePse = 2 };
+
+template <typename T, int D, int MODE>
 __global__ void __launch_bounds__(192, 1)
 fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tq,
                    const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
@@ -285,8 +287,10 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         const int row = quad * 32 + lane;
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
         const bool causal = (a.c.mask_type == 9 || a.c.mask_type == 3);
-        const bool alibi = (a.c.mask_type == 3);
         const float sl2 = a.c.scale_log2;
+        // plain mode with a positive scale: mask raw scores and fold the scale
+        // into the exponent (one FFMA per element)
+        const bool fold = (MODE == kModePlain) && (sl2 > 0.f);
         uint32_t s_it = 0, p_it = 0, o_it = 0;
         T *outp = reinterpret_cast<T *>(a.c.out);
         for (int idx = it_begin; idx < it_end; ++idx) {
@@ -304,16 +308,20 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 __syncwarp();
                 continue;
             }
-            const float slope2 = alibi ? a.c.slopes[gm.h] * kLog2e : 0.f;
+            float slope2 = 0.f;
+            if constexpr (MODE == kModeAlibi) slope2 = a.c.slopes[gm.h] * kLog2e;
             const T *pse_row = nullptr;
-            if (a.c.pse && valid)
+            if constexpr (MODE == kModePse) {
+                // rows past seqLen read row 0 of the sequence (their output is dropped)
                 pse_row = reinterpret_cast<const T *>(a.c.pse) +
-                          (((int64_t)gm.b * a.c.H + gm.h) * a.c.pse_q + i) * a.c.pse_kv;
+                          (((int64_t)gm.b * a.c.H + gm.h) * a.c.pse_q + (valid ? i : 0)) * a.c.pse_kv;
+            }
             float m = -INFINITY, l = 0.f;
             for (int j = 0; j < gm.n; ++j) {
                 dbg_j = j;
                 const int sb = s_it & 1;
                 const uint32_t scol = t_lane + (sb ? Cfg::kColS1 : Cfg::kColS0);
+                const int tb = j * kPrefillBN;
                 FIA_WAIT(&s_full[sb], (s_it >> 1) & 1, 30);
                 __syncwarp();          // tcgen05.ld/st below are warp-collective (.aligned)
                 tc_fence_after();
@@ -325,56 +333,68 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 for (int cc = 0; cc < 4; ++cc) reg_fence32(sr[cc]);
                 ++s_it;
 
-                // scores in log2 units, masks, bias
-                const int tb = j * kPrefillBN;
+                // ---- scores (log2 units unless folded), bias, masks ----
                 const bool edge = (tb + kPrefillBN > gm.kvlen) || (causal && tb + kPrefillBN - 1 > qpos);
-                float mx = -INFINITY;
+                if constexpr (MODE == kModeAlibi) {
+                    const float base = slope2 * (float)(tb - qpos);
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
+                    for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) {
-                        const int t = tb + cc * 32 + x;
-                        float v = __uint_as_float(sr[cc][x]) * sl2;
-                        if (alibi) v = fmaf(slope2, (float)(t - qpos), v);
-                        if (edge) {
-                            const bool keep = (t < gm.kvlen) && !(causal && t > qpos);
-                            v = keep ? v : -INFINITY;
+                        for (int x = 0; x < 32; ++x) {
+                            const float bias = fmaf(slope2, (float)(cc * 32 + x), base);
+                            sr[cc][x] = __float_as_uint(fmaf(__uint_as_float(sr[cc][x]), sl2, bias));
                         }
-                        sr[cc][x] = __float_as_uint(v);
-                    }
-                }
-                if (pse_row) {
+                } else if constexpr (MODE == kModePse) {
 #pragma unroll
                     for (int cc = 0; cc < 4; ++cc) {
 #pragma unroll
                         for (int x8 = 0; x8 < 4; ++x8) {
                             const int t = tb + cc * 32 + x8 * 8;
+                            T pv[8];
                             if (a.c.pse_vec && t + 8 <= gm.kvlen) {
-                                const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(pse_row + t));
-                                const T *pv = reinterpret_cast<const T *>(&raw);
-#pragma unroll
-                                for (int e = 0; e < 8; ++e) {
-                                    float v = __uint_as_float(sr[cc][x8 * 8 + e]);
-                                    sr[cc][x8 * 8 + e] = __float_as_uint(fmaf(to_f32<T>(pv[e]), kLog2e, v));
-                                }
+                                *reinterpret_cast<uint4 *>(pv) =
+                                    __ldg(reinterpret_cast<const uint4 *>(pse_row + t));
                             } else {
 #pragma unroll
-                                for (int e = 0; e < 8; ++e) {
-                                    if (t + e < gm.kvlen) {
-                                        float v = __uint_as_float(sr[cc][x8 * 8 + e]);
-                                        sr[cc][x8 * 8 + e] =
-                                            __float_as_uint(fmaf(to_f32<T>(pse_row[t + e]), kLog2e, v));
-                                    }
-                                }
+                                for (int e = 0; e < 8; ++e)
+                                    pv[e] = (t + e < gm.kvlen) ? pse_row[t + e] : pv[0];
+                            }
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const float bias = to_f32<T>(pv[e]) * kLog2e;
+                                sr[cc][x8 * 8 + e] = __float_as_uint(
+                                    fmaf(__uint_as_float(sr[cc][x8 * 8 + e]), sl2, bias));
                             }
                         }
                     }
+                    __syncwarp();      // reconverge after the per-row pse loads
+                } else if (!fold) {
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+                        for (int x = 0; x < 32; ++x)
+                            sr[cc][x] = __float_as_uint(__uint_as_float(sr[cc][x]) * sl2);
                 }
-                __syncwarp();          // reconverge after the per-row pse loads
+                if (edge) {
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc)
+                    for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) mx = fmaxf(mx, __uint_as_float(sr[cc][x]));
+                        for (int x = 0; x < 32; ++x) {
+                            const int t = tb + cc * 32 + x;
+                            const bool keep = (t < gm.kvlen) && !(causal && t > qpos);
+                            if (!keep) sr[cc][x] = __float_as_uint(-INFINITY);
+                        }
+                }
+                // tree max (8 independent chains)
+                float mx8[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) mx8[k] = __uint_as_float(sr[0][k]);
+#pragma unroll
+                for (int e = 8; e < 128; ++e)
+                    mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(sr[e >> 5][e & 31]));
+                float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+                if (fold) mx = (mx == -INFINITY) ? -INFINITY : mx * sl2;
 
                 // running max: exact on the first tile, afterwards raised only
                 // when it grows by more than 2^8 (O and l stay consistent with m)
@@ -392,20 +412,29 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 const float mu = (m == -INFINITY) ? 0.f : m;
 
                 // P = 2^(s - m) in the input dtype, stored over S's first 64 columns
-                float ls = 0.f;
+                float ls8[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) ls8[k] = 0.f;
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int x = 0; x < 16; ++x) {
-                        const float p0 = ex2(__uint_as_float(sr[cc][2 * x]) - mu);
-                        const float p1 = ex2(__uint_as_float(sr[cc][2 * x + 1]) - mu);
-                        ls += p0 + p1;
+                        float p0, p1;
+                        if (fold) {
+                            p0 = ex2(fmaf(__uint_as_float(sr[cc][2 * x]), sl2, -mu));
+                            p1 = ex2(fmaf(__uint_as_float(sr[cc][2 * x + 1]), sl2, -mu));
+                        } else {
+                            p0 = ex2(__uint_as_float(sr[cc][2 * x]) - mu);
+                            p1 = ex2(__uint_as_float(sr[cc][2 * x + 1]) - mu);
+                        }
+                        ls8[(2 * x) & 7] += p0;
+                        ls8[(2 * x + 1) & 7] += p1;
                         pk[x] = pack2<T>(p0, p1);
                     }
                     tmem_st16(scol + cc * 16, pk);
                 }
-                l += ls;
+                l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
 
                 // The previous PV must be complete before this warp signals P_j:
                 // (1) O may be rescaled below; (2) it keeps every softmax warp
@@ -485,11 +514,11 @@ done:
     }
 }
 
-template <typename T, int D>
+template <typename T, int D, int MODE>
 static cudaError_t launch_prefill_t(const PrefillArgs &a, const CUtensorMap &tq,
                                     const CUtensorMap &tk, const CUtensorMap &tv, int grid,
                                     cudaStream_t s) {
-    auto kern = fia_prefill_kernel<T, D>;
+    auto kern = fia_prefill_kernel<T, D, MODE>;
     const int smem = PrefillCfg<D>::kSmem;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -497,15 +526,24 @@ static cudaError_t launch_prefill_t(const PrefillArgs &a, const CUtensorMap &tq,
     return cudaGetLastError();
 }
 
+template <typename T, int D>
+static cudaError_t launch_prefill_mode(const PrefillArgs &a, const CUtensorMap &tq,
+                                       const CUtensorMap &tk, const CUtensorMap &tv, int grid,
+                                       cudaStream_t s) {
+    if (a.c.pse) return launch_prefill_t<T, D, kModePse>(a, tq, tk, tv, grid, s);
+    if (a.c.mask_type == 3) return launch_prefill_t<T, D, kModeAlibi>(a, tq, tk, tv, grid, s);
+    return launch_prefill_t<T, D, kModePlain>(a, tq, tk, tv, grid, s);
+}
+
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tq, const CUtensorMap &tk,
                            const CUtensorMap &tv, int q_dtype, int grid, cudaStream_t s) {
     const bool bf = (q_dtype == 1);
     if (a.c.D == 128)
-        return bf ? launch_prefill_t<__nv_bfloat16, 128>(a, tq, tk, tv, grid, s)
-                  : launch_prefill_t<__half, 128>(a, tq, tk, tv, grid, s);
+        return bf ? launch_prefill_mode<__nv_bfloat16, 128>(a, tq, tk, tv, grid, s)
+                  : launch_prefill_mode<__half, 128>(a, tq, tk, tv, grid, s);
     if (a.c.D == 64)
-        return bf ? launch_prefill_t<__nv_bfloat16, 64>(a, tq, tk, tv, grid, s)
-                  : launch_prefill_t<__half, 64>(a, tq, tk, tv, grid, s);
+        return bf ? launch_prefill_mode<__nv_bfloat16, 64>(a, tq, tk, tv, grid, s)
+                  : launch_prefill_mode<__half, 64>(a, tq, tk, tv, grid, s);
     return cudaErrorInvalidValue;
 }
 
