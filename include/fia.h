@@ -198,6 +198,35 @@ typedef struct {
 
 FIA_API fia_status fia_op_get_plan_info(const fia_op *op, fia_plan_info *info);
 
+/*
+ * Decode without a caller workspace (no counterpart in the pages: the aclnn and
+ * ATB interfaces always take a caller-allocated workspace).
+ *
+ * For callers that cannot allocate device memory when they run attention --
+ * an engine whose device memory is all handed out by its own pool at start-up,
+ * or a runtime that forbids cudaMalloc/cudaFree on its serving path -- this runs
+ * a decode-path op (split-KV decode + combine; fia_op_get_plan_info path == 1)
+ * with its scratch in a fixed array inside libfia.so instead of the `workspace`
+ * argument of fia_run.  Inputs and outputs are still the caller's tensors given
+ * to fia_get_workspace_size.  Nothing here allocates: no cudaMalloc, no
+ * cudaFree, no allocating library call.
+ *
+ *  - The array is FIA_STATIC_WORKSPACE_BYTES (32 MiB) per device.  Every GPU
+ *    that loads the library holds it until the process exits.
+ *  - An op whose workspaceSize exceeds it gets FIA_ERR_WORKSPACE; a prefill op
+ *    gets FIA_ERR_UNSUPPORTED; a no-op op returns FIA_OK.  Nothing is launched
+ *    in those cases.
+ *  - Call it with the op's device current.  The first call on a device looks up
+ *    the array's device address (cudaGetSymbolAddress); make that first call
+ *    before any stream capture.  A failed lookup returns FIA_ERR_CUDA.
+ *  - All calls on a device share the one array, which keeps the last call's
+ *    contents.  Calls that overlap on the GPU (two streams, or two host threads
+ *    without ordering) race on it: serialise them.
+ *  - Asynchronous on `stream` (a cudaStream_t passed as void*), like fia_run.
+ */
+#define FIA_STATIC_WORKSPACE_BYTES (32u * 1024u * 1024u)
+FIA_API fia_status fia_decode_run_static(fia_op *op, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

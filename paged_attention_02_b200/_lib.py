@@ -72,6 +72,8 @@ def _load():
     lib.fia_op_set_timing_events.restype = ctypes.c_int
     lib.fia_op_get_plan_info.argtypes = [P, ctypes.POINTER(fia_plan_info)]
     lib.fia_op_get_plan_info.restype = ctypes.c_int
+    lib.fia_decode_run_static.argtypes = [P, P]
+    lib.fia_decode_run_static.restype = ctypes.c_int
     return lib
 
 
@@ -105,3 +107,12 @@ def fia_op_set_timing_events(op, start, stop) -> int:
 
 def fia_op_get_plan_info(op, info) -> int:
     return _lib.fia_op_get_plan_info(op, info)
+
+
+FIA_STATIC_WORKSPACE_BYTES = 32 * 1024 * 1024
+
+
+def fia_decode_run_static(op, stream) -> int:
+    """Decode-path run with the library's fixed scratch array (no workspace
+    argument, no allocation); see include/fia.h."""
+    return _lib.fia_decode_run_static(op, stream)

@@ -1,6 +1,10 @@
 """Builds libfia.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m paged_attention_02_b200.build [--force] [--verbose]
+    python paged_attention_02_b200/build.py [--force] [--verbose] [--ptxas-info]
+
+Run it as a script (or load it by file path, as ``load_builder()`` in
+``__graft_entry__`` does): importing it through the package would first load
+the library it is meant to build.
 
 Static CUDA runtime, no libcuda link dependency (the driver entry point for
 TMA descriptor encoding is looked up at run time), so the library loads on a

@@ -22,6 +22,7 @@
 #include <cmath>
 #include <cstring>
 #include <functional>
+#include <mutex>
 #include <numeric>
 #include <queue>
 #include <vector>
@@ -505,6 +506,83 @@ fia_status fia_run(void *workspace, uint64_t workspaceSize, fia_op *op, void *st
         return FIA_ERR_CUDA;
     }
     if (op->ev_stop && cudaEventRecord(op->ev_stop, s) != cudaSuccess) {
+        cudaGetLastError();
+        return FIA_ERR_CUDA;
+    }
+    return FIA_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode with library-owned scratch (fia_decode_run_static).  The scratch is a
+// file-scope device array; host code only ever sees its address through
+// cudaGetSymbolAddress, looked up once per device and cached.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int kMaxStaticDevices = 64;
+static __device__ __align__(256) uint8_t g_fia_static_ws[FIA_STATIC_WORKSPACE_BYTES];
+std::mutex g_static_mu;
+void *g_static_addr[kMaxStaticDevices] = {};
+}  // namespace
+
+extern "C" {
+
+fia_status fia_decode_run_static(fia_op *op, void *stream_ptr) {
+    if (!op) return FIA_ERR_NULLPTR;
+    if (op->path == 0) return FIA_OK;
+    if (op->path != 1) return FIA_ERR_UNSUPPORTED;
+    if (op->ws_size > FIA_STATIC_WORKSPACE_BYTES) return FIA_ERR_WORKSPACE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxStaticDevices) {
+        cudaGetLastError();
+        return FIA_ERR_CUDA;
+    }
+    uint8_t *ws = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_static_mu);
+        if (!g_static_addr[dev]) {
+            void *addr = nullptr;
+            if (cudaGetSymbolAddress(&addr, g_fia_static_ws) != cudaSuccess || !addr) {
+                cudaGetLastError();
+                return FIA_ERR_CUDA;
+            }
+            g_static_addr[dev] = addr;
+        }
+        ws = reinterpret_cast<uint8_t *>(g_static_addr[dev]);
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_ptr);
+    // The plan (which also clears the error word) is rewritten on every call;
+    // every partial the combine reads is written by the decode kernel first.
+    if (cudaMemcpyAsync(ws, op->plan_host, op->plan_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+        cudaGetLastError();
+        return FIA_ERR_CUDA;
+    }
+    CommonArgs c = op->common;
+    c.seq = reinterpret_cast<const SeqInfo *>(ws + op->off_seq);
+    c.err = reinterpret_cast<uint32_t *>(ws + op->off_err);
+    DecodeArgs d{};
+    d.c = c;
+    d.units = reinterpret_cast<const DecodeUnit *>(ws + op->off_units);
+    d.part_o = reinterpret_cast<float *>(ws + op->off_part_o);
+    d.part_ml = reinterpret_cast<float2 *>(ws + op->off_part_ml);
+    d.k_scale = op->k_scale;
+    d.k_offset = op->k_offset;
+    d.n_units = op->grid;
+    cudaError_t e = cudaSuccess;
+    if (op->grid > 0) e = launch_decode(d, op->tk, op->tv, op->q_dtype, op->kv_int8, op->grid, s);
+    if (e == cudaSuccess && op->grid2 > 0) {
+        CombineArgs cb{};
+        cb.c = c;
+        cb.items = reinterpret_cast<const CombineItem *>(ws + op->off_citems);
+        cb.part_o = d.part_o;
+        cb.part_ml = d.part_ml;
+        cb.v_scale = op->v_scale;
+        cb.v_offset = op->v_offset;
+        cb.n_items = op->grid2;
+        e = launch_combine(cb, op->q_dtype, op->kv_int8, op->grid2, s);
+    }
+    if (e != cudaSuccess) {
         cudaGetLastError();
         return FIA_ERR_CUDA;
     }

@@ -23,7 +23,8 @@ def _declared_functions():
 
 
 def test_library_builds_and_exports_every_declared_symbol():
-    from paged_attention_02_b200 import build
+    import __graft_entry__
+    build = __graft_entry__.load_builder()
     build.build()
     lib = ctypes.CDLL(build.LIB_PATH)
     names = _declared_functions()
