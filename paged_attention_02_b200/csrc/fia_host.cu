@@ -393,19 +393,49 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
     } else {
         o->path = 2;
         const bool causal = (maskType != FIA_MASK_NONE);
+        // Pairs of 128-token tiles that read the same KV head: two heads of a
+        // GQA group (same tile), else two consecutive tiles of one head.  Tile
+        // 0 of a pair needs no more key tiles than tile 1.
+        auto ntiles = [&](int b, int q0) {
+            const int ql = seqLen[b], kl = kvSeqLen[b];
+            const int rows = std::min(kPrefillBM, ql - q0);
+            int kv_end = causal ? std::min(kl, kl - ql + q0 + rows) : kl;
+            kv_end = std::max(kv_end, 0);
+            return (kv_end + kPrefillBN - 1) / kPrefillBN;
+        };
         struct Cand {
             PrefillItem it;
             double cost;
         };
         std::vector<Cand> items;
+        auto add = [&](int b, int kvh, int q0a, int ha, int q0b, int hb) {
+            PrefillItem it{};
+            it.b = b;
+            it.kvh = kvh;
+            it.q0[0] = q0a; it.h[0] = ha;
+            it.q0[1] = q0b; it.h[1] = hb;
+            const int nb = ntiles(b, q0b);
+            items.push_back({it, nb + 0.75});
+        };
         for (int b = 0; b < batch; ++b) {
-            const int ql = seqLen[b], kl = kvSeqLen[b];
-            for (int q0 = 0; q0 < ql; q0 += kPrefillBM) {
-                const int rows = std::min(kPrefillBM, ql - q0);
-                int kv_end = causal ? std::min(kl, kl - ql + q0 + rows) : kl;
-                kv_end = std::max(kv_end, 0);
-                const int n = (kv_end + kPrefillBN - 1) / kPrefillBN;
-                for (int h = 0; h < headNum; ++h) items.push_back({{b, q0, h, 0}, n + 0.5});
+            const int ql = seqLen[b];
+            const int nqt = (ql + kPrefillBM - 1) / kPrefillBM;
+            if (g >= 2) {
+                for (int qt = 0; qt < nqt; ++qt) {
+                    const int q0 = qt * kPrefillBM;
+                    for (int kvh = 0; kvh < kvHeadNum; ++kvh) {
+                        int h = kvh * g;
+                        for (; h + 1 < (kvh + 1) * g; h += 2) add(b, kvh, q0, h, q0, h + 1);
+                        if (h < (kvh + 1) * g) add(b, kvh, 0, -1, q0, h);
+                    }
+                }
+            } else {
+                for (int h = 0; h < headNum; ++h) {
+                    int qt = 0;
+                    for (; qt + 1 < nqt; qt += 2)
+                        add(b, h, qt * kPrefillBM, h, (qt + 1) * kPrefillBM, h);
+                    if (qt < nqt) add(b, h, 0, -1, qt * kPrefillBM, h);
+                }
             }
         }
         std::stable_sort(items.begin(), items.end(),

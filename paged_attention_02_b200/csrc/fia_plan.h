@@ -26,9 +26,14 @@ struct CombineItem {
     int32_t slot0, nsplit, b, kvh;
 };
 
-// Prefill work item: 128 new tokens of one sequence for one query head.
+// Prefill work item: a pair of 128-new-token tiles of one sequence that read
+// the same KV head, processed together by one CTA (they share every K/V tile).
+// Tile 0 needs no more key tiles than tile 1; h[0] < 0 when tile 0 is absent.
 struct PrefillItem {
-    int32_t b, q0, h, pad;
+    int32_t b, kvh;
+    int32_t q0[2];   // first new token of each tile within the sequence
+    int32_t h[2];    // query head of each tile
+    int32_t pad[2];
 };
 
 constexpr int kDecodeRows = 16;      // rows (new token x head-in-group) per decode unit

@@ -1,28 +1,32 @@
 // prefill_kernel.cu -- paged prefill / prefix-encoder attention on sm_100a
 // tensor cores (tcgen05 UMMA, TMEM accumulators, TMA-staged paged K/V).
 //
-// Computes, for 128 new tokens of one sequence and one query head at a time,
+// Computes, for tiles of 128 new tokens of one sequence and one query head,
 //     O = Softmax(qkScale * Q K^T + bias) V
 // (aclnnFusedInferAttentionScoreV4 / V3 "Formula"; ATB PrefixEncoder: new
 // tokens attend to the cached prefix and to themselves, maskType 9 causal
 // generated internally, maskType 3 ALiBi from per-head slopes; V4 alibi
 // fullmask = pse tensor; V4 learnable sink; V3 lse bullet).
 //
-// One persistent CTA per SM walks a host-planned, longest-first list of
-// (sequence, 128-token tile, head) items.  Warp roles:
-//   warp 0   TMA producer: Q tile once per item, then K and V tiles of 128
-//            keys, each tile gathered block by block through the block table
-//            into a 2-stage ring (128-byte swizzled, K-major rows).
-//   warp 1   UMMA issuer (one elected lane): S_j = Q K_j^T into one of two
-//            TMEM S buffers, then O += P_{j-1} V_{j-1} into the TMEM O buffer,
-//            so the next QK^T overlaps the softmax of the previous tile.
-//            It also zeroes the V rows past kvSeqLen in a ragged last tile.
-//   warps 2-5 softmax + epilogue, one query row per thread (TMEM lane):
-//            tcgen05.ld the S row, scale / mask / bias in registers, online
-//            softmax in fp32 (log2 domain, rescale of O in TMEM only when the
-//            running max grows by more than 2^8), P rounded to the input dtype
-//            into shared memory for the PV MMA; at the end O / l, the sink
-//            term and lse.
+// One persistent CTA per SM walks a host-planned, longest-first list of tile
+// PAIRS: two 128-token tiles that read the same KV head (two heads of one GQA
+// group, or two consecutive tiles of one head), so every K/V tile fetched
+// serves 2 x 128 query rows.  Warp roles (10 warps):
+//   warp 0     TMA producer: both Q tiles once per pair, then K and V tiles
+//              of 128 keys, each gathered block by block through the block
+//              table (3-stage K ring, 2-stage V ring, 128-byte swizzle).
+//   warp 1     UMMA issuer (one lane): S_X = Q_X K_j^T into TMEM, and
+//              O_X += P_X V_j with P_X read from TMEM (TS form).  One thread's
+//              tcgen05.mma ops run in issue order, so QK_X(j+1) may be issued
+//              right after PV_X(j) over the same TMEM columns.  It zeroes the V
+//              rows past kvSeqLen in a ragged last tile.
+//   warps 2-5  softmax + epilogue of tile 0, warps 6-9 of tile 1: one query
+//              row per thread (TMEM lane), S row -> registers, scale / mask /
+//              bias, online softmax in fp32 (log2 domain; O rescaled in TMEM
+//              only when the running max grows by more than 2^8), P in the
+//              input dtype written back over S; at the end O / l, sink, lse.
+// TMEM (512 columns): S_0 | S_1 | O_0 | O_1.  While one softmax group works on
+// its S, the tensor core runs the other tile's PV and QK^T.
 // Every mbarrier wait is bounded in time (see fia_device.cuh).
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -41,19 +45,21 @@ struct PrefillCfg {
     static constexpr int kTileBytes = 128 * D * 2;         // Q, K or V tile (128 rows)
     static constexpr int kGroupBytes = 128 * 128;          // one 128-row x 128-byte group
     static constexpr int kKStages = 3;
-    static constexpr int kVStages = 3;
-    static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + kTileBytes;                   // K[s]
+    static constexpr int kVStages = 2;
+    static constexpr int kOffQ = 0;                                    // Q[2]
+    static constexpr int kOffK = kOffQ + 2 * kTileBytes;               // K[s]
     static constexpr int kOffV = kOffK + kKStages * kTileBytes;        // V[s]
     static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
-    // q_full, q_empty, k_full[3], k_empty[3], v_full[3], v_empty[3],
-    // s_full[2], s_empty[2], p_full, pv_done, o_full
-    static constexpr int kNumBar = 2 + 4 * 3 + 4 + 3;
+    // q_full, q_empty, k_full/k_empty[KS], v_full/v_empty[VS],
+    // s_full[2], p_full[2], pv_done[2], o_full[2]
+    static constexpr int kNumBar = 2 + 2 * kKStages + 2 * kVStages + 8;
     static constexpr int kUsed = kOffBar + kNumBar * 8 + 16;
     // Keep one CTA per SM (each CTA holds all 512 TMEM columns).
     static constexpr int kSmem = 1024 + (kUsed > 118 * 1024 ? kUsed : 118 * 1024);
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+    static constexpr uint32_t col_s(int x) { return (uint32_t)x * 128u; }
+    static constexpr uint32_t col_o(int x) { return 256u + (uint32_t)x * D; }
+    static constexpr int kThreads = 320;
 };
 
 int prefill_smem_bytes(int D) {
@@ -62,23 +68,39 @@ int prefill_smem_bytes(int D) {
     return -1;
 }
 
-struct ItemGeom {
-    int b, q0, h, kvh, cu_q, qlen, kvlen, rows, kv_end, n;
+struct SubGeom {
+    bool valid;
+    int q0, h, rows, n;
+};
+struct PairGeom {
+    int b, kvh, cu_q, qlen, kvlen;
+    SubGeom t[2];
+    int nA, nB;   // key tiles of tile 0 (0 if absent) and tile 1; nA <= nB
 };
 
-__device__ __forceinline__ ItemGeom item_geom(const PrefillArgs &a, int idx) {
+__device__ __forceinline__ PairGeom pair_geom(const PrefillArgs &a, int idx) {
     const PrefillItem it = a.items[idx];
     const SeqInfo si = a.c.seq[it.b];
-    ItemGeom g;
-    g.b = it.b; g.q0 = it.q0; g.h = it.h; g.kvh = it.h / a.c.g;
-    g.cu_q = si.cu_q; g.qlen = si.qlen; g.kvlen = si.kvlen;
-    g.rows = min(kPrefillBM, si.qlen - it.q0);
     const bool causal = (a.c.mask_type == 9 || a.c.mask_type == 3);
-    g.kv_end = causal ? min(si.kvlen, si.kvlen - si.qlen + it.q0 + g.rows) : si.kvlen;
-    if (g.kv_end < 0) g.kv_end = 0;
-    g.n = (g.kv_end + kPrefillBN - 1) / kPrefillBN;
+    PairGeom g;
+    g.b = it.b; g.kvh = it.kvh; g.cu_q = si.cu_q; g.qlen = si.qlen; g.kvlen = si.kvlen;
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+        SubGeom &s = g.t[x];
+        s.valid = it.h[x] >= 0;
+        s.q0 = it.q0[x];
+        s.h = it.h[x];
+        s.rows = s.valid ? min(kPrefillBM, si.qlen - it.q0[x]) : 0;
+        int kv_end = causal ? min(si.kvlen, si.kvlen - si.qlen + it.q0[x] + s.rows) : si.kvlen;
+        kv_end = max(kv_end, 0);
+        s.n = s.valid ? (kv_end + kPrefillBN - 1) / kPrefillBN : 0;
+    }
+    g.nA = g.t[0].n;
+    g.nB = g.t[1].n;
     return g;
 }
+
+enum { kModePlain = 0, kModeAlibi = 1, kModePse = 2 };
 
 // Bounded wait; on failure lane 0 leaves a trail record (item, tile, parity).
 #define FIA_WAIT(bar, parity, where)                                                      \
@@ -91,10 +113,8 @@ __device__ __forceinline__ ItemGeom item_geom(const PrefillArgs &a, int idx) {
         }                                                                                 \
     } while (0)
 
-enum { kModePlain = 0, kModeAlibi = 1, kModePse = 2 };
-
 template <typename T, int D, int MODE>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
 fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tq,
                    const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
     using Cfg = PrefillCfg<D>;
@@ -113,11 +133,10 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     uint64_t *k_empty = k_full + KS;        // [KS]
     uint64_t *v_full = k_empty + KS;        // [VS]
     uint64_t *v_empty = v_full + VS;        // [VS]
-    uint64_t *s_full = v_empty + VS;        // [2]
-    uint64_t *s_empty = s_full + 2;         // [2]  (released by the PV that read P from it)
-    uint64_t *p_full = s_empty + 2;
-    uint64_t *pv_done = p_full + 1;
-    uint64_t *o_full = pv_done + 1;
+    uint64_t *s_full = v_empty + VS;        // [2]  QK_X done
+    uint64_t *p_full = s_full + 2;          // [2]  P_X written (4 warps)
+    uint64_t *pv_done = p_full + 2;         // [2]  PV_X done
+    uint64_t *o_full = pv_done + 2;         // [2]  last PV_X of the pair done
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + Cfg::kNumBar);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -130,10 +149,12 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         mbar_init(q_empty, 1);
         for (int s = 0; s < KS; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
         for (int s = 0; s < VS; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
-        for (int s = 0; s < 2; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], 1); }
-        mbar_init(p_full, 4);
-        mbar_init(pv_done, 1);
-        mbar_init(o_full, 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&s_full[x], 1);
+            mbar_init(&p_full[x], 4);
+            mbar_init(&pv_done[x], 1);
+            mbar_init(&o_full[x], 1);
+        }
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tq);
@@ -149,6 +170,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     int dbg_j = -1;     // tile index recorded in failure trails
+    int idx = -1;
 
     const int it_begin = a.cta_off[blockIdx.x];
     const int it_end = a.cta_off[blockIdx.x + 1];
@@ -161,17 +183,21 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         if (lane == 0) {
             uint32_t q_it = 0, kv_it = 0;
             const int br = a.c.box_rows;
-            for (int idx = it_begin; idx < it_end; ++idx) {
-                const ItemGeom gm = item_geom(a, idx);
-                if (gm.n == 0) continue;
+            for (idx = it_begin; idx < it_end; ++idx) {
+                const PairGeom gm = pair_geom(a, idx);
+                if (gm.nB == 0) continue;
                 FIA_WAIT(q_empty, (q_it & 1) ^ 1, 10);
-                mbar_arrive_expect_tx(q_full, Cfg::kTileBytes);
-                for (int hv = 0; hv < Cfg::kHalves; ++hv)
-                    tma_load_3d(smem + Cfg::kOffQ + hv * Cfg::kGroupBytes, &tq, q_full, hv * 64,
-                                gm.h, gm.cu_q + gm.q0);
+                mbar_arrive_expect_tx(q_full, (gm.t[0].valid ? 2 : 1) * Cfg::kTileBytes);
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    if (!gm.t[x].valid) continue;
+                    for (int hv = 0; hv < Cfg::kHalves; ++hv)
+                        tma_load_3d(smem + Cfg::kOffQ + x * Cfg::kTileBytes + hv * Cfg::kGroupBytes,
+                                    &tq, q_full, hv * 64, gm.t[x].h, gm.cu_q + gm.t[x].q0);
+                }
                 ++q_it;
                 const int32_t *bt_row = a.c.bt + (int64_t)gm.b * a.c.bt_stride;
-                for (int j = 0; j < gm.n; ++j, ++kv_it) {
+                for (int j = 0; j < gm.nB; ++j, ++kv_it) {
                     dbg_j = j;
                     const int t0 = j * kPrefillBN;
                     const int t1 = min(t0 + kPrefillBN, gm.kvlen);
@@ -203,89 +229,122 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ UMMA issuer
-        uint32_t q_it = 0, kv_it = 0, s_it = 0, p_it = 0;
-        for (int idx = it_begin; idx < it_end; ++idx) {
-            const ItemGeom gm = item_geom(a, idx);
-            if (gm.n == 0) continue;
+        uint32_t q_it = 0, kv_it = 0, p_it[2] = {0, 0};
+        auto issue_qk = [&](int x, int ks) {
+            const uint32_t qb = sm_q + x * Cfg::kTileBytes;
+            const uint32_t kb = sm_k0 + ks * Cfg::kTileBytes;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * Cfg::kGroupBytes + (kk & 3) * 32;
+                umma_ss(tmem + Cfg::col_s(x), umma_desc_sw128(qb + off, 16, 1024),
+                        umma_desc_sw128(kb + off, 16, 1024), IDESC_QK, kk > 0);
+            }
+        };
+        auto issue_pv = [&](int x, int vs, bool acc) {
+            const uint32_t vb = sm_v0 + vs * Cfg::kTileBytes;
+#pragma unroll
+            for (int kk = 0; kk < kPrefillBN / 16; ++kk)
+                umma_ts(tmem + Cfg::col_o(x), tmem + Cfg::col_s(x) + kk * 8,
+                        umma_desc_sw128(vb + kk * 2048, Cfg::kGroupBytes, 1024), IDESC_PV,
+                        (acc || kk > 0) ? 1u : 0u);
+        };
+        for (idx = it_begin; idx < it_end; ++idx) {
+            const PairGeom gm = pair_geom(a, idx);
+            if (gm.nB == 0) continue;
+            dbg_j = -1;
             FIA_WAIT(q_full, q_it & 1, 20);
             ++q_it;
             const uint32_t kv_base = kv_it;
-            const uint32_t s_base = s_it;
-            for (int j = 0; j <= gm.n; ++j) {
+            {
+                // QK for key tile 0 (both tiles)
+                const int ks = kv_base % KS;
+                FIA_WAIT(&k_full[ks], (kv_base / KS) & 1, 21);
+                __syncwarp();
+                tc_fence_after();
+                if (lane == 0) {
+                    if (gm.nA > 0) { issue_qk(0, ks); umma_commit(&s_full[0]); }
+                    issue_qk(1, ks);
+                    umma_commit(&s_full[1]);
+                    umma_commit(&k_empty[ks]);
+                    if (gm.nB == 1) umma_commit(q_empty);
+                }
+                __syncwarp();
+            }
+            for (int j = 0; j < gm.nB; ++j) {
                 dbg_j = j;
-                if (j < gm.n) {
-                    // S_j = Q K_j^T  into TMEM buffer j % 2
-                    const uint32_t kvi = kv_base + j;
-                    const int ks = kvi % KS;
-                    FIA_WAIT(&k_full[ks], (kvi / KS) & 1, 21);
-                    const int sb = s_it & 1;
-                    FIA_WAIT(&s_empty[sb], ((s_it >> 1) & 1) ^ 1, 22);
+                const uint32_t kvi = kv_base + j;
+                const int vs = kvi % VS;
+                FIA_WAIT(&v_full[vs], (kvi / VS) & 1, 24);
+                __syncwarp();
+                const int valid = gm.kvlen - j * kPrefillBN;
+                if (valid < kPrefillBN) {
+                    // rows past kvSeqLen: P is 0 there, but the slots may
+                    // hold anything (NaN * 0 = NaN in the MMA) -> zero them.
+                    uint8_t *vd = smem + Cfg::kOffV + vs * Cfg::kTileBytes;
+                    const int nbytes = (kPrefillBN - valid) * 128;
+                    for (int hv = 0; hv < Cfg::kHalves; ++hv) {
+                        uint4 *p = reinterpret_cast<uint4 *>(vd + hv * Cfg::kGroupBytes + valid * 128);
+                        for (int x = lane; x < nbytes / 16; x += 32) p[x] = make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                const bool more = (j + 1 < gm.nB);
+                const uint32_t kn = kv_base + j + 1;
+                const int ksn = kn % KS;
+                if (j < gm.nA) {
+                    FIA_WAIT(&p_full[0], p_it[0] & 1, 23);
+                    ++p_it[0];
                     __syncwarp();
                     tc_fence_after();
                     if (lane == 0) {
-                        const uint32_t kbase = sm_k0 + ks * Cfg::kTileBytes;
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t off = (kk >> 2) * Cfg::kGroupBytes + (kk & 3) * 32;
-                            umma_ss(tmem + (sb ? Cfg::kColS1 : Cfg::kColS0),
-                                    umma_desc_sw128(sm_q + off, 16, 1024),
-                                    umma_desc_sw128(kbase + off, 16, 1024), IDESC_QK, kk > 0);
-                        }
-                        umma_commit(&s_full[sb]);
-                        umma_commit(&k_empty[ks]);
-                        if (j == gm.n - 1) umma_commit(q_empty);
+                        issue_pv(0, vs, j > 0);
+                        umma_commit(&pv_done[0]);
+                        if (j == gm.nA - 1) umma_commit(&o_full[0]);
                     }
                     __syncwarp();
-                    ++s_it;
-                }
-                if (j >= 1) {
-                    // O += P_{j-1} V_{j-1}; P is in TMEM (aliasing S buffer (j-1) % 2)
-                    const int jj = j - 1;
-                    const uint32_t kvi = kv_base + jj;
-                    const int vs = kvi % VS;
-                    const int sb = (s_base + jj) & 1;
-                    FIA_WAIT(p_full, p_it & 1, 23);
-                    FIA_WAIT(&v_full[vs], (kvi / VS) & 1, 24);
-                    __syncwarp();
-                    const uint32_t vbase = sm_v0 + vs * Cfg::kTileBytes;
-                    const int valid = gm.kvlen - jj * kPrefillBN;
-                    if (valid < kPrefillBN) {
-                        // rows past kvSeqLen: P is 0 there, but the slots may
-                        // hold anything (NaN * 0 = NaN in the MMA) -> zero them.
-                        uint8_t *vd = smem + Cfg::kOffV + vs * Cfg::kTileBytes;
-                        const int nbytes = (kPrefillBN - valid) * 128;
-                        for (int hv = 0; hv < Cfg::kHalves; ++hv) {
-                            uint4 *p = reinterpret_cast<uint4 *>(vd + hv * Cfg::kGroupBytes + valid * 128);
-                            for (int x = lane; x < nbytes / 16; x += 32) p[x] = make_uint4(0, 0, 0, 0);
-                        }
-                        fence_proxy_async_smem();
+                    if (j + 1 < gm.nA) {
+                        FIA_WAIT(&k_full[ksn], (kn / KS) & 1, 22);
+                        __syncwarp();
+                        tc_fence_after();
+                        if (lane == 0) { issue_qk(0, ksn); umma_commit(&s_full[0]); }
                         __syncwarp();
                     }
+                }
+                FIA_WAIT(&p_full[1], p_it[1] & 1, 25);
+                ++p_it[1];
+                __syncwarp();
+                tc_fence_after();
+                if (lane == 0) {
+                    issue_pv(1, vs, j > 0);
+                    umma_commit(&pv_done[1]);
+                    umma_commit(&v_empty[vs]);
+                    if (j == gm.nB - 1) umma_commit(&o_full[1]);
+                }
+                __syncwarp();
+                if (more) {
+                    FIA_WAIT(&k_full[ksn], (kn / KS) & 1, 26);
+                    __syncwarp();
                     tc_fence_after();
                     if (lane == 0) {
-                        const uint32_t pcol = tmem + (sb ? Cfg::kColS1 : Cfg::kColS0);
-#pragma unroll
-                        for (int kk = 0; kk < kPrefillBN / 16; ++kk) {
-                            umma_ts(tmem + Cfg::kColO, pcol + kk * 8,
-                                    umma_desc_sw128(vbase + kk * 2048, Cfg::kGroupBytes, 1024),
-                                    IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
-                        }
-                        umma_commit(pv_done);
-                        umma_commit(&v_empty[vs]);
-                        umma_commit(&s_empty[sb]);
-                        if (jj == gm.n - 1) umma_commit(o_full);
+                        issue_qk(1, ksn);
+                        umma_commit(&s_full[1]);
+                        umma_commit(&k_empty[ksn]);
+                        if (j + 1 == gm.nB - 1) umma_commit(q_empty);
                     }
                     __syncwarp();
-                    ++p_it;
                 }
             }
-            kv_it = kv_base + gm.n;
+            kv_it = kv_base + gm.nB;
         }
     } else {
         // ------------------------------------------------------------ softmax + epilogue
+        const int X = (warp - 2) >> 2;             // which tile of the pair
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
+        const uint32_t scol = t_lane + Cfg::col_s(X);
+        const uint32_t ocol = t_lane + Cfg::col_o(X);
         const bool causal = (a.c.mask_type == 9 || a.c.mask_type == 3);
         const float sl2 = a.c.scale_log2;
         // plain mode with a positive scale: mask raw scores and fold the scale
@@ -293,13 +352,15 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         const bool fold = (MODE == kModePlain) && (sl2 > 0.f);
         uint32_t s_it = 0, p_it = 0, o_it = 0;
         T *outp = reinterpret_cast<T *>(a.c.out);
-        for (int idx = it_begin; idx < it_end; ++idx) {
-            const ItemGeom gm = item_geom(a, idx);
-            const int i = gm.q0 + row;
+        for (idx = it_begin; idx < it_end; ++idx) {
+            const PairGeom gm = pair_geom(a, idx);
+            const SubGeom sg = gm.t[X];
+            if (!sg.valid) continue;
+            const int i = sg.q0 + row;
             const bool valid = i < gm.qlen;
             const int qpos = gm.kvlen - gm.qlen + i;
-            const int64_t orow = ((int64_t)(gm.cu_q + i) * a.c.H + gm.h);
-            if (gm.n == 0) {
+            const int64_t orow = ((int64_t)(gm.cu_q + i) * a.c.H + sg.h);
+            if (sg.n == 0) {
                 if (valid) {
                     uint4 *dst = reinterpret_cast<uint4 *>(outp + orow * D);
                     for (int x = 0; x < D * 2 / 16; ++x) dst[x] = make_uint4(0, 0, 0, 0);
@@ -309,20 +370,19 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 continue;
             }
             float slope2 = 0.f;
-            if constexpr (MODE == kModeAlibi) slope2 = a.c.slopes[gm.h] * kLog2e;
+            if constexpr (MODE == kModeAlibi) slope2 = a.c.slopes[sg.h] * kLog2e;
             const T *pse_row = nullptr;
             if constexpr (MODE == kModePse) {
                 // rows past seqLen read row 0 of the sequence (their output is dropped)
                 pse_row = reinterpret_cast<const T *>(a.c.pse) +
-                          (((int64_t)gm.b * a.c.H + gm.h) * a.c.pse_q + (valid ? i : 0)) * a.c.pse_kv;
+                          (((int64_t)gm.b * a.c.H + sg.h) * a.c.pse_q + (valid ? i : 0)) * a.c.pse_kv;
             }
             float m = -INFINITY, l = 0.f;
-            for (int j = 0; j < gm.n; ++j) {
+            for (int j = 0; j < sg.n; ++j) {
                 dbg_j = j;
-                const int sb = s_it & 1;
-                const uint32_t scol = t_lane + (sb ? Cfg::kColS1 : Cfg::kColS0);
                 const int tb = j * kPrefillBN;
-                FIA_WAIT(&s_full[sb], (s_it >> 1) & 1, 30);
+                FIA_WAIT(&s_full[X], s_it & 1, 30);
+                ++s_it;
                 __syncwarp();          // tcgen05.ld/st below are warp-collective (.aligned)
                 tc_fence_after();
                 uint32_t sr[4][32];
@@ -331,7 +391,6 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 tmem_ld_wait();
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) reg_fence32(sr[cc]);
-                ++s_it;
 
                 // ---- scores (log2 units unless folded), bias, masks ----
                 const bool edge = (tb + kPrefillBN > gm.kvlen) || (causal && tb + kPrefillBN - 1 > qpos);
@@ -357,7 +416,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                             } else {
 #pragma unroll
                                 for (int e = 0; e < 8; ++e)
-                                    pv[e] = (t + e < gm.kvlen) ? pse_row[t + e] : pv[0];
+                                    pv[e] = (t + e < gm.kvlen) ? pse_row[t + e] : pse_row[0];
                             }
 #pragma unroll
                             for (int e = 0; e < 8; ++e) {
@@ -436,47 +495,45 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 }
                 l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
 
-                // The previous PV must be complete before this warp signals P_j:
-                // (1) O may be rescaled below; (2) it keeps every softmax warp
-                // within one tile of the others, so the 4 arrivals that complete
-                // a p_full phase always belong to the same tile, and pv_done can
-                // never run two phases ahead of this parity wait.
-                if (j > 0) {
-                    FIA_WAIT(pv_done, (p_it - 1) & 1, 31);
-                    __syncwarp();
-                    tc_fence_after();
-                }
-                // rescale O (rare)
+                // Rescale O (rare).  The previous PV of this tile must be done
+                // with O first.  (The softmax warps cannot drift apart: S for
+                // the next key tile is only produced after all four warps have
+                // signalled this P, so p_full phases never mix tiles.)
                 if (__any_sync(0xffffffffu, need)) {
+                    if (j > 0) {
+                        FIA_WAIT(&pv_done[X], (p_it - 1) & 1, 31);
+                        __syncwarp();
+                        tc_fence_after();
+                    }
 #pragma unroll
                     for (int cc = 0; cc < D / 32; ++cc) {
                         uint32_t orr[32];
-                        tmem_ld32(t_lane + Cfg::kColO + cc * 32, orr);
+                        tmem_ld32(ocol + cc * 32, orr);
                         tmem_ld_wait();
                         reg_fence32(orr);
 #pragma unroll
                         for (int x = 0; x < 32; ++x)
                             orr[x] = __float_as_uint(__uint_as_float(orr[x]) * alpha);
-                        tmem_st32(t_lane + Cfg::kColO + cc * 32, orr);
+                        tmem_st32(ocol + cc * 32, orr);
                     }
                 }
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(p_full);
+                if (lane == 0) mbar_arrive(&p_full[X]);
                 ++p_it;
             }
 
             // ---- epilogue: O / l (+ sink), lse ----
-            dbg_j = gm.n;
-            FIA_WAIT(o_full, o_it & 1, 32);
+            dbg_j = sg.n;
+            FIA_WAIT(&o_full[X], o_it & 1, 32);
             ++o_it;
             __syncwarp();
             tc_fence_after();
             const float mu = (m == -INFINITY) ? 0.f : m;
             float M = mu, lt = l;
             if (a.c.sink) {
-                const float s2 = a.c.sink[gm.h] * kLog2e;
+                const float s2 = a.c.sink[sg.h] * kLog2e;
                 M = fmaxf(mu, s2);
                 lt = l * ex2(mu - M) + ex2(s2 - M);
             }
@@ -484,7 +541,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
 #pragma unroll
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t orr[32];
-                tmem_ld32(t_lane + Cfg::kColO + cc * 32, orr);
+                tmem_ld32(ocol + cc * 32, orr);
                 tmem_ld_wait();
                 reg_fence32(orr);
                 if (valid) {
@@ -522,7 +579,7 @@ static cudaError_t launch_prefill_t(const PrefillArgs &a, const CUtensorMap &tq,
     const int smem = PrefillCfg<D>::kSmem;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, 192, smem, s>>>(a, tq, tk, tv);
+    kern<<<grid, PrefillCfg<D>::kThreads, smem, s>>>(a, tq, tk, tv);
     return cudaGetLastError();
 }
 
