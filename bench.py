@@ -84,20 +84,25 @@ def io_bytes(p) -> int:
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 20 ms from before the
+    warm-up to after the timed region; each line is stamped with host time so
+    the samples inside the timed window can be picked out."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, gpu_index: int):
         self.idx = gpu_index
         self.proc = None
         self.lines = []
+        self.window = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.idx), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -105,9 +110,14 @@ class ClockSampler:
             self.proc = None
         return self
 
+    def wait_first(self, timeout=5.0):
+        t0 = time.time()
+        while self.proc is not None and not self.lines and time.time() - t0 < timeout:
+            time.sleep(0.01)
+
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
 
     def __exit__(self, *a):
         if self.proc is not None:
@@ -117,10 +127,9 @@ class ClockSampler:
             except Exception:
                 self.proc.kill()
 
-    def summary(self):
+    def _parse(self, lines):
         sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for _, ln in lines:
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -129,11 +138,23 @@ class ClockSampler:
                 mx = float(parts[2])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
+            for n, v in zip(self.NAMES, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
+        return sm, mx, reasons
+
+    def summary(self):
+        inside = self.lines
+        scope = "timed region"
+        if self.window is not None:
+            t0, t1 = self.window
+            inside = [x for x in self.lines if t0 <= x[0] <= t1 + 0.025]
+            if not inside:
+                inside = self.lines
+                scope = "warm-up + timed region (timed region shorter than the 20 ms sample period)"
+        sm, mx, reasons = self._parse(inside)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "scope": scope}
 
 
 # ---------------------------------------------------------------------------
@@ -246,8 +267,8 @@ def cpu_baseline(p, budget_s=12.0):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
@@ -304,19 +325,22 @@ def main():
     t = to_dev(p, dev)
     op = make_op(p, t)
     info = op.plan_info()
-    # warm-up + timed steps, bracketed by barrier + synchronize
-    for _ in range(args.warmup):
-        flush.zero_()
-        op.run()
-    torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
     with ClockSampler(local) as clk:
+        clk.wait_first()
+        # warm-up + timed steps, bracketed by barrier + synchronize
+        for _ in range(args.warmup):
+            flush.zero_()
+            op.run()
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t_start = time.time()
         run_ms, kern_ms = time_op(op, args.steps, 0, flush)
-    torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
+        torch.cuda.synchronize()
+        clk.window = (t_start, time.time())
+        if dist is not None:
+            dist.barrier()
     ms = statistics.mean(run_ms)
     kms = statistics.mean(kern_ms)
     if dist is not None:

@@ -60,7 +60,7 @@ int decode_smem_bytes(int D, bool kv_int8) {
 }
 
 template <typename T, int D, bool INT8>
-__global__ void __launch_bounds__(128, 2)
+__global__ void __launch_bounds__(128, INT8 ? 3 : 2)
 fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv) {
     using Cfg = DecodeCfg<D, INT8>;
@@ -178,11 +178,11 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
             cs_a += __shfl_xor_sync(0xffffffffu, cs_a, x);
             cs_b += __shfl_xor_sync(0xffffffffu, cs_b, x);
         }
-        // Scale each row by a power of two so that max|q'| lands below 2^14
-        // (f16 range), then undo it on the fp32 accumulator.
+        // Scale each row by a power of two so that max|q'| lands below 2^11
+        // (well inside f16 range), then undo it on the fp32 accumulator.
         int ea = 0, eb = 0;
-        if (mx_a > 0.f) { frexpf(mx_a, &ea); ea = 14 - ea; }
-        if (mx_b > 0.f) { frexpf(mx_b, &eb); eb = 14 - eb; }
+        if (mx_a > 0.f) { frexpf(mx_a, &ea); ea = 11 - ea; }
+        if (mx_b > 0.f) { frexpf(mx_b, &eb); eb = 11 - eb; }
 #pragma unroll
         for (int kk = 0; kk < KT; ++kk) {
             qf[kk][0] = pack2<__half>(ldexpf(qa[kk][0], ea), ldexpf(qa[kk][1], ea));
@@ -192,8 +192,26 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
         }
         sc_a = ldexpf(a.c.scale_log2, -ea);
         sc_b = ldexpf(a.c.scale_log2, -eb);
-        add_a = cs_a * a.c.scale_log2;
-        add_b = cs_b * a.c.scale_log2;
+        // The MMA sees each key byte as the f16 value 1152 + k (see the QK loop),
+        // so the raw score carries 1152 * sum_d q'_d, with q' exactly as the MMA
+        // saw it (f16): remove it here, together with the key offset term.
+        float sq_a = 0.f, sq_b = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < KT; ++kk) {
+            const float2 fa0 = __half22float2(*reinterpret_cast<const __half2 *>(&qf[kk][0]));
+            const float2 fa1 = __half22float2(*reinterpret_cast<const __half2 *>(&qf[kk][2]));
+            const float2 fb0 = __half22float2(*reinterpret_cast<const __half2 *>(&qf[kk][1]));
+            const float2 fb1 = __half22float2(*reinterpret_cast<const __half2 *>(&qf[kk][3]));
+            sq_a += (fa0.x + fa0.y) + (fa1.x + fa1.y);
+            sq_b += (fb0.x + fb0.y) + (fb1.x + fb1.y);
+        }
+#pragma unroll
+        for (int x = 1; x <= 2; x <<= 1) {
+            sq_a += __shfl_xor_sync(0xffffffffu, sq_a, x);
+            sq_b += __shfl_xor_sync(0xffffffffu, sq_b, x);
+        }
+        add_a = cs_a * a.c.scale_log2 - 1152.0f * sq_a * sc_a;
+        add_b = cs_b * a.c.scale_log2 - 1152.0f * sq_b * sc_b;
     }
     const bool causal = (a.c.mask_type == 9 || a.c.mask_type == 3);
     const bool alibi = a.c.mask_type == 3;
@@ -242,9 +260,12 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
                     const int tok = warp * 16 + nt * 8 + r;
+                    // bytes biased to 128 + k under the f16 exponent pattern:
+                    // f16 values 1152 + k, exact; the 1152 * sum(q') term is
+                    // removed from the row constant above
                     const uint32_t w = lds32(kst + swz128(tok, kk) + 4 * c) ^ 0x80808080u;
-                    mma_16816<false>(sacc[nt], qf[kk], i8pair_to_h2<0x4140>(w),
-                                     i8pair_to_h2<0x4342>(w));
+                    mma_16816<false>(sacc[nt], qf[kk], prmt(w, 0x64646464u, 0x4140u),
+                                     prmt(w, 0x64646464u, 0x4342u));
                 }
             }
         }

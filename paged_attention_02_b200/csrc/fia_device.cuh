@@ -54,14 +54,14 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
-// try_wait with a suspend-time hint: a waiting warp is parked by the hardware
-// (up to ~0.5 ms) instead of spinning through issue slots the softmax warps need.
+// try_wait (the hardware may briefly park the warp; no explicit suspend hint:
+// a measured hint woke the waiter later than plain polling did).
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
                  "selp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(500000u) : "memory");
+                 : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
     return ok != 0;
 }
 
@@ -74,7 +74,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 3u) == 3u) {
+        if ((it & 63u) == 63u) {
             if (*abort) return false;
             if (globaltimer_ns() - t0 > kWaitLimitNs) {
                 *abort = 1;
@@ -328,6 +328,66 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// ---- packed fp32 pairs (Blackwell f32x2 FMA/ADD on a 64-bit register pair) ----
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x for a pair of fp32 values on the FMA/ALU pipes (no MUFU), used for a
+// share of the softmax exponentials so that they do not all queue on the
+// special-function unit.  Method: x = n + f with n = round(x) obtained by
+// adding 1.5*2^23 (the sum's low mantissa bits hold n), f in [-1/2, 1/2];
+// 2^f by a degree-3 polynomial whose coefficients were fitted here to the
+// relative error of 2^f on [-1/2, 1/2] (least squares on Chebyshev nodes with
+// Lawson reweighting toward minimax; worst relative error 1.0e-4 evaluated in
+// fp32, below half an fp16 ulp); 2^n joins by an integer add to the exponent
+// field.  Because 1.5*2^23 has its low 9 bits clear, (bits(t) << 23) equals
+// n << 23 exactly, so the join is one integer multiply-add.  Inputs are
+// clamped at -126 (smaller results are negligible against the row sum >= 1;
+// -inf gives ~1e-38 instead of 0).
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
+    float x0, x1;
+    f2unpack(x2, x0, x1);
+    x2 = f2pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+    const uint64_t kShift = f2pack(12582912.0f, 12582912.0f);
+    const uint64_t kNegShift = f2pack(-12582912.0f, -12582912.0f);
+    const uint64_t kNegOne = f2pack(-1.0f, -1.0f);
+    const uint64_t t = fadd2(x2, kShift);            // round(x) in the low mantissa bits
+    const uint64_t r = fadd2(t, kNegShift);          // round(x) as a float
+    const uint64_t f = ffma2(r, kNegOne, x2);        // x - round(x) in [-1/2, 1/2]
+    uint64_t p = ffma2(f2pack(0.0550089031f, 0.0550089031f), f,
+                       f2pack(0.2422109693f, 0.2422109693f));
+    p = ffma2(p, f, f2pack(0.6932829618f, 0.6932829618f));
+    p = ffma2(p, f, f2pack(1.0f, 1.0f));
+    float p0, p1, t0, t1;
+    f2unpack(p, p0, p1);
+    f2unpack(t, t0, t1);
+    uint32_t r0, r1;
+    asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(r0) : "r"(__float_as_uint(t0)), "r"(__float_as_uint(p0)));
+    asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(r1) : "r"(__float_as_uint(t1)), "r"(__float_as_uint(p1)));
+    return f2pack(__uint_as_float(r0), __uint_as_float(r1));
 }
 
 template <typename T> __device__ __forceinline__ uint32_t pack2(float lo, float hi);

@@ -444,15 +444,18 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                             if (!keep) sr[cc][x] = __float_as_uint(-INFINITY);
                         }
                 }
-                // tree max (8 independent chains)
+                // tree max: 8 independent chains of 3-input max
+#define FIA_EL(e) __uint_as_float(sr[(e) >> 5][(e) & 31])
                 float mx8[8];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) mx8[k] = __uint_as_float(sr[0][k]);
+                for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(FIA_EL(k), FIA_EL(k + 8));
 #pragma unroll
-                for (int e = 8; e < 128; ++e)
-                    mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(sr[e >> 5][e & 31]));
-                float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+                for (int e = 16; e < 128; e += 16)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) mx8[k] = fmax3(mx8[k], FIA_EL(e + k), FIA_EL(e + 8 + k));
+#undef FIA_EL
+                float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                                 fmaxf(mx8[6], mx8[7]));
                 if (fold) mx = (mx == -INFINITY) ? -INFINITY : mx * sl2;
 
                 // running max: exact on the first tile, afterwards raised only
@@ -470,30 +473,40 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 }
                 const float mu = (m == -INFINITY) ? 0.f : m;
 
-                // P = 2^(s - m) in the input dtype, stored over S's first 64 columns
-                float ls8[8];
+                // P = 2^(s - m) in the input dtype, stored over S's first 64
+                // columns; pairs of columns go through f32x2 math.  (Moving a
+                // share of the exponentials to the FMA-pipe polynomial
+                // exp2_poly_x2 measured slower here: the loop is latency-bound,
+                // not MUFU-throughput-bound, at this warp count.)
+                const uint64_t negmu2 = f2pack(-mu, -mu);
+                const uint64_t sl2x2 = f2pack(sl2, sl2);
+                uint64_t acc2[4];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) ls8[k] = 0.f;
+                for (int k = 0; k < 4; ++k) acc2[k] = f2pack(0.f, 0.f);
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int x = 0; x < 16; ++x) {
+                        const uint64_t s2 = f2pack(__uint_as_float(sr[cc][2 * x]),
+                                                   __uint_as_float(sr[cc][2 * x + 1]));
+                        const uint64_t xx = fold ? ffma2(s2, sl2x2, negmu2) : fadd2(s2, negmu2);
+                        float a0, a1;
+                        f2unpack(xx, a0, a1);
+                        const uint64_t pp = f2pack(ex2(a0), ex2(a1));
+                        acc2[x & 3] = fadd2(acc2[x & 3], pp);
                         float p0, p1;
-                        if (fold) {
-                            p0 = ex2(fmaf(__uint_as_float(sr[cc][2 * x]), sl2, -mu));
-                            p1 = ex2(fmaf(__uint_as_float(sr[cc][2 * x + 1]), sl2, -mu));
-                        } else {
-                            p0 = ex2(__uint_as_float(sr[cc][2 * x]) - mu);
-                            p1 = ex2(__uint_as_float(sr[cc][2 * x + 1]) - mu);
-                        }
-                        ls8[(2 * x) & 7] += p0;
-                        ls8[(2 * x + 1) & 7] += p1;
+                        f2unpack(pp, p0, p1);
                         pk[x] = pack2<T>(p0, p1);
                     }
                     tmem_st16(scol + cc * 16, pk);
                 }
-                l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
+                {
+                    const uint64_t s01 = fadd2(fadd2(acc2[0], acc2[1]), fadd2(acc2[2], acc2[3]));
+                    float l0, l1;
+                    f2unpack(s01, l0, l1);
+                    l += l0 + l1;
+                }
 
                 // Rescale O (rare).  The previous PV of this tile must be done
                 // with O first.  (The softmax warps cannot drift apart: S for
