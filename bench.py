@@ -272,9 +272,26 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
-    ap.add_argument("--only", default=None, help="profile helper: run one named workload only")
+    ap.add_argument("--profile", default=None, metavar="WORKLOAD",
+                    help="run --warmup + --steps plain fia_run calls of one named workload "
+                         "(%s) and exit: the command profiled by ncu" % ", ".join(W.NAMED))
     args = ap.parse_args()
-    args.warmup = max(args.warmup, 3)
+    if not args.profile:
+        args.warmup = max(args.warmup, 3)
+
+    if args.profile:
+        import paged_attention_02_b200  # noqa: F401
+        dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+        torch.cuda.set_device(dev)
+        q = W.NAMED[args.profile]()
+        op = make_op(q, to_dev(q, dev))
+        for _ in range(args.warmup + args.steps):
+            op.run()
+        torch.cuda.synchronize()
+        assert op.error_word() == 0
+        print(json.dumps({"profile": args.profile, "launches": args.warmup + args.steps,
+                          "plan": op.plan_info()}))
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -17,13 +17,16 @@
 //     group form the 16-row A operand of m16n8k16 tensor-core MMAs:
 //     S = Q K^T (keys as N), online softmax in fp32 on the accumulator
 //     fragments, then O += P V with P fed straight from registers.
-//   * int8 caches are widened to f16 in registers (exact for |x| <= 127); the
-//     per-channel K scale is folded into q (with a power-of-two range fix) and
-//     the K offset becomes one additive constant per row; the V scale/offset
+//   * int8 caches are widened to f16 in registers by placing each byte (+128)
+//     under the f16 exponent pattern for 1024, i.e. the exact value 1152 + x;
+//     the 1152 bias is removed afterwards (for K from the per-row constant,
+//     for V through a per-row sum of P from one extra MMA against ones).  The
+//     per-channel K scale is folded into q (with a power-of-two range fix), the
+//     K offset becomes one additive constant per row, and the V scale/offset
 //     are applied once in the combine.
 //   * Warps merge their (m, l, O) in shared memory and the CTA writes one
 //     partial per unit.
-// Kernel 2, fia_combine_kernel: one CTA per (b, kvh); merges the unit
+// Kernel 2, fia_combine_kernel: one CTA per (b, kvh, row); merges the unit
 //   partials in fixed logical order (deterministic), adds the learnable sink
 //   to the denominator, applies int8 V dequantisation, writes out and lse.
 #include <cuda.h>
@@ -225,6 +228,9 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
     }
 
     float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+    // int8: sum of the (f16-rounded) P each row fed to the MMA, to remove the
+    // 1152 bias of the value operand (see the PV loop)
+    float osum[4] = {0.f, 0.f, 0.f, 0.f};
     float o[D / 8][4];
 #pragma unroll
     for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
@@ -300,12 +306,15 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
             mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, x));
             mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, x));
         }
+        // Running max raised only when it grows by more than 2^8 (P stays
+        // <= 2^8, fine for f16/bf16); O, l and m stay mutually consistent.
         const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
-        const float mu_a = (mn_a == -INFINITY) ? 0.f : mn_a;
-        const float mu_b = (mn_b == -INFINITY) ? 0.f : mn_b;
-        const float al_a = ex2(m_a - mu_a), al_b = ex2(m_b - mu_b);
-        m_a = mn_a;
-        m_b = mn_b;
+        const bool up_a = mn_a > m_a + 8.0f, up_b = mn_b > m_b + 8.0f;
+        float al_a = 1.0f, al_b = 1.0f;
+        if (up_a) { al_a = ex2(m_a - mn_a); m_a = mn_a; }
+        if (up_b) { al_b = ex2(m_b - mn_b); m_b = mn_b; }
+        const float mu_a = (m_a == -INFINITY) ? 0.f : m_a;
+        const float mu_b = (m_b == -INFINITY) ? 0.f : m_b;
         float ps_a = 0.f, ps_b = 0.f;
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
@@ -319,10 +328,16 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
         }
         l_a = fmaf(l_a, al_a, ps_a);
         l_b = fmaf(l_b, al_b, ps_b);
+        if (__any_sync(0xffffffffu, up_a || up_b)) {
 #pragma unroll
-        for (int jj = 0; jj < D / 8; ++jj) {
-            o[jj][0] *= al_a; o[jj][1] *= al_a;
-            o[jj][2] *= al_b; o[jj][3] *= al_b;
+            for (int jj = 0; jj < D / 8; ++jj) {
+                o[jj][0] *= al_a; o[jj][1] *= al_a;
+                o[jj][2] *= al_b; o[jj][3] *= al_b;
+            }
+            if constexpr (INT8) {
+                osum[0] *= al_a; osum[1] *= al_a;
+                osum[2] *= al_b; osum[3] *= al_b;
+            }
         }
         using PT = typename std::conditional<INT8, __half, T>::type;
         uint32_t pa[4];
@@ -372,11 +387,16 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
                 const uint32_t x23 = prmt(w0, w1, 0x7362u) ^ 0x80808080u;
                 const uint32_t y01 = prmt(w2, w3, 0x5140u) ^ 0x80808080u;
                 const uint32_t y23 = prmt(w2, w3, 0x7362u) ^ 0x80808080u;
-                mma_16816<false>(o[4 * i + 0], pa, i8pair_to_h2<0x4140>(x01), i8pair_to_h2<0x4140>(y01));
-                mma_16816<false>(o[4 * i + 1], pa, i8pair_to_h2<0x4342>(x01), i8pair_to_h2<0x4342>(y01));
-                mma_16816<false>(o[4 * i + 2], pa, i8pair_to_h2<0x4140>(x23), i8pair_to_h2<0x4140>(y23));
-                mma_16816<false>(o[4 * i + 3], pa, i8pair_to_h2<0x4342>(x23), i8pair_to_h2<0x4342>(y23));
+                // values as f16 (1152 + v), exact; the bias is removed at the end
+                const uint32_t F = 0x64646464u;
+                mma_16816<false>(o[4 * i + 0], pa, prmt(x01, F, 0x4140u), prmt(y01, F, 0x4140u));
+                mma_16816<false>(o[4 * i + 1], pa, prmt(x01, F, 0x4342u), prmt(y01, F, 0x4342u));
+                mma_16816<false>(o[4 * i + 2], pa, prmt(x23, F, 0x4140u), prmt(y23, F, 0x4140u));
+                mma_16816<false>(o[4 * i + 3], pa, prmt(x23, F, 0x4342u), prmt(y23, F, 0x4342u));
             }
+            // sum_t p~_t per row with the same rounding and accumulation as O
+            const uint32_t ones = 0x3C003C00u;   // f16x2 (1, 1)
+            mma_16816<false>(osum, pa, ones, ones);
         }
 
         __syncwarp();
@@ -410,8 +430,13 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
                 // n-tile jj = 4i + q covers dims 32i + 4n + q for column n
                 d = (jj >> 2) * 32 + 4 * (2 * c + e) + (jj & 3);
             }
-            oww[ra * D + d] = o[jj][e];
-            oww[rb * D + d] = o[jj][2 + e];
+            if constexpr (INT8) {
+                oww[ra * D + d] = fmaf(-1152.0f, osum[0], o[jj][e]);
+                oww[rb * D + d] = fmaf(-1152.0f, osum[2], o[jj][2 + e]);
+            } else {
+                oww[ra * D + d] = o[jj][e];
+                oww[rb * D + d] = o[jj][2 + e];
+            }
         }
     }
     if (c == 0) {
@@ -443,49 +468,49 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
 
 // ---------------------------------------------------------------------------
 template <typename T, int D, bool INT8>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(D)
 fia_combine_kernel(const __grid_constant__ CombineArgs a) {
+    // one CTA per (sequence, kv head, row); one thread per channel d
     const CombineItem it = a.items[blockIdx.x];
     const SeqInfo si = a.c.seq[it.b];
     const int g = a.c.g;
-    const int R = si.qlen * g;
+    const int row = blockIdx.y;
+    if (row >= si.qlen * g) return;
+    const int d = threadIdx.x;
+    const int head = it.kvh * g + row % g;
+    const int token = si.cu_q + row / g;
     T *out = reinterpret_cast<T *>(a.c.out);
-    for (int idx = threadIdx.x; idx < R * D; idx += blockDim.x) {
-        const int row = idx / D, d = idx % D;
-        const int head = it.kvh * g + row % g;
-        const int token = si.cu_q + row / g;
-        float M = -INFINITY;
-        for (int s = 0; s < it.nsplit; ++s)
-            M = fmaxf(M, a.part_ml[(int64_t)(it.slot0 + s) * kDecodeRows + row].x);
-        float val = 0.f, lse = INFINITY;
-        if (M != -INFINITY) {
-            const float sink2 = a.c.sink ? a.c.sink[head] * kLog2e : -INFINITY;
-            const float M2 = fmaxf(M, sink2);
-            float L = 0.f, acc = 0.f;
-            for (int s = 0; s < it.nsplit; ++s) {
-                const int64_t slot = it.slot0 + s;
-                const float2 ml = a.part_ml[slot * kDecodeRows + row];
-                if (ml.x == -INFINITY) continue;
-                const float f = ex2(ml.x - M2);
-                L = fmaf(ml.y, f, L);
-                acc = fmaf(a.part_o[(slot * kDecodeRows + row) * D + d], f, acc);
-            }
-            const float Lt = L + (a.c.sink ? ex2(sink2 - M2) : 0.f);
-            if constexpr (INT8) {
-                const float vs = a.v_scale[it.kvh * D + d];
-                const float vo = a.v_offset ? a.v_offset[it.kvh * D + d] : 0.f;
-                acc = vs * fmaf(vo, L, acc);
-            }
-            val = acc / Lt;
-            lse = (M2 + log2f(Lt)) * kLn2;
+    float M = -INFINITY;
+    for (int s = 0; s < it.nsplit; ++s)
+        M = fmaxf(M, a.part_ml[(int64_t)(it.slot0 + s) * kDecodeRows + row].x);
+    float val = 0.f, lse = INFINITY;
+    if (M != -INFINITY) {
+        const float sink2 = a.c.sink ? a.c.sink[head] * kLog2e : -INFINITY;
+        const float M2 = fmaxf(M, sink2);
+        float L = 0.f, acc = 0.f;
+        for (int s = 0; s < it.nsplit; ++s) {
+            const int64_t slot = it.slot0 + s;
+            const float2 ml = a.part_ml[slot * kDecodeRows + row];
+            if (ml.x == -INFINITY) continue;
+            const float f = ex2(ml.x - M2);
+            L = fmaf(ml.y, f, L);
+            acc = fmaf(a.part_o[(slot * kDecodeRows + row) * D + d], f, acc);
         }
-        if constexpr (MmaType<T>::bf16) {
-            out[((int64_t)token * a.c.H + head) * D + d] = __float2bfloat16_rn(val);
-        } else {
-            out[((int64_t)token * a.c.H + head) * D + d] = __float2half_rn(val);
+        const float Lt = L + (a.c.sink ? ex2(sink2 - M2) : 0.f);
+        if constexpr (INT8) {
+            const float vs = a.v_scale[it.kvh * D + d];
+            const float vo = a.v_offset ? a.v_offset[it.kvh * D + d] : 0.f;
+            acc = vs * fmaf(vo, L, acc);
         }
-        if (d == 0 && a.c.lse) a.c.lse[(int64_t)token * a.c.H + head] = lse;
+        val = acc / Lt;
+        lse = (M2 + log2f(Lt)) * kLn2;
     }
+    if constexpr (MmaType<T>::bf16) {
+        out[((int64_t)token * a.c.H + head) * D + d] = __float2bfloat16_rn(val);
+    } else {
+        out[((int64_t)token * a.c.H + head) * D + d] = __float2half_rn(val);
+    }
+    if (d == 0 && a.c.lse) a.c.lse[(int64_t)token * a.c.H + head] = lse;
 }
 
 // ---------------------------------------------------------------------------
@@ -517,7 +542,7 @@ cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap &tk, const CUte
 
 template <typename T, int D, bool INT8>
 static cudaError_t launch_combine_t(const CombineArgs &a, int grid, cudaStream_t s) {
-    fia_combine_kernel<T, D, INT8><<<grid, 128, 0, s>>>(a);
+    fia_combine_kernel<T, D, INT8><<<dim3(grid, kDecodeRows), D, 0, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -308,19 +308,6 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return r;
 }
 
-// Two int8 lanes -> f16x2, exactly.  `u` holds the bytes already biased by
-// +128 (x ^ 0x80); byte selectors pick the two bytes.  Placing a byte under
-// the f16 exponent pattern 0x64 gives 1024 + byte; subtracting 1152 leaves
-// the signed value (all integers in [-128, 127] are exact in f16).
-template <uint32_t SEL>
-__device__ __forceinline__ uint32_t i8pair_to_h2(uint32_t u) {
-    uint32_t h = prmt(u, 0x64646464u, SEL);
-    uint32_t r;
-    const uint32_t bias = 0x64806480u;   // f16x2 (1152, 1152)
-    asm("sub.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h), "r"(bias));
-    return r;
-}
-
 // ---------------------------------------------------------------------------
 // Numerics.
 // ---------------------------------------------------------------------------

@@ -50,6 +50,8 @@ struct fia_op {
     int64_t work_items = 0;
     int32_t split_tokens = 0;
     cudaEvent_t ev_start = nullptr, ev_stop = nullptr;
+    // prefill plans small enough to travel as a kernel parameter
+    PlanBytes<kInlinePlanBytes> *inline_plan = nullptr;
 };
 
 namespace {
@@ -471,6 +473,18 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
         std::memcpy(host.data() + o->off_seq, seq.data(), sizeof(SeqInfo) * batch);
         std::memcpy(host.data() + o->off_cta, cta_off.data(), sizeof(int32_t) * (grid + 1));
         std::memcpy(host.data() + o->off_items, flat.data(), sizeof(PrefillItem) * flat.size());
+        if (o->plan_bytes <= (size_t)kInlinePlanBytes) {
+            // the plan rides in the launch parameters; the workspace keeps only
+            // the error words (cleared by the kernel itself)
+            o->inline_plan = new PlanBytes<kInlinePlanBytes>();
+            std::memset(o->inline_plan->b, 0, sizeof(o->inline_plan->b));
+            std::memcpy(o->inline_plan->b, host.data(), o->plan_bytes);
+            o->off_err = 0;
+            o->ws_size = align_up(kErrRegionBytes, 256);
+            *workspaceSize = o->ws_size;
+            *op = o;
+            return FIA_OK;
+        }
     }
     if (cudaMallocHost(reinterpret_cast<void **>(&o->plan_host), o->plan_bytes) != cudaSuccess) {
         cudaGetLastError();
@@ -491,7 +505,8 @@ fia_status fia_run(void *workspace, uint64_t workspaceSize, fia_op *op, void *st
         return FIA_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_ptr);
     uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
-    if (cudaMemcpyAsync(ws, op->plan_host, op->plan_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+    if (!op->inline_plan &&
+        cudaMemcpyAsync(ws, op->plan_host, op->plan_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
         cudaGetLastError();
         return FIA_ERR_CUDA;
     }
@@ -527,9 +542,13 @@ fia_status fia_run(void *workspace, uint64_t workspaceSize, fia_op *op, void *st
     } else {
         PrefillArgs p{};
         p.c = c;
-        p.cta_off = reinterpret_cast<const int32_t *>(ws + op->off_cta);
-        p.items = reinterpret_cast<const PrefillItem *>(ws + op->off_items);
-        if (op->grid > 0) e = launch_prefill(p, op->tq, op->tk, op->tv, op->q_dtype, op->grid, s);
+        p.plan = op->inline_plan ? nullptr : ws;
+        p.off_seq = (int32_t)op->off_seq;
+        p.off_cta = (int32_t)op->off_cta;
+        p.off_items = (int32_t)op->off_items;
+        if (op->grid > 0)
+            e = launch_prefill(p, op->tq, op->tk, op->tv, op->q_dtype, op->grid,
+                               op->inline_plan ? op->inline_plan->b : nullptr, s);
     }
     if (e != cudaSuccess) {
         cudaGetLastError();
@@ -622,6 +641,7 @@ fia_status fia_decode_run_static(fia_op *op, void *stream_ptr) {
 void fia_op_destroy(fia_op *op) {
     if (!op) return;
     if (op->plan_host) cudaFreeHost(op->plan_host);
+    delete op->inline_plan;
     delete op;
 }
 

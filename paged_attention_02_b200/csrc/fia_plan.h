@@ -79,8 +79,17 @@ struct CombineArgs {
 
 struct PrefillArgs {
     CommonArgs c;
-    const int32_t *cta_off;        // [grid + 1]
-    const PrefillItem *items;
+    // Plan location: either the workspace (device pointer `plan`) or the
+    // kernel's inline plan parameter; offsets are bytes from the plan start.
+    const uint8_t *plan;
+    int32_t off_seq, off_cta, off_items;
+};
+
+// A plan of at most this many bytes travels as a kernel parameter (no
+// host-to-device copy per run).
+constexpr int kInlinePlanBytes = 24576;
+template <int N> struct PlanBytes {
+    uint8_t b[N];
 };
 
 // Kernel launchers (defined in the .cu files).
@@ -88,8 +97,10 @@ cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap &tk, const CUte
                           int q_dtype, bool kv_int8, int grid, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs &a, int q_dtype, bool kv_int8, int grid,
                            cudaStream_t s);
+// inline_plan: nullptr (plan in the workspace) or kInlinePlanBytes of host data.
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tq, const CUtensorMap &tk,
-                           const CUtensorMap &tv, int q_dtype, int grid, cudaStream_t s);
+                           const CUtensorMap &tv, int q_dtype, int grid, const uint8_t *inline_plan,
+                           cudaStream_t s);
 int decode_smem_bytes(int D, bool kv_int8);
 int prefill_smem_bytes(int D);
 

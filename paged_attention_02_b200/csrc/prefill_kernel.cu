@@ -78,9 +78,10 @@ struct PairGeom {
     int nA, nB;   // key tiles of tile 0 (0 if absent) and tile 1; nA <= nB
 };
 
-__device__ __forceinline__ PairGeom pair_geom(const PrefillArgs &a, int idx) {
-    const PrefillItem it = a.items[idx];
-    const SeqInfo si = a.c.seq[it.b];
+__device__ __forceinline__ PairGeom pair_geom(const PrefillArgs &a, const PrefillItem *items,
+                                              const SeqInfo *seqs, int idx) {
+    const PrefillItem it = items[idx];
+    const SeqInfo si = seqs[it.b];
     const bool causal = (a.c.mask_type == 9 || a.c.mask_type == 3);
     PairGeom g;
     g.b = it.b; g.kvh = it.kvh; g.cu_q = si.cu_q; g.qlen = si.qlen; g.kvlen = si.kvlen;
@@ -113,10 +114,11 @@ enum { kModePlain = 0, kModeAlibi = 1, kModePse = 2 };
         }                                                                                 \
     } while (0)
 
-template <typename T, int D, int MODE>
+template <typename T, int D, int MODE, int PB>
 __global__ void __launch_bounds__(320, 1)
 fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tq,
-                   const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv) {
+                   const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                   const __grid_constant__ PlanBytes<PB> pl) {
     using Cfg = PrefillCfg<D>;
     constexpr int KS = Cfg::kKStages, VS = Cfg::kVStages;
     constexpr bool BF = MmaType<T>::bf16;
@@ -144,6 +146,12 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     const int warp = tid >> 5;
     const int lane = tid & 31;
 
+    if (PB >= kInlinePlanBytes && blockIdx.x == 0 && tid == 0 && a.c.err) {
+        // nothing clears the error words per run on this path; a wait can
+        // only give up seconds after this store
+        a.c.err[0] = 0u;
+        a.c.err[1] = 0u;
+    }
     if (tid == 0) {
         mbar_init(q_full, 1);
         mbar_init(q_empty, 1);
@@ -172,8 +180,13 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     int dbg_j = -1;     // tile index recorded in failure trails
     int idx = -1;
 
-    const int it_begin = a.cta_off[blockIdx.x];
-    const int it_end = a.cta_off[blockIdx.x + 1];
+    // the plan: inline kernel parameter, or the workspace copy
+    const uint8_t *plan = (PB >= kInlinePlanBytes) ? pl.b : a.plan;
+    const SeqInfo *seqs = reinterpret_cast<const SeqInfo *>(plan + a.off_seq);
+    const int32_t *cta_off = reinterpret_cast<const int32_t *>(plan + a.off_cta);
+    const PrefillItem *items = reinterpret_cast<const PrefillItem *>(plan + a.off_items);
+    const int it_begin = cta_off[blockIdx.x];
+    const int it_end = cta_off[blockIdx.x + 1];
     const uint32_t sm_q = smem_u32(smem + Cfg::kOffQ);
     const uint32_t sm_k0 = smem_u32(smem + Cfg::kOffK);
     const uint32_t sm_v0 = smem_u32(smem + Cfg::kOffV);
@@ -184,7 +197,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             uint32_t q_it = 0, kv_it = 0;
             const int br = a.c.box_rows;
             for (idx = it_begin; idx < it_end; ++idx) {
-                const PairGeom gm = pair_geom(a, idx);
+                const PairGeom gm = pair_geom(a, items, seqs, idx);
                 if (gm.nB == 0) continue;
                 FIA_WAIT(q_empty, (q_it & 1) ^ 1, 10);
                 mbar_arrive_expect_tx(q_full, (gm.t[0].valid ? 2 : 1) * Cfg::kTileBytes);
@@ -249,7 +262,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                         (acc || kk > 0) ? 1u : 0u);
         };
         for (idx = it_begin; idx < it_end; ++idx) {
-            const PairGeom gm = pair_geom(a, idx);
+            const PairGeom gm = pair_geom(a, items, seqs, idx);
             if (gm.nB == 0) continue;
             dbg_j = -1;
             FIA_WAIT(q_full, q_it & 1, 20);
@@ -353,7 +366,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         uint32_t s_it = 0, p_it = 0, o_it = 0;
         T *outp = reinterpret_cast<T *>(a.c.out);
         for (idx = it_begin; idx < it_end; ++idx) {
-            const PairGeom gm = pair_geom(a, idx);
+            const PairGeom gm = pair_geom(a, items, seqs, idx);
             const SubGeom sg = gm.t[X];
             if (!sg.valid) continue;
             const int i = sg.q0 + row;
@@ -587,33 +600,44 @@ done:
 template <typename T, int D, int MODE>
 static cudaError_t launch_prefill_t(const PrefillArgs &a, const CUtensorMap &tq,
                                     const CUtensorMap &tk, const CUtensorMap &tv, int grid,
-                                    cudaStream_t s) {
-    auto kern = fia_prefill_kernel<T, D, MODE>;
+                                    const uint8_t *inline_plan, cudaStream_t s) {
     const int smem = PrefillCfg<D>::kSmem;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    kern<<<grid, PrefillCfg<D>::kThreads, smem, s>>>(a, tq, tk, tv);
+    if (inline_plan) {
+        auto kern = fia_prefill_kernel<T, D, MODE, kInlinePlanBytes>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        // inline_plan points at a full PlanBytes<kInlinePlanBytes> kept by the op
+        kern<<<grid, PrefillCfg<D>::kThreads, smem, s>>>(
+            a, tq, tk, tv, *reinterpret_cast<const PlanBytes<kInlinePlanBytes> *>(inline_plan));
+    } else {
+        auto kern = fia_prefill_kernel<T, D, MODE, 16>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        PlanBytes<16> pl{};
+        kern<<<grid, PrefillCfg<D>::kThreads, smem, s>>>(a, tq, tk, tv, pl);
+    }
     return cudaGetLastError();
 }
 
 template <typename T, int D>
 static cudaError_t launch_prefill_mode(const PrefillArgs &a, const CUtensorMap &tq,
                                        const CUtensorMap &tk, const CUtensorMap &tv, int grid,
-                                       cudaStream_t s) {
-    if (a.c.pse) return launch_prefill_t<T, D, kModePse>(a, tq, tk, tv, grid, s);
-    if (a.c.mask_type == 3) return launch_prefill_t<T, D, kModeAlibi>(a, tq, tk, tv, grid, s);
-    return launch_prefill_t<T, D, kModePlain>(a, tq, tk, tv, grid, s);
+                                       const uint8_t *ip, cudaStream_t s) {
+    if (a.c.pse) return launch_prefill_t<T, D, kModePse>(a, tq, tk, tv, grid, ip, s);
+    if (a.c.mask_type == 3) return launch_prefill_t<T, D, kModeAlibi>(a, tq, tk, tv, grid, ip, s);
+    return launch_prefill_t<T, D, kModePlain>(a, tq, tk, tv, grid, ip, s);
 }
 
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tq, const CUtensorMap &tk,
-                           const CUtensorMap &tv, int q_dtype, int grid, cudaStream_t s) {
+                           const CUtensorMap &tv, int q_dtype, int grid, const uint8_t *inline_plan,
+                           cudaStream_t s) {
     const bool bf = (q_dtype == 1);
     if (a.c.D == 128)
-        return bf ? launch_prefill_mode<__nv_bfloat16, 128>(a, tq, tk, tv, grid, s)
-                  : launch_prefill_mode<__half, 128>(a, tq, tk, tv, grid, s);
+        return bf ? launch_prefill_mode<__nv_bfloat16, 128>(a, tq, tk, tv, grid, inline_plan, s)
+                  : launch_prefill_mode<__half, 128>(a, tq, tk, tv, grid, inline_plan, s);
     if (a.c.D == 64)
-        return bf ? launch_prefill_mode<__nv_bfloat16, 64>(a, tq, tk, tv, grid, s)
-                  : launch_prefill_mode<__half, 64>(a, tq, tk, tv, grid, s);
+        return bf ? launch_prefill_mode<__nv_bfloat16, 64>(a, tq, tk, tv, grid, inline_plan, s)
+                  : launch_prefill_mode<__half, 64>(a, tq, tk, tv, grid, inline_plan, s);
     return cudaErrorInvalidValue;
 }
 
