@@ -11,20 +11,22 @@
 // One persistent CTA per SM walks a host-planned, longest-first list of tile
 // PAIRS: two 128-token tiles that read the same KV head (two heads of one GQA
 // group, or two consecutive tiles of one head), so every K/V tile fetched
-// serves 2 x 128 query rows.  Warp roles (10 warps):
+// serves 2 x 128 query rows.  Warp roles (18 warps):
 //   warp 0     TMA producer: both Q tiles once per pair, then K and V tiles
 //              of 128 keys, each gathered block by block through the block
-//              table (3-stage K ring, 2-stage V ring, 128-byte swizzle).
+//              table (2-stage K and V rings, 128-byte swizzle).
 //   warp 1     UMMA issuer (one lane): S_X = Q_X K_j^T into TMEM, and
 //              O_X += P_X V_j with P_X read from TMEM (TS form).  One thread's
 //              tcgen05.mma ops run in issue order, so QK_X(j+1) may be issued
 //              right after PV_X(j) over the same TMEM columns.  It zeroes the V
 //              rows past kvSeqLen in a ragged last tile.
-//   warps 2-5  softmax + epilogue of tile 0, warps 6-9 of tile 1: one query
-//              row per thread (TMEM lane), S row -> registers, scale / mask /
-//              bias, online softmax in fp32 (log2 domain; O rescaled in TMEM
-//              only when the running max grows by more than 2^8), P in the
-//              input dtype written back over S; at the end O / l, sink, lse.
+//   warps 2-9  softmax + epilogue of tile 0, warps 10-17 of tile 1: each query
+//              row is shared by two warps (same TMEM lanes, 64 key columns
+//              each; they swap row maxima through shared memory), S ->
+//              registers, scale / mask / bias, online softmax in fp32 (log2
+//              domain; O rescaled in TMEM only when the running max grows by
+//              more than 2^8), P in the input dtype written back over S; at
+//              the end O / l, sink, lse (each warp writes half of the row).
 // TMEM (512 columns): S_0 | S_1 | O_0 | O_1.  While one softmax group works on
 // its S, the tensor core runs the other tile's PV and QK^T.
 // Every mbarrier wait is bounded in time (see fia_device.cuh).
@@ -44,22 +46,26 @@ struct PrefillCfg {
     static constexpr int kHalves = D / 64;                 // 128-byte column groups
     static constexpr int kTileBytes = 128 * D * 2;         // Q, K or V tile (128 rows)
     static constexpr int kGroupBytes = 128 * 128;          // one 128-row x 128-byte group
-    static constexpr int kKStages = 3;
+    static constexpr int kKStages = 2;
     static constexpr int kVStages = 2;
     static constexpr int kOffQ = 0;                                    // Q[2]
     static constexpr int kOffK = kOffQ + 2 * kTileBytes;               // K[s]
     static constexpr int kOffV = kOffK + kKStages * kTileBytes;        // V[s]
-    static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
+    // row-max / row-sum exchange between the two warps sharing a TMEM lane
+    // quadrant: [parity][tile X][quadrant][column half][lane] floats
+    static constexpr int kOffX = kOffV + kVStages * kTileBytes;
+    static constexpr int kXBytes = 2 * 2 * 4 * 2 * 32 * 4;
+    static constexpr int kOffBar = kOffX + kXBytes;
     // q_full, q_empty, k_full/k_empty[KS], v_full/v_empty[VS],
-    // s_full[2], p_full[2], pv_done[2], o_full[2]
-    static constexpr int kNumBar = 2 + 2 * kKStages + 2 * kVStages + 8;
+    // s_full[2], p_full[2], pv_done[2], o_full[2], xch[2][4]
+    static constexpr int kNumBar = 2 + 2 * kKStages + 2 * kVStages + 8 + 8;
     static constexpr int kUsed = kOffBar + kNumBar * 8 + 16;
     // Keep one CTA per SM (each CTA holds all 512 TMEM columns).
     static constexpr int kSmem = 1024 + (kUsed > 118 * 1024 ? kUsed : 118 * 1024);
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t col_s(int x) { return (uint32_t)x * 128u; }
     static constexpr uint32_t col_o(int x) { return 256u + (uint32_t)x * D; }
-    static constexpr int kThreads = 320;
+    static constexpr int kThreads = 576;   // producer, UMMA, 2 x 8 softmax warps
 };
 
 int prefill_smem_bytes(int D) {
@@ -115,7 +121,7 @@ enum { kModePlain = 0, kModeAlibi = 1, kModePse = 2 };
     } while (0)
 
 template <typename T, int D, int MODE, int PB>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(576, 1)
 fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tq,
                    const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                    const __grid_constant__ PlanBytes<PB> pl) {
@@ -139,6 +145,8 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     uint64_t *p_full = s_full + 2;          // [2]  P_X written (4 warps)
     uint64_t *pv_done = p_full + 2;         // [2]  PV_X done
     uint64_t *o_full = pv_done + 2;         // [2]  last PV_X of the pair done
+    uint64_t *xch = o_full + 2;             // [2][4] max / sum exchange (2 warps)
+    float *xbuf = reinterpret_cast<float *>(smem + Cfg::kOffX);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + Cfg::kNumBar);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -159,10 +167,11 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         for (int s = 0; s < VS; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
         for (int x = 0; x < 2; ++x) {
             mbar_init(&s_full[x], 1);
-            mbar_init(&p_full[x], 4);
+            mbar_init(&p_full[x], 8);
             mbar_init(&pv_done[x], 1);
             mbar_init(&o_full[x], 1);
         }
+        for (int x = 0; x < 8; ++x) mbar_init(&xch[x], 2);
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tq);
@@ -352,19 +361,42 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         }
     } else {
         // ------------------------------------------------------------ softmax + epilogue
-        const int X = (warp - 2) >> 2;             // which tile of the pair
+        // 8 warps per tile: warp (quadrant q, half h) owns query rows
+        // 32q..32q+31 (its TMEM lanes) and key columns 64h..64h+63 of S.
+        const int sw = warp - 2;
+        const int X = sw >> 3;                     // which tile of the pair
+        const int half = (sw >> 2) & 1;            // which 64 columns
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
-        const uint32_t scol = t_lane + Cfg::col_s(X);
-        const uint32_t ocol = t_lane + Cfg::col_o(X);
+        const uint32_t scol = t_lane + Cfg::col_s(X) + 64 * half;      // S columns
+        const uint32_t pcol = t_lane + Cfg::col_s(X) + 32 * half;      // P columns (2 keys each)
+        constexpr int DH = D / 2;                                      // O columns per warp
+        const uint32_t ocol = t_lane + Cfg::col_o(X) + DH * half;
+        uint64_t *xb = &xch[X * 4 + quad];
+        float *xmine = xbuf + ((X * 4 + quad) * 2 + half) * 32 + lane;     // + parity * 512
+        const float *xpeer = xbuf + ((X * 4 + quad) * 2 + (half ^ 1)) * 32 + lane;
         const bool causal = (a.c.mask_type == 9 || a.c.mask_type == 3);
         const float sl2 = a.c.scale_log2;
         // plain mode with a positive scale: mask raw scores and fold the scale
         // into the exponent (one FFMA per element)
         const bool fold = (MODE == kModePlain) && (sl2 > 0.f);
-        uint32_t s_it = 0, p_it = 0, o_it = 0;
+        uint32_t s_it = 0, p_it = 0, o_it = 0, x_it = 0;
         T *outp = reinterpret_cast<T *>(a.c.out);
+
+        // Exchange one float per row with the partner warp (bounded wait).
+#define FIA_EXCHANGE(val, out)                                                            \
+    do {                                                                                  \
+        const int _par = x_it & 1;                                                        \
+        xmine[_par * 512] = (val);                                                        \
+        __syncwarp();                                                                     \
+        if (lane == 0) mbar_arrive(xb);                                                   \
+        FIA_WAIT(xb, x_it & 1, 33);                                                       \
+        __syncwarp();                                                                     \
+        (out) = xpeer[_par * 512];                                                        \
+        ++x_it;                                                                           \
+    } while (0)
+
         for (idx = it_begin; idx < it_end; ++idx) {
             const PairGeom gm = pair_geom(a, items, seqs, idx);
             const SubGeom sg = gm.t[X];
@@ -375,9 +407,9 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             const int64_t orow = ((int64_t)(gm.cu_q + i) * a.c.H + sg.h);
             if (sg.n == 0) {
                 if (valid) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(outp + orow * D);
-                    for (int x = 0; x < D * 2 / 16; ++x) dst[x] = make_uint4(0, 0, 0, 0);
-                    if (a.c.lse) a.c.lse[orow] = INFINITY;
+                    uint4 *dst = reinterpret_cast<uint4 *>(outp + orow * D + DH * half);
+                    for (int x = 0; x < DH * 2 / 16; ++x) dst[x] = make_uint4(0, 0, 0, 0);
+                    if (a.c.lse && half == 0) a.c.lse[orow] = INFINITY;
                 }
                 __syncwarp();
                 continue;
@@ -393,24 +425,24 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             float m = -INFINITY, l = 0.f;
             for (int j = 0; j < sg.n; ++j) {
                 dbg_j = j;
-                const int tb = j * kPrefillBN;
+                const int tb = j * kPrefillBN + 64 * half;     // first key of this warp
                 FIA_WAIT(&s_full[X], s_it & 1, 30);
                 ++s_it;
                 __syncwarp();          // tcgen05.ld/st below are warp-collective (.aligned)
                 tc_fence_after();
-                uint32_t sr[4][32];
+                uint32_t sr[2][32];
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) tmem_ld32(scol + cc * 32, sr[cc]);
+                for (int cc = 0; cc < 2; ++cc) tmem_ld32(scol + cc * 32, sr[cc]);
                 tmem_ld_wait();
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) reg_fence32(sr[cc]);
+                for (int cc = 0; cc < 2; ++cc) reg_fence32(sr[cc]);
 
                 // ---- scores (log2 units unless folded), bias, masks ----
-                const bool edge = (tb + kPrefillBN > gm.kvlen) || (causal && tb + kPrefillBN - 1 > qpos);
+                const bool edge = (tb + 64 > gm.kvlen) || (causal && tb + 63 > qpos);
                 if constexpr (MODE == kModeAlibi) {
                     const float base = slope2 * (float)(tb - qpos);
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc)
+                    for (int cc = 0; cc < 2; ++cc)
 #pragma unroll
                         for (int x = 0; x < 32; ++x) {
                             const float bias = fmaf(slope2, (float)(cc * 32 + x), base);
@@ -418,7 +450,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                         }
                 } else if constexpr (MODE == kModePse) {
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
+                    for (int cc = 0; cc < 2; ++cc) {
 #pragma unroll
                         for (int x8 = 0; x8 < 4; ++x8) {
                             const int t = tb + cc * 32 + x8 * 8;
@@ -442,14 +474,14 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                     __syncwarp();      // reconverge after the per-row pse loads
                 } else if (!fold) {
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc)
+                    for (int cc = 0; cc < 2; ++cc)
 #pragma unroll
                         for (int x = 0; x < 32; ++x)
                             sr[cc][x] = __float_as_uint(__uint_as_float(sr[cc][x]) * sl2);
                 }
                 if (edge) {
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc)
+                    for (int cc = 0; cc < 2; ++cc)
 #pragma unroll
                         for (int x = 0; x < 32; ++x) {
                             const int t = tb + cc * 32 + x;
@@ -457,19 +489,23 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                             if (!keep) sr[cc][x] = __float_as_uint(-INFINITY);
                         }
                 }
-                // tree max: 8 independent chains of 3-input max
+                // tree max over this warp's 64 columns, then with the partner's
 #define FIA_EL(e) __uint_as_float(sr[(e) >> 5][(e) & 31])
-                float mx8[8];
+                float mx4[4];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(FIA_EL(k), FIA_EL(k + 8));
+                for (int k = 0; k < 4; ++k) mx4[k] = fmaxf(FIA_EL(k), FIA_EL(k + 4));
 #pragma unroll
-                for (int e = 16; e < 128; e += 16)
+                for (int e = 8; e < 64; e += 8)
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) mx8[k] = fmax3(mx8[k], FIA_EL(e + k), FIA_EL(e + 8 + k));
+                    for (int k = 0; k < 4; ++k) mx4[k] = fmax3(mx4[k], FIA_EL(e + k), FIA_EL(e + 4 + k));
 #undef FIA_EL
-                float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                                 fmaxf(mx8[6], mx8[7]));
+                float mx = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
                 if (fold) mx = (mx == -INFINITY) ? -INFINITY : mx * sl2;
+                {
+                    float mp;
+                    FIA_EXCHANGE(mx, mp);
+                    mx = fmaxf(mx, mp);
+                }
 
                 // running max: exact on the first tile, afterwards raised only
                 // when it grows by more than 2^8 (O and l stay consistent with m)
@@ -486,18 +522,14 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 }
                 const float mu = (m == -INFINITY) ? 0.f : m;
 
-                // P = 2^(s - m) in the input dtype, stored over S's first 64
-                // columns; pairs of columns go through f32x2 math.  (Moving a
-                // share of the exponentials to the FMA-pipe polynomial
-                // exp2_poly_x2 measured slower here: the loop is latency-bound,
-                // not MUFU-throughput-bound, at this warp count.)
+                // P = 2^(s - m) in the input dtype over this warp's part of S
                 const uint64_t negmu2 = f2pack(-mu, -mu);
                 const uint64_t sl2x2 = f2pack(sl2, sl2);
                 uint64_t acc2[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) acc2[k] = f2pack(0.f, 0.f);
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
+                for (int cc = 0; cc < 2; ++cc) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int x = 0; x < 16; ++x) {
@@ -512,7 +544,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                         f2unpack(pp, p0, p1);
                         pk[x] = pack2<T>(p0, p1);
                     }
-                    tmem_st16(scol + cc * 16, pk);
+                    tmem_st16(pcol + cc * 16, pk);
                 }
                 {
                     const uint64_t s01 = fadd2(fadd2(acc2[0], acc2[1]), fadd2(acc2[2], acc2[3]));
@@ -521,10 +553,10 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                     l += l0 + l1;
                 }
 
-                // Rescale O (rare).  The previous PV of this tile must be done
-                // with O first.  (The softmax warps cannot drift apart: S for
-                // the next key tile is only produced after all four warps have
-                // signalled this P, so p_full phases never mix tiles.)
+                // Rescale this warp's half of O (rare).  The previous PV of this
+                // tile must be done with O first.  (The softmax warps cannot
+                // drift apart: S for the next key tile is only produced after
+                // all eight warps have signalled this P.)
                 if (__any_sync(0xffffffffu, need)) {
                     if (j > 0) {
                         FIA_WAIT(&pv_done[X], (p_it - 1) & 1, 31);
@@ -532,7 +564,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                         tc_fence_after();
                     }
 #pragma unroll
-                    for (int cc = 0; cc < D / 32; ++cc) {
+                    for (int cc = 0; cc < DH / 32; ++cc) {
                         uint32_t orr[32];
                         tmem_ld32(ocol + cc * 32, orr);
                         tmem_ld_wait();
@@ -550,8 +582,13 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 ++p_it;
             }
 
-            // ---- epilogue: O / l (+ sink), lse ----
+            // ---- epilogue: O / l (+ sink), lse; this warp writes D/2 columns ----
             dbg_j = sg.n;
+            {
+                float lp;
+                FIA_EXCHANGE(l, lp);
+                l += lp;
+            }
             FIA_WAIT(&o_full[X], o_it & 1, 32);
             ++o_it;
             __syncwarp();
@@ -565,7 +602,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             }
             const float oscale = ex2(mu - M) / lt;
 #pragma unroll
-            for (int cc = 0; cc < D / 32; ++cc) {
+            for (int cc = 0; cc < DH / 32; ++cc) {
                 uint32_t orr[32];
                 tmem_ld32(ocol + cc * 32, orr);
                 tmem_ld_wait();
@@ -576,17 +613,18 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                     for (int x = 0; x < 16; ++x)
                         pk[x] = pack2<T>(__uint_as_float(orr[2 * x]) * oscale,
                                          __uint_as_float(orr[2 * x + 1]) * oscale);
-                    uint4 *dst = reinterpret_cast<uint4 *>(outp + orow * D + cc * 32);
+                    uint4 *dst = reinterpret_cast<uint4 *>(outp + orow * D + DH * half + cc * 32);
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
                         dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
                 }
                 __syncwarp();
             }
-            if (valid && a.c.lse) a.c.lse[orow] = (M + log2f(lt)) * kLn2;
+            if (valid && a.c.lse && half == 0) a.c.lse[orow] = (M + log2f(lt)) * kLn2;
             tc_fence_before();
             __syncwarp();
         }
+#undef FIA_EXCHANGE
     }
 done:
     tc_fence_before();
