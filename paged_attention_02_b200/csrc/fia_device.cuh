@@ -342,41 +342,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return d;
 }
 
-// 2^x for a pair of fp32 values on the FMA/ALU pipes (no MUFU), used for a
-// share of the softmax exponentials so that they do not all queue on the
-// special-function unit.  Method: x = n + f with n = round(x) obtained by
-// adding 1.5*2^23 (the sum's low mantissa bits hold n), f in [-1/2, 1/2];
-// 2^f by a degree-3 polynomial whose coefficients were fitted here to the
-// relative error of 2^f on [-1/2, 1/2] (least squares on Chebyshev nodes with
-// Lawson reweighting toward minimax; worst relative error 1.0e-4 evaluated in
-// fp32, below half an fp16 ulp); 2^n joins by an integer add to the exponent
-// field.  Because 1.5*2^23 has its low 9 bits clear, (bits(t) << 23) equals
-// n << 23 exactly, so the join is one integer multiply-add.  Inputs are
-// clamped at -126 (smaller results are negligible against the row sum >= 1;
-// -inf gives ~1e-38 instead of 0).
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
-    float x0, x1;
-    f2unpack(x2, x0, x1);
-    x2 = f2pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
-    const uint64_t kShift = f2pack(12582912.0f, 12582912.0f);
-    const uint64_t kNegShift = f2pack(-12582912.0f, -12582912.0f);
-    const uint64_t kNegOne = f2pack(-1.0f, -1.0f);
-    const uint64_t t = fadd2(x2, kShift);            // round(x) in the low mantissa bits
-    const uint64_t r = fadd2(t, kNegShift);          // round(x) as a float
-    const uint64_t f = ffma2(r, kNegOne, x2);        // x - round(x) in [-1/2, 1/2]
-    uint64_t p = ffma2(f2pack(0.0550089031f, 0.0550089031f), f,
-                       f2pack(0.2422109693f, 0.2422109693f));
-    p = ffma2(p, f, f2pack(0.6932829618f, 0.6932829618f));
-    p = ffma2(p, f, f2pack(1.0f, 1.0f));
-    float p0, p1, t0, t1;
-    f2unpack(p, p0, p1);
-    f2unpack(t, t0, t1);
-    uint32_t r0, r1;
-    asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(r0) : "r"(__float_as_uint(t0)), "r"(__float_as_uint(p0)));
-    asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(r1) : "r"(__float_as_uint(t1)), "r"(__float_as_uint(p1)));
-    return f2pack(__uint_as_float(r0), __uint_as_float(r1));
-}
-
 template <typename T> __device__ __forceinline__ uint32_t pack2(float lo, float hi);
 template <> __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

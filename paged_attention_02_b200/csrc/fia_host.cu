@@ -37,7 +37,7 @@ struct fia_op {
     int32_t path = 0;          // 0 no-op, 1 decode, 2 prefill
     int32_t q_dtype = 0;       // 0 f16, 1 bf16
     bool kv_int8 = false;
-    CUtensorMap tq{}, tk{}, tv{};
+    CUtensorMap tq{}, tk{}, tv{}, tp{};
     CommonArgs common{};
     const float *k_scale = nullptr, *k_offset = nullptr, *v_scale = nullptr, *v_offset = nullptr;
     // plan, uploaded to the front of the workspace by every fia_run
@@ -321,6 +321,22 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
                   encode_3d(&o->tv, kdt, kv_es, value->data, D, kvHeadNum, nb * bs, box_inner, box_rows);
     if (!decode)
         enc_ok = enc_ok && encode_3d(&o->tq, tdt, 2, query->data, D, headNum, n_tokens, 64, kPrefillBM);
+    if (!decode && pse && (pse->dims[3] % 8) == 0 && aligned16(pse->data)) {
+        // pse viewed as {maxKV, maxQ, B*H}; one softmax warp fetches a
+        // {64 keys, 32 rows} box (128-byte swizzle)
+        auto fn = encode_fn();
+        cuuint64_t dims[3] = {(cuuint64_t)pse->dims[3], (cuuint64_t)pse->dims[2],
+                              (cuuint64_t)(pse->dims[0] * pse->dims[1])};
+        cuuint64_t strides[2] = {(cuuint64_t)pse->dims[3] * 2,
+                                 (cuuint64_t)(pse->dims[2] * pse->dims[3] * 2)};
+        cuuint32_t box[3] = {64, 32, 1};
+        cuuint32_t es[3] = {1, 1, 1};
+        enc_ok = enc_ok && fn &&
+                 fn(&o->tp, tdt, 3, pse->data, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+        c.pse_tma = 1;
+    }
     if (!enc_ok) {
         delete o;
         return FIA_ERR_CUDA;
@@ -547,7 +563,7 @@ fia_status fia_run(void *workspace, uint64_t workspaceSize, fia_op *op, void *st
         p.off_cta = (int32_t)op->off_cta;
         p.off_items = (int32_t)op->off_items;
         if (op->grid > 0)
-            e = launch_prefill(p, op->tq, op->tk, op->tv, op->q_dtype, op->grid,
+            e = launch_prefill(p, op->tq, op->tk, op->tv, op->tp, op->q_dtype, op->grid,
                                op->inline_plan ? op->inline_plan->b : nullptr, s);
     }
     if (e != cudaSuccess) {

@@ -56,6 +56,7 @@ struct CommonArgs {
     int32_t H, KVH, g, D, bs, box_rows;
     int32_t mask_type;
     int32_t pse_vec;        // pse rows 16-byte aligned (vector loads allowed)
+    int32_t pse_tma;        // prefill: pse boxes fetched by TMA (tensor map tp)
     float scale_log2;       // qkScale * log2(e)
 };
 
@@ -98,9 +99,10 @@ cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap &tk, const CUte
 cudaError_t launch_combine(const CombineArgs &a, int q_dtype, bool kv_int8, int grid,
                            cudaStream_t s);
 // inline_plan: nullptr (plan in the workspace) or kInlinePlanBytes of host data.
+// tp: pse tensor map (used when a.c.pse_tma).
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tq, const CUtensorMap &tk,
-                           const CUtensorMap &tv, int q_dtype, int grid, const uint8_t *inline_plan,
-                           cudaStream_t s);
+                           const CUtensorMap &tv, const CUtensorMap &tp, int q_dtype, int grid,
+                           const uint8_t *inline_plan, cudaStream_t s);
 int decode_smem_bytes(int D, bool kv_int8);
 int prefill_smem_bytes(int D);
 

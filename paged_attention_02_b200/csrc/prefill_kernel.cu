@@ -41,13 +41,16 @@
 
 namespace fia {
 
-template <int D>
+enum { kModePlain = 0, kModeAlibi = 1, kModePse = 2 };
+
+template <int D, int MODE = kModePlain>
 struct PrefillCfg {
     static constexpr int kHalves = D / 64;                 // 128-byte column groups
     static constexpr int kTileBytes = 128 * D * 2;         // Q, K or V tile (128 rows)
     static constexpr int kGroupBytes = 128 * 128;          // one 128-row x 128-byte group
-    static constexpr int kKStages = 2;
-    static constexpr int kVStages = 2;
+    // pse mode gives one K and one V stage to the per-warp pse slots
+    static constexpr int kKStages = (MODE == kModePse) ? 1 : 2;
+    static constexpr int kVStages = (MODE == kModePse) ? 1 : 2;
     static constexpr int kOffQ = 0;                                    // Q[2]
     static constexpr int kOffK = kOffQ + 2 * kTileBytes;               // K[s]
     static constexpr int kOffV = kOffK + kKStages * kTileBytes;        // V[s]
@@ -55,10 +58,14 @@ struct PrefillCfg {
     // quadrant: [parity][tile X][quadrant][column half][lane] floats
     static constexpr int kOffX = kOffV + kVStages * kTileBytes;
     static constexpr int kXBytes = 2 * 2 * 4 * 2 * 32 * 4;
-    static constexpr int kOffBar = kOffX + kXBytes;
+    // pse mode: one 32-row x 64-key pse box (4 KB, 128-byte swizzle) per
+    // softmax warp, fetched by that warp one key tile ahead
+    static constexpr int kOffPse = kOffX + kXBytes;
+    static constexpr int kPseBytes = (MODE == kModePse) ? 16 * 4096 : 0;
+    static constexpr int kOffBar = kOffPse + kPseBytes;
     // q_full, q_empty, k_full/k_empty[KS], v_full/v_empty[VS],
-    // s_full[2], p_full[2], pv_done[2], o_full[2], xch[2][4]
-    static constexpr int kNumBar = 2 + 2 * kKStages + 2 * kVStages + 8 + 8;
+    // s_full[2], p_full[2], pv_done[2], o_full[2], xch[2][4], pse_full[16]
+    static constexpr int kNumBar = 2 + 2 * kKStages + 2 * kVStages + 8 + 8 + 16;
     static constexpr int kUsed = kOffBar + kNumBar * 8 + 16;
     // Keep one CTA per SM (each CTA holds all 512 TMEM columns).
     static constexpr int kSmem = 1024 + (kUsed > 118 * 1024 ? kUsed : 118 * 1024);
@@ -69,8 +76,8 @@ struct PrefillCfg {
 };
 
 int prefill_smem_bytes(int D) {
-    if (D == 64) return PrefillCfg<64>::kSmem;
-    if (D == 128) return PrefillCfg<128>::kSmem;
+    if (D == 64) return PrefillCfg<64, kModePse>::kSmem;
+    if (D == 128) return PrefillCfg<128, kModePse>::kSmem;
     return -1;
 }
 
@@ -107,8 +114,6 @@ __device__ __forceinline__ PairGeom pair_geom(const PrefillArgs &a, const Prefil
     return g;
 }
 
-enum { kModePlain = 0, kModeAlibi = 1, kModePse = 2 };
-
 // Bounded wait; on failure lane 0 leaves a trail record (item, tile, parity).
 #define FIA_WAIT(bar, parity, where)                                                      \
     do {                                                                                  \
@@ -124,8 +129,8 @@ template <typename T, int D, int MODE, int PB>
 __global__ void __launch_bounds__(576, 1)
 fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tq,
                    const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
-                   const __grid_constant__ PlanBytes<PB> pl) {
-    using Cfg = PrefillCfg<D>;
+                   const __grid_constant__ CUtensorMap tp, const __grid_constant__ PlanBytes<PB> pl) {
+    using Cfg = PrefillCfg<D, MODE>;
     constexpr int KS = Cfg::kKStages, VS = Cfg::kVStages;
     constexpr bool BF = MmaType<T>::bf16;
     constexpr uint32_t IDESC_QK = umma_idesc_f16(BF, false, false, 128, kPrefillBN);
@@ -146,6 +151,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     uint64_t *pv_done = p_full + 2;         // [2]  PV_X done
     uint64_t *o_full = pv_done + 2;         // [2]  last PV_X of the pair done
     uint64_t *xch = o_full + 2;             // [2][4] max / sum exchange (2 warps)
+    uint64_t *pse_full = xch + 8;           // [16] per softmax warp (pse mode)
     float *xbuf = reinterpret_cast<float *>(smem + Cfg::kOffX);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + Cfg::kNumBar);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -172,11 +178,13 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             mbar_init(&o_full[x], 1);
         }
         for (int x = 0; x < 8; ++x) mbar_init(&xch[x], 2);
+        for (int x = 0; x < 16; ++x) mbar_init(&pse_full[x], 1);
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tq);
         tma_prefetch_desc(&tk);
         tma_prefetch_desc(&tv);
+        if (MODE == kModePse && a.c.pse_tma) tma_prefetch_desc(&tp);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, Cfg::kTmemCols);
@@ -381,8 +389,19 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         // plain mode with a positive scale: mask raw scores and fold the scale
         // into the exponent (one FFMA per element)
         const bool fold = (MODE == kModePlain) && (sl2 > 0.f);
-        uint32_t s_it = 0, p_it = 0, o_it = 0, x_it = 0;
+        uint32_t s_it = 0, p_it = 0, o_it = 0, x_it = 0, ps_it = 0;
         T *outp = reinterpret_cast<T *>(a.c.out);
+        const bool pse_tma = (MODE == kModePse) && a.c.pse_tma;
+        uint8_t *pslot = smem + Cfg::kOffPse + sw * 4096;
+        uint64_t *pbar = &pse_full[sw];
+        // lane 0 fetches this warp's pse box (32 rows x 64 keys) of key tile jt
+        auto pse_fetch = [&](const PairGeom &g2, const SubGeom &s2, int jt) {
+            if (lane == 0) {
+                mbar_arrive_expect_tx(pbar, 4096);
+                tma_load_3d(pslot, &tp, pbar, jt * kPrefillBN + 64 * half, s2.q0 + 32 * quad,
+                            g2.b * a.c.H + s2.h);
+            }
+        };
 
         // Exchange one float per row with the partner warp (bounded wait).
 #define FIA_EXCHANGE(val, out)                                                            \
@@ -423,6 +442,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                           (((int64_t)gm.b * a.c.H + sg.h) * a.c.pse_q + (valid ? i : 0)) * a.c.pse_kv;
             }
             float m = -INFINITY, l = 0.f;
+            if (pse_tma) pse_fetch(gm, sg, 0);
             for (int j = 0; j < sg.n; ++j) {
                 dbg_j = j;
                 const int tb = j * kPrefillBN + 64 * half;     // first key of this warp
@@ -448,6 +468,31 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                             const float bias = fmaf(slope2, (float)(cc * 32 + x), base);
                             sr[cc][x] = __float_as_uint(fmaf(__uint_as_float(sr[cc][x]), sl2, bias));
                         }
+                } else if (MODE == kModePse && pse_tma) {
+                    // this warp's pse box for tile j, 128-byte swizzled rows
+                    FIA_WAIT(pbar, ps_it & 1, 34);
+                    ++ps_it;
+                    const uint32_t prow = smem_u32(pslot) + lane * 128;
+#pragma unroll
+                    for (int c16 = 0; c16 < 8; ++c16) {
+                        uint32_t w4[4];
+                        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                                     : "=r"(w4[0]), "=r"(w4[1]), "=r"(w4[2]), "=r"(w4[3])
+                                     : "r"(prow + ((c16 ^ (lane & 7)) << 4)));
+                        const T *pv = reinterpret_cast<const T *>(w4);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int col = c16 * 8 + e;
+                            const float bias = to_f32<T>(pv[e]) * kLog2e;
+                            sr[col >> 5][col & 31] = __float_as_uint(
+                                fmaf(__uint_as_float(sr[col >> 5][col & 31]), sl2, bias));
+                        }
+                    }
+                    // the slot is free: fetch the next tile's box (generic-proxy
+                    // reads ordered before the async-proxy write)
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (j + 1 < sg.n) pse_fetch(gm, sg, j + 1);
                 } else if constexpr (MODE == kModePse) {
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
@@ -637,45 +682,47 @@ done:
 
 template <typename T, int D, int MODE>
 static cudaError_t launch_prefill_t(const PrefillArgs &a, const CUtensorMap &tq,
-                                    const CUtensorMap &tk, const CUtensorMap &tv, int grid,
+                                    const CUtensorMap &tk, const CUtensorMap &tv,
+                                    const CUtensorMap &tp, int grid,
                                     const uint8_t *inline_plan, cudaStream_t s) {
-    const int smem = PrefillCfg<D>::kSmem;
+    const int smem = PrefillCfg<D, MODE>::kSmem;
     if (inline_plan) {
         auto kern = fia_prefill_kernel<T, D, MODE, kInlinePlanBytes>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         // inline_plan points at a full PlanBytes<kInlinePlanBytes> kept by the op
-        kern<<<grid, PrefillCfg<D>::kThreads, smem, s>>>(
-            a, tq, tk, tv, *reinterpret_cast<const PlanBytes<kInlinePlanBytes> *>(inline_plan));
+        kern<<<grid, PrefillCfg<D, MODE>::kThreads, smem, s>>>(
+            a, tq, tk, tv, tp, *reinterpret_cast<const PlanBytes<kInlinePlanBytes> *>(inline_plan));
     } else {
         auto kern = fia_prefill_kernel<T, D, MODE, 16>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         PlanBytes<16> pl{};
-        kern<<<grid, PrefillCfg<D>::kThreads, smem, s>>>(a, tq, tk, tv, pl);
+        kern<<<grid, PrefillCfg<D, MODE>::kThreads, smem, s>>>(a, tq, tk, tv, tp, pl);
     }
     return cudaGetLastError();
 }
 
 template <typename T, int D>
 static cudaError_t launch_prefill_mode(const PrefillArgs &a, const CUtensorMap &tq,
-                                       const CUtensorMap &tk, const CUtensorMap &tv, int grid,
-                                       const uint8_t *ip, cudaStream_t s) {
-    if (a.c.pse) return launch_prefill_t<T, D, kModePse>(a, tq, tk, tv, grid, ip, s);
-    if (a.c.mask_type == 3) return launch_prefill_t<T, D, kModeAlibi>(a, tq, tk, tv, grid, ip, s);
-    return launch_prefill_t<T, D, kModePlain>(a, tq, tk, tv, grid, ip, s);
+                                       const CUtensorMap &tk, const CUtensorMap &tv,
+                                       const CUtensorMap &tp, int grid, const uint8_t *ip,
+                                       cudaStream_t s) {
+    if (a.c.pse) return launch_prefill_t<T, D, kModePse>(a, tq, tk, tv, tp, grid, ip, s);
+    if (a.c.mask_type == 3) return launch_prefill_t<T, D, kModeAlibi>(a, tq, tk, tv, tp, grid, ip, s);
+    return launch_prefill_t<T, D, kModePlain>(a, tq, tk, tv, tp, grid, ip, s);
 }
 
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tq, const CUtensorMap &tk,
-                           const CUtensorMap &tv, int q_dtype, int grid, const uint8_t *inline_plan,
-                           cudaStream_t s) {
+                           const CUtensorMap &tv, const CUtensorMap &tp, int q_dtype, int grid,
+                           const uint8_t *inline_plan, cudaStream_t s) {
     const bool bf = (q_dtype == 1);
     if (a.c.D == 128)
-        return bf ? launch_prefill_mode<__nv_bfloat16, 128>(a, tq, tk, tv, grid, inline_plan, s)
-                  : launch_prefill_mode<__half, 128>(a, tq, tk, tv, grid, inline_plan, s);
+        return bf ? launch_prefill_mode<__nv_bfloat16, 128>(a, tq, tk, tv, tp, grid, inline_plan, s)
+                  : launch_prefill_mode<__half, 128>(a, tq, tk, tv, tp, grid, inline_plan, s);
     if (a.c.D == 64)
-        return bf ? launch_prefill_mode<__nv_bfloat16, 64>(a, tq, tk, tv, grid, inline_plan, s)
-                  : launch_prefill_mode<__half, 64>(a, tq, tk, tv, grid, inline_plan, s);
+        return bf ? launch_prefill_mode<__nv_bfloat16, 64>(a, tq, tk, tv, tp, grid, inline_plan, s)
+                  : launch_prefill_mode<__half, 64>(a, tq, tk, tv, tp, grid, inline_plan, s);
     return cudaErrorInvalidValue;
 }
 

@@ -69,6 +69,22 @@ PREFILL_CASES = {
                                    mask_type=W.MASK_CAUSAL, tail_fill=float("nan")),
     "wide_group_decode_shape": dict(seq_len=[1, 1], kv_seq_len=[300, 129], head_num=32,
                                     kv_head_num=1, head_size=128, block_size=16),
+    # tile pairing: odd group size -> one pair + one single tile per KV head
+    "odd_group_g3": dict(seq_len=[150, 20], kv_seq_len=[400, 20], head_num=6, kv_head_num=2,
+                         head_size=128, block_size=32, mask_type=W.MASK_CAUSAL),
+    # g = 1: consecutive token tiles pair up with unequal key-tile counts
+    "mha_three_tiles_prefix": dict(seq_len=[300], kv_seq_len=[700], head_num=2, kv_head_num=2,
+                                   head_size=128, block_size=64, mask_type=W.MASK_CAUSAL,
+                                   dtype="f16"),
+    # pse rows 16-byte aligned: fetched by TMA into per-warp slots
+    "pse_tma_rows_aligned": dict(seq_len=[200, 70], kv_seq_len=[264, 70], head_num=4,
+                                 kv_head_num=2, head_size=128, block_size=16,
+                                 mask_type=W.MASK_CAUSAL, pse=True),
+    "pse_no_mask_d64": dict(seq_len=[130], kv_seq_len=[256], head_num=2, kv_head_num=2,
+                            head_size=64, block_size=32, pse=True, dtype="f16"),
+    "d64_pairs_causal_sink": dict(seq_len=[256, 100], kv_seq_len=[300, 400], head_num=8,
+                                  kv_head_num=2, head_size=64, block_size=64,
+                                  mask_type=W.MASK_CAUSAL, sink=True),
 }
 
 
