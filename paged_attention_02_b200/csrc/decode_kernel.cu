@@ -279,27 +279,44 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
         // ---- scores, masks, online softmax ----
         float sv[2][4];
         float mx_a = -INFINITY, mx_b = -INFINITY;
+        // Interior tile without bias: every key of the 16 is visible to every
+        // row (rows past R only carry zeros and are never written out).
+        const bool simple = !alibi && !a.c.pse && (tw + 16 <= u.t_end) &&
+                            (!causal || tw + 15 <= si.kvlen - si.qlen);
+        if (simple) {
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
+            for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int t = tw + nt * 8 + 2 * c + e;
-                const bool in = t < u.t_end;
-                float x = fmaf(sacc[nt][e], sc_a, add_a);
-                float y = fmaf(sacc[nt][2 + e], sc_b, add_b);
-                if (alibi) {
-                    x = fmaf(slope_a, (float)(t - qpos_a), x);
-                    y = fmaf(slope_b, (float)(t - qpos_b), y);
+                for (int e = 0; e < 2; ++e) {
+                    sv[nt][e] = fmaf(sacc[nt][e], sc_a, add_a);
+                    sv[nt][2 + e] = fmaf(sacc[nt][2 + e], sc_b, add_b);
                 }
-                if (pse_a && in) x = fmaf(to_f32<T>(pse_a[t]), kLog2e, x);
-                if (pse_b && in) y = fmaf(to_f32<T>(pse_b[t]), kLog2e, y);
-                const bool ka = in && va && !(causal && t > qpos_a);
-                const bool kb = in && vb && !(causal && t > qpos_b);
-                sv[nt][e] = ka ? x : -INFINITY;
-                sv[nt][2 + e] = kb ? y : -INFINITY;
-                mx_a = fmaxf(mx_a, sv[nt][e]);
-                mx_b = fmaxf(mx_b, sv[nt][2 + e]);
+            mx_a = fmax3(fmax3(sv[0][0], sv[0][1], sv[1][0]), sv[1][1], -INFINITY);
+            mx_b = fmax3(fmax3(sv[0][2], sv[0][3], sv[1][2]), sv[1][3], -INFINITY);
+        } else {
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int t = tw + nt * 8 + 2 * c + e;
+                    const bool in = t < u.t_end;
+                    float x = fmaf(sacc[nt][e], sc_a, add_a);
+                    float y = fmaf(sacc[nt][2 + e], sc_b, add_b);
+                    if (alibi) {
+                        x = fmaf(slope_a, (float)(t - qpos_a), x);
+                        y = fmaf(slope_b, (float)(t - qpos_b), y);
+                    }
+                    if (pse_a && in) x = fmaf(to_f32<T>(pse_a[t]), kLog2e, x);
+                    if (pse_b && in) y = fmaf(to_f32<T>(pse_b[t]), kLog2e, y);
+                    const bool ka = in && va && !(causal && t > qpos_a);
+                    const bool kb = in && vb && !(causal && t > qpos_b);
+                    sv[nt][e] = ka ? x : -INFINITY;
+                    sv[nt][2 + e] = kb ? y : -INFINITY;
+                    mx_a = fmaxf(mx_a, sv[nt][e]);
+                    mx_b = fmaxf(mx_b, sv[nt][2 + e]);
+                }
             }
+            __syncwarp();
         }
 #pragma unroll
         for (int x = 1; x <= 2; x <<= 1) {
@@ -358,16 +375,20 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
             }
             const int mi = lane >> 3;
             const int tok = warp * 16 + (mi & 1) * 8 + (lane & 7);
+            auto pv_tile = [&](auto masked) {
 #pragma unroll
-            for (int jj = 0; jj < D / 16; ++jj) {
-                const int chunk = 2 * jj + (mi >> 1);
-                const uint32_t addr = vst + (chunk >> 3) * (kDecodeTile * 128) + swz128(tok, chunk & 7);
-                uint32_t v0, v1, v2, v3;
-                ldsm_x4_t(addr, v0, v1, v2, v3);
-                v0 &= mk0; v1 &= mk1; v2 &= mk0; v3 &= mk1;
-                mma_16816<MMA_BF16>(o[2 * jj], pa, v0, v1);
-                mma_16816<MMA_BF16>(o[2 * jj + 1], pa, v2, v3);
-            }
+                for (int jj = 0; jj < D / 16; ++jj) {
+                    const int chunk = 2 * jj + (mi >> 1);
+                    const uint32_t addr = vst + (chunk >> 3) * (kDecodeTile * 128) + swz128(tok, chunk & 7);
+                    uint32_t v0, v1, v2, v3;
+                    ldsm_x4_t(addr, v0, v1, v2, v3);
+                    if (decltype(masked)::value) { v0 &= mk0; v1 &= mk1; v2 &= mk0; v3 &= mk1; }
+                    mma_16816<MMA_BF16>(o[2 * jj], pa, v0, v1);
+                    mma_16816<MMA_BF16>(o[2 * jj + 1], pa, v2, v3);
+                }
+            };
+            if (tail) pv_tile(std::true_type{});
+            else pv_tile(std::false_type{});
         } else {
             const int tk0 = warp * 16 + 2 * c;
             const int tg = tw + 2 * c;
@@ -379,10 +400,11 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
             for (int i = 0; i < D / 32; ++i) {
                 const int chunk = 2 * i + (r >> 2);
                 const int wo = 4 * (r & 3);
-                const uint32_t w0 = lds32(vst + swz128(tk0, chunk) + wo) & z0;
-                const uint32_t w1 = lds32(vst + swz128(tk0 + 1, chunk) + wo) & z1;
-                const uint32_t w2 = lds32(vst + swz128(tk0 + 8, chunk) + wo) & z2;
-                const uint32_t w3 = lds32(vst + swz128(tk0 + 9, chunk) + wo) & z3;
+                uint32_t w0 = lds32(vst + swz128(tk0, chunk) + wo);
+                uint32_t w1 = lds32(vst + swz128(tk0 + 1, chunk) + wo);
+                uint32_t w2 = lds32(vst + swz128(tk0 + 8, chunk) + wo);
+                uint32_t w3 = lds32(vst + swz128(tk0 + 9, chunk) + wo);
+                if (tail) { w0 &= z0; w1 &= z1; w2 &= z2; w3 &= z3; }
                 const uint32_t x01 = prmt(w0, w1, 0x5140u) ^ 0x80808080u;
                 const uint32_t x23 = prmt(w0, w1, 0x7362u) ^ 0x80808080u;
                 const uint32_t y01 = prmt(w2, w3, 0x5140u) ^ 0x80808080u;
