@@ -264,6 +264,52 @@ def cpu_baseline(p, budget_s=12.0):
 
 
 # ---------------------------------------------------------------------------
+# replicas: every rank runs the same workload on its own GPU; the job's time
+# is the slowest rank's, its throughput all ranks' work over that time
+# ---------------------------------------------------------------------------
+def replica_max(vals, dist=None, dev=None):
+    """Element-wise max of per-rank floats over all ranks (identity alone)."""
+    if dist is None:
+        return [float(v) for v in vals]
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def whole_job_rate(world, flops_per_replica, ms):
+    """TFLOP/s of the whole job: N replicas' flops over the slowest rank's ms."""
+    return world * flops_per_replica / (ms * 1e-3) / 1e12
+
+
+def reference_line(args, world):
+    """The oracle timed as it stands on this host's cores: --warmup short
+    untimed samples, then --steps samples that share --ref-seconds of work."""
+    p = W.prefill_prefix()
+    warm_s = min(1.0, args.ref_seconds / 10.0)
+    step_s = max(0.2, args.ref_seconds / max(args.steps, 1))
+    for _ in range(args.warmup):
+        cpu_baseline(p, budget_s=warm_s)
+    rates = []
+    t_all = time.perf_counter()
+    for _ in range(args.steps):
+        r, cores, desc = cpu_baseline(p, budget_s=step_s)
+        rates.append(r)
+    val = statistics.mean(rates)
+    return {"metric": "prefill attention TFLOP/s", "value": val, "unit": "TFLOP/s",
+            "impl": "reference", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": p.name, "batch": 4, "seq_len": [128, 256, 512, 1024],
+                       "prefix": [0, 512, 1024, 3072], "head_num": 32, "kv_head_num": 8,
+                       "head_size": 128, "block_size": 128, "mask": "causal"},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores,
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "wall_s": time.perf_counter() - t_all}
+
+
+# ---------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -272,6 +318,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the secondary workloads")
+    ap.add_argument("--ref-seconds", type=float, default=60.0,
+                    help="reference arm: CPU seconds of oracle work spread over the timed steps")
     ap.add_argument("--profile", default=None, metavar="WORKLOAD",
                     help="run --warmup + --steps plain fia_run calls of one named workload "
                          "(%s) and exit: the command profiled by ncu" % ", ".join(W.NAMED))
@@ -296,43 +344,21 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        # the oracle arm runs on rank 0 alone; the other ranks do no work and
+        # join no process group
+        if rank == 0:
+            print(json.dumps(reference_line(args, world)), flush=True)
+        return
+
     dist = None
     if world > 1:
         import datetime
         import torch.distributed as dist
-        dist.init_process_group("nccl" if args.impl == "ours" else "gloo",
-                                timeout=datetime.timedelta(seconds=120))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     hbm, tfl, tfl_sus, peak_src = measured_peaks()
     p = W.prefill_prefix()
     F = flops(p)
-
-    if args.impl == "reference":
-        if rank == 0:
-            rates = []
-            for _ in range(args.warmup):
-                cpu_baseline(p, budget_s=1.0)
-            t_all = time.perf_counter()
-            for _ in range(args.steps):
-                r, cores, desc = cpu_baseline(p, budget_s=max(2.0, 60.0 / max(args.steps, 1)))
-                rates.append(r)
-            val = statistics.mean(rates)
-            line = {"metric": "prefill attention TFLOP/s", "value": val, "unit": "TFLOP/s",
-                    "impl": "reference", "n_gpus": args.gpus, "steps": args.steps,
-                    "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
-                    "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                    "config": {"workload": p.name, "batch": 4, "seq_len": [128, 256, 512, 1024],
-                               "prefix": [0, 512, 1024, 3072], "head_num": 32, "kv_head_num": 8,
-                               "head_size": 128, "block_size": 128, "mask": "causal"},
-                    "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores,
-                                     "kind": "oracle", "sample": desc},
-                    "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
-                            "d2h_bytes_per_step": 0},
-                    "wall_s": time.perf_counter() - t_all}
-            print(json.dumps(line), flush=True)
-        if dist is not None:
-            dist.barrier()
-            dist.destroy_process_group()
-        return
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
@@ -358,17 +384,13 @@ def main():
         clk.window = (t_start, time.time())
         if dist is not None:
             dist.barrier()
-    ms = statistics.mean(run_ms)
-    kms = statistics.mean(kern_ms)
-    if dist is not None:
-        tt = torch.tensor([ms, kms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, kms = float(tt[0]), float(tt[1])
-    value = world * F / (ms * 1e-3) / 1e12
+    ms, kms = replica_max([statistics.mean(run_ms), statistics.mean(kern_ms)], dist, dev)
+    value = whole_job_rate(world, F, ms)
     achieved = F / (kms * 1e-3) / 1e12
 
     e2e_ms, h2d, d2h = time_e2e(p, max(3, args.steps // 4), 2, dev)
-    e2e_val = world * F / (e2e_ms * 1e-3) / 1e12
+    (e2e_ms,) = replica_max([e2e_ms], dist, dev)
+    e2e_val = whole_job_rate(world, F, e2e_ms)
 
     extra = {}
     if not args.no_extra:
