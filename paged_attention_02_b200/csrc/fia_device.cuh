@@ -168,6 +168,69 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
                  : "memory");
 }
 
+// Eight UMMA K-steps of one block from a single asm statement, with every
+// descriptor prepared beforehand: one instruction per MMA on the issuing
+// thread.  The issuing warp shares its SM sub-partition with busy softmax
+// warps, and each instruction it issues competes with theirs.
+// `acc_first` != 0 accumulates into D at the first step; the other steps
+// always accumulate.
+__device__ __forceinline__ void umma_ss_x8(uint32_t d_tmem, const uint64_t (&a)[8],
+                                           const uint64_t (&b)[8], uint32_t idesc,
+                                           uint32_t acc_first) {
+    asm volatile("{\n\t.reg .pred p, t;\n\t"
+                 "setp.ne.b32 p, %18, 0;\n\t"
+                 "setp.eq.b32 t, %17, %17;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %9, %17, p;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %10, %17, t;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %11, %17, t;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %12, %17, t;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %13, %17, t;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %6, %14, %17, t;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %15, %17, t;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %8, %16, %17, t;\n\t}"
+                 ::"r"(d_tmem), "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(a[4]),
+                   "l"(a[5]), "l"(a[6]), "l"(a[7]), "l"(b[0]), "l"(b[1]), "l"(b[2]),
+                   "l"(b[3]), "l"(b[4]), "l"(b[5]), "l"(b[6]), "l"(b[7]), "r"(idesc),
+                   "r"(acc_first)
+                 : "memory");
+}
+// Four K-steps (a 64-wide contraction), same conventions.
+__device__ __forceinline__ void umma_ss_x4(uint32_t d_tmem, const uint64_t (&a)[4],
+                                           const uint64_t (&b)[4], uint32_t idesc,
+                                           uint32_t acc_first) {
+    asm volatile("{\n\t.reg .pred p, t;\n\t"
+                 "setp.ne.b32 p, %10, 0;\n\t"
+                 "setp.eq.b32 t, %9, %9;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %5, %9, p;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %6, %9, t;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %7, %9, t;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %9, t;\n\t}"
+                 ::"r"(d_tmem), "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(b[0]),
+                   "l"(b[1]), "l"(b[2]), "l"(b[3]), "r"(idesc), "r"(acc_first)
+                 : "memory");
+}
+// The same with A read from TMEM (a[k]: TMEM address of K-step k).
+__device__ __forceinline__ void umma_ts_x8(uint32_t d_tmem, const uint32_t (&a)[8],
+                                           const uint64_t (&b)[8], uint32_t idesc,
+                                           uint32_t acc_first) {
+    asm volatile("{\n\t.reg .pred p, t;\n\t"
+                 "setp.ne.b32 p, %18, 0;\n\t"
+                 "setp.eq.b32 t, %17, %17;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %9, %17, p;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %10, %17, t;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %11, %17, t;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %12, %17, t;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%5], %13, %17, t;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%6], %14, %17, t;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%7], %15, %17, t;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%8], %16, %17, t;\n\t}"
+                 ::"r"(d_tmem), "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]),
+                   "r"(a[5]), "r"(a[6]), "r"(a[7]), "l"(b[0]), "l"(b[1]), "l"(b[2]),
+                   "l"(b[3]), "l"(b[4]), "l"(b[5]), "l"(b[6]), "l"(b[7]), "r"(idesc),
+                   "r"(acc_first)
+                 : "memory");
+}
+
 // Arrive (once) on `bar` when every tcgen05 op this thread issued so far is done.
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -238,15 +301,52 @@ __device__ __forceinline__ void tmem_st_wait() {
 // Shared-memory matrix descriptor for UMMA (sm_100 layout: start>>4 in
 // [0,14), leading-byte-offset>>4 in [16,30), stride-byte-offset>>4 in
 // [32,46), version 1 in [46,48), swizzle mode in [61,64); 2 = 128-byte swizzle).
-__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr, uint32_t lbo_bytes,
-                                                    uint32_t sbo_bytes) {
-    uint64_t d = 0;
-    d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
-    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
-    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
-    d |= (uint64_t)1u << 46;
-    d |= (uint64_t)2u << 61;
-    return d;
+__host__ __device__ __forceinline__ constexpr uint64_t umma_desc_sw128(uint32_t smem_addr,
+                                                                      uint32_t lbo_bytes,
+                                                                      uint32_t sbo_bytes) {
+    return (uint64_t)((smem_addr >> 4) & 0x3FFFu)
+           | (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16
+           | (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32
+           | (uint64_t)1u << 46
+           | (uint64_t)2u << 61;
+}
+// The same descriptor as two 32-bit words.  The low word (start address,
+// leading byte offset) is the one that moves along K; adding (bytes >> 4) to
+// it advances the start address as long as the address stays below 256 KB
+// (always true for shared memory), so the per-step cost is one 32-bit add.
+__host__ __device__ __forceinline__ constexpr uint32_t umma_desc_lo(uint32_t smem_addr,
+                                                                   uint32_t lbo_bytes) {
+    return ((smem_addr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+__host__ __device__ __forceinline__ constexpr uint32_t umma_desc_hi_sw128(uint32_t sbo_bytes) {
+    return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+}
+static_assert(umma_desc_sw128(0x2A400u + 0x460u, 16384u, 1024u) ==
+                  (((uint64_t)umma_desc_hi_sw128(1024u) << 32) |
+                   (umma_desc_lo(0x2A400u, 16384u) + (0x460u >> 4))),
+              "split UMMA descriptor words disagree with the 64-bit form");
+
+// UMMA issue with split descriptor words (see umma_desc_lo).
+__device__ __forceinline__ void umma_ss_w(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi,
+                                          uint32_t b_lo, uint32_t b_hi, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+                 "setp.ne.b32 p, %6, 0;\n\t"
+                 "mov.b64 da, {%1, %2};\n\t"
+                 "mov.b64 db, {%3, %4};\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}"
+                 ::"r"(d_tmem), "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc),
+                   "r"(accumulate)
+                 : "memory");
+}
+__device__ __forceinline__ void umma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                          uint32_t b_hi, uint32_t idesc, uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+                 "setp.ne.b32 p, %5, 0;\n\t"
+                 "mov.b64 db, {%2, %3};\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}"
+                 ::"r"(d_tmem), "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+                 : "memory");
 }
 
 // Instruction descriptor for kind::f16 with an f32 accumulator.

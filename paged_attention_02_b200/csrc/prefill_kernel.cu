@@ -260,40 +260,62 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     } else if (warp == 1) {
         // ------------------------------------------------------------ UMMA issuer
         uint32_t q_it = 0, kv_it = 0, p_it[2] = {0, 0};
-        auto issue_qk = [&](int x, int ks) {
-            const uint32_t qb = sm_q + x * Cfg::kTileBytes;
-            const uint32_t kb = sm_k0 + ks * Cfg::kTileBytes;
+        // The issuing warp shares its SM sub-partition with four busy softmax
+        // warps, so it is starved of issue slots: every block of MMAs is
+        // issued from one asm statement, with its descriptors prepared before
+        // the wait that precedes it (off the critical path).
+        constexpr int NKQ = D / 16;                     // K-steps of QK^T
+        constexpr uint32_t kHi = umma_desc_hi_sw128(1024);
+        constexpr uint32_t kTileStep = Cfg::kTileBytes >> 4;
+        const uint32_t q_lo = umma_desc_lo(sm_q, 16);
+        const uint32_t k_lo = umma_desc_lo(sm_k0, 16);
+        const uint32_t v_lo = umma_desc_lo(sm_v0, Cfg::kGroupBytes);
+        // K-major 128-row operand (a Q or K tile): 16 columns per K-step
+        auto kmajor = [&](uint32_t lo, uint64_t (&d)[NKQ]) {
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * Cfg::kGroupBytes + (kk & 3) * 32;
-                umma_ss(tmem + Cfg::col_s(x), umma_desc_sw128(qb + off, 16, 1024),
-                        umma_desc_sw128(kb + off, 16, 1024), IDESC_QK, kk > 0);
-            }
+            for (int kk = 0; kk < NKQ; ++kk)
+                d[kk] = ((uint64_t)kHi << 32) |
+                        (lo + (((kk >> 2) * Cfg::kGroupBytes + (kk & 3) * 32) >> 4));
         };
-        auto issue_pv = [&](int x, int vs, bool acc) {
-            const uint32_t vb = sm_v0 + vs * Cfg::kTileBytes;
+        // MN-major V tile: 16 keys (2048 bytes) per K-step
+        auto vmajor = [&](uint32_t lo, uint64_t (&d)[8]) {
 #pragma unroll
-            for (int kk = 0; kk < kPrefillBN / 16; ++kk)
-                umma_ts(tmem + Cfg::col_o(x), tmem + Cfg::col_s(x) + kk * 8,
-                        umma_desc_sw128(vb + kk * 2048, Cfg::kGroupBytes, 1024), IDESC_PV,
-                        (acc || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 8; ++kk) d[kk] = ((uint64_t)kHi << 32) | (lo + kk * (2048 >> 4));
         };
+        auto ptmem = [&](int x, uint32_t (&d)[8]) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) d[kk] = tmem + Cfg::col_s(x) + kk * 8;
+        };
+        auto qk = [&](int x, const uint64_t (&qd)[NKQ], const uint64_t (&kd)[NKQ]) {
+            if constexpr (NKQ == 8) umma_ss_x8(tmem + Cfg::col_s(x), qd, kd, IDESC_QK, 0u);
+            else umma_ss_x4(tmem + Cfg::col_s(x), qd, kd, IDESC_QK, 0u);
+        };
+        static_assert(kPrefillBN / 16 == 8, "PV issue assumes 8 key steps per tile");
+        static_assert(NKQ == 4 || NKQ == 8, "QK issue assumes D = 64 or 128");
         for (idx = it_begin; idx < it_end; ++idx) {
             const PairGeom gm = pair_geom(a, items, seqs, idx);
             if (gm.nB == 0) continue;
             dbg_j = -1;
+            uint64_t qd[NKQ], kd[NKQ], vd[8];
+            uint32_t pa[8];
             FIA_WAIT(q_full, q_it & 1, 20);
             ++q_it;
             const uint32_t kv_base = kv_it;
             {
                 // QK for key tile 0 (both tiles)
                 const int ks = kv_base % KS;
+                kmajor(k_lo + ks * kTileStep, kd);
                 FIA_WAIT(&k_full[ks], (kv_base / KS) & 1, 21);
                 __syncwarp();
                 tc_fence_after();
                 if (lane == 0) {
-                    if (gm.nA > 0) { issue_qk(0, ks); umma_commit(&s_full[0]); }
-                    issue_qk(1, ks);
+                    if (gm.nA > 0) {
+                        kmajor(q_lo, qd);
+                        qk(0, qd, kd);
+                        umma_commit(&s_full[0]);
+                    }
+                    kmajor(q_lo + kTileStep, qd);
+                    qk(1, qd, kd);
                     umma_commit(&s_full[1]);
                     umma_commit(&k_empty[ks]);
                     if (gm.nB == 1) umma_commit(q_empty);
@@ -304,65 +326,126 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 dbg_j = j;
                 const uint32_t kvi = kv_base + j;
                 const int vs = kvi % VS;
+                const bool more = (j + 1 < gm.nB);
+                const uint32_t kn = kv_base + j + 1;
+                const int ksn = kn % KS;
+                vmajor(v_lo + vs * kTileStep, vd);
+                kmajor(k_lo + ksn * kTileStep, kd);
                 FIA_WAIT(&v_full[vs], (kvi / VS) & 1, 24);
                 __syncwarp();
                 const int valid = gm.kvlen - j * kPrefillBN;
                 if (valid < kPrefillBN) {
                     // rows past kvSeqLen: P is 0 there, but the slots may
                     // hold anything (NaN * 0 = NaN in the MMA) -> zero them.
-                    uint8_t *vd = smem + Cfg::kOffV + vs * Cfg::kTileBytes;
+                    uint8_t *vdst = smem + Cfg::kOffV + vs * Cfg::kTileBytes;
                     const int nbytes = (kPrefillBN - valid) * 128;
                     for (int hv = 0; hv < Cfg::kHalves; ++hv) {
-                        uint4 *p = reinterpret_cast<uint4 *>(vd + hv * Cfg::kGroupBytes + valid * 128);
+                        uint4 *p = reinterpret_cast<uint4 *>(vdst + hv * Cfg::kGroupBytes + valid * 128);
                         for (int x = lane; x < nbytes / 16; x += 32) p[x] = make_uint4(0, 0, 0, 0);
                     }
                     fence_proxy_async_smem();
                     __syncwarp();
                 }
-                const bool more = (j + 1 < gm.nB);
-                const uint32_t kn = kv_base + j + 1;
-                const int ksn = kn % KS;
-                if (j < gm.nA) {
-                    FIA_WAIT(&p_full[0], p_it[0] & 1, 23);
-                    ++p_it[0];
-                    __syncwarp();
-                    tc_fence_after();
-                    if (lane == 0) {
-                        issue_pv(0, vs, j > 0);
-                        umma_commit(&pv_done[0]);
-                        if (j == gm.nA - 1) umma_commit(&o_full[0]);
-                    }
-                    __syncwarp();
-                    if (j + 1 < gm.nA) {
-                        FIA_WAIT(&k_full[ksn], (kn / KS) & 1, 22);
+                if constexpr (KS >= 2) {
+                    // Every wait comes before a block, so each tile's PV(j) and
+                    // QK(j+1) go out back to back from one thread with only
+                    // commits between them (the issuing warp is starved of
+                    // issue slots by the softmax warps beside it, so any
+                    // instruction between two blocks leaves the tensor pipe
+                    // idle).  K(j+1) was requested a whole key tile earlier:
+                    // waiting for it up front almost never waits.
+                    if (more) FIA_WAIT(&k_full[ksn], (kn / KS) & 1, 22);
+                    if (j < gm.nA) {
+                        ptmem(0, pa);
+                        kmajor(q_lo, qd);
+                        FIA_WAIT(&p_full[0], p_it[0] & 1, 23);
+                        ++p_it[0];
                         __syncwarp();
                         tc_fence_after();
-                        if (lane == 0) { issue_qk(0, ksn); umma_commit(&s_full[0]); }
+                        if (lane == 0) {
+                            umma_ts_x8(tmem + Cfg::col_o(0), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
+                            umma_commit(&pv_done[0]);
+                            if (j + 1 < gm.nA) {
+                                qk(0, qd, kd);
+                                umma_commit(&s_full[0]);
+                            } else {
+                                umma_commit(&o_full[0]);
+                            }
+                        }
                         __syncwarp();
                     }
-                }
-                FIA_WAIT(&p_full[1], p_it[1] & 1, 25);
-                ++p_it[1];
-                __syncwarp();
-                tc_fence_after();
-                if (lane == 0) {
-                    issue_pv(1, vs, j > 0);
-                    umma_commit(&pv_done[1]);
-                    umma_commit(&v_empty[vs]);
-                    if (j == gm.nB - 1) umma_commit(&o_full[1]);
-                }
-                __syncwarp();
-                if (more) {
-                    FIA_WAIT(&k_full[ksn], (kn / KS) & 1, 26);
+                    ptmem(1, pa);
+                    kmajor(q_lo + kTileStep, qd);
+                    FIA_WAIT(&p_full[1], p_it[1] & 1, 25);
+                    ++p_it[1];
                     __syncwarp();
                     tc_fence_after();
                     if (lane == 0) {
-                        issue_qk(1, ksn);
-                        umma_commit(&s_full[1]);
-                        umma_commit(&k_empty[ksn]);
-                        if (j + 1 == gm.nB - 1) umma_commit(q_empty);
+                        umma_ts_x8(tmem + Cfg::col_o(1), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
+                        umma_commit(&pv_done[1]);
+                        umma_commit(&v_empty[vs]);
+                        if (more) {
+                            qk(1, qd, kd);
+                            umma_commit(&s_full[1]);
+                            umma_commit(&k_empty[ksn]);
+                            if (j + 1 == gm.nB - 1) umma_commit(q_empty);
+                        } else {
+                            umma_commit(&o_full[1]);
+                        }
                     }
                     __syncwarp();
+                } else {
+                    // One K stage: K(j+1) is loaded only after QK(j) of both
+                    // tiles, so it is waited for between the PV and QK blocks.
+                    if (j < gm.nA) {
+                        ptmem(0, pa);
+                        kmajor(q_lo, qd);
+                        FIA_WAIT(&p_full[0], p_it[0] & 1, 23);
+                        ++p_it[0];
+                        __syncwarp();
+                        tc_fence_after();
+                        if (lane == 0) {
+                            umma_ts_x8(tmem + Cfg::col_o(0), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
+                            umma_commit(&pv_done[0]);
+                            if (j == gm.nA - 1) umma_commit(&o_full[0]);
+                        }
+                        __syncwarp();
+                        if (j + 1 < gm.nA) {
+                            FIA_WAIT(&k_full[ksn], (kn / KS) & 1, 22);
+                            __syncwarp();
+                            tc_fence_after();
+                            if (lane == 0) {
+                                qk(0, qd, kd);
+                                umma_commit(&s_full[0]);
+                            }
+                            __syncwarp();
+                        }
+                    }
+                    ptmem(1, pa);
+                    kmajor(q_lo + kTileStep, qd);
+                    FIA_WAIT(&p_full[1], p_it[1] & 1, 25);
+                    ++p_it[1];
+                    __syncwarp();
+                    tc_fence_after();
+                    if (lane == 0) {
+                        umma_ts_x8(tmem + Cfg::col_o(1), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
+                        umma_commit(&pv_done[1]);
+                        umma_commit(&v_empty[vs]);
+                        if (j == gm.nB - 1) umma_commit(&o_full[1]);
+                    }
+                    __syncwarp();
+                    if (more) {
+                        FIA_WAIT(&k_full[ksn], (kn / KS) & 1, 26);
+                        __syncwarp();
+                        tc_fence_after();
+                        if (lane == 0) {
+                            qk(1, qd, kd);
+                            umma_commit(&s_full[1]);
+                            umma_commit(&k_empty[ksn]);
+                            if (j + 1 == gm.nB - 1) umma_commit(q_empty);
+                        }
+                        __syncwarp();
+                    }
                 }
             }
             kv_it = kv_base + gm.nB;
