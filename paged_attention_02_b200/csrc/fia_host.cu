@@ -322,14 +322,14 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
     if (!decode)
         enc_ok = enc_ok && encode_3d(&o->tq, tdt, 2, query->data, D, headNum, n_tokens, 64, kPrefillBM);
     if (!decode && pse && (pse->dims[3] % 8) == 0 && aligned16(pse->data)) {
-        // pse viewed as {maxKV, maxQ, B*H}; one softmax warp fetches a
-        // {64 keys, 32 rows} box (128-byte swizzle)
+        // pse viewed as {maxKV, maxQ, B*H}; one softmax warp fetches two
+        // {64 keys, 16 rows} boxes per key tile (128-byte swizzle)
         auto fn = encode_fn();
         cuuint64_t dims[3] = {(cuuint64_t)pse->dims[3], (cuuint64_t)pse->dims[2],
                               (cuuint64_t)(pse->dims[0] * pse->dims[1])};
         cuuint64_t strides[2] = {(cuuint64_t)pse->dims[3] * 2,
                                  (cuuint64_t)(pse->dims[2] * pse->dims[3] * 2)};
-        cuuint32_t box[3] = {64, 32, 1};
+        cuuint32_t box[3] = {64, 16, 1};
         cuuint32_t es[3] = {1, 1, 1};
         enc_ok = enc_ok && fn &&
                  fn(&o->tp, tdt, 3, pse->data, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,

@@ -20,13 +20,15 @@
 //              tcgen05.mma ops run in issue order, so QK_X(j+1) may be issued
 //              right after PV_X(j) over the same TMEM columns.  It zeroes the V
 //              rows past kvSeqLen in a ragged last tile.
-//   warps 2-9  softmax + epilogue of tile 0, warps 10-17 of tile 1: each query
-//              row is shared by two warps (same TMEM lanes, 64 key columns
-//              each; they swap row maxima through shared memory), S ->
-//              registers, scale / mask / bias, online softmax in fp32 (log2
-//              domain; O rescaled in TMEM only when the running max grows by
-//              more than 2^8), P in the input dtype written back over S; at
-//              the end O / l, sink, lse (each warp writes half of the row).
+//   warps 2-9  softmax + epilogue of tile 0, warps 10-17 of tile 1: each warp
+//              owns 16 query rows (TMEM lanes) of its lane quadrant; lanes t
+//              and t + 16 hold the two 64-key halves of one row (16x32bx2
+//              TMEM access), so row maxima and sums are combined with one
+//              shuffle.  S -> registers, scale / mask / bias, online softmax
+//              in fp32 (log2 domain; O rescaled in TMEM only when the running
+//              max grows by more than 2^8), P in the input dtype written back
+//              over S; at the end O / l, sink, lse (each lane writes half of
+//              its row).
 // TMEM (512 columns): S_0 | S_1 | O_0 | O_1.  While one softmax group works on
 // its S, the tensor core runs the other tile's PV and QK^T.
 // Every mbarrier wait is bounded in time (see fia_device.cuh).
@@ -54,18 +56,14 @@ struct PrefillCfg {
     static constexpr int kOffQ = 0;                                    // Q[2]
     static constexpr int kOffK = kOffQ + 2 * kTileBytes;               // K[s]
     static constexpr int kOffV = kOffK + kKStages * kTileBytes;        // V[s]
-    // row-max / row-sum exchange between the two warps sharing a TMEM lane
-    // quadrant: [parity][tile X][quadrant][column half][lane] floats
-    static constexpr int kOffX = kOffV + kVStages * kTileBytes;
-    static constexpr int kXBytes = 2 * 2 * 4 * 2 * 32 * 4;
-    // pse mode: one 32-row x 64-key pse box (4 KB, 128-byte swizzle) per
-    // softmax warp, fetched by that warp one key tile ahead
-    static constexpr int kOffPse = kOffX + kXBytes;
+    // pse mode: two 16-row x 64-key pse boxes (2 x 2 KB, 128-byte swizzle)
+    // per softmax warp, fetched by that warp one key tile ahead
+    static constexpr int kOffPse = kOffV + kVStages * kTileBytes;
     static constexpr int kPseBytes = (MODE == kModePse) ? 16 * 4096 : 0;
     static constexpr int kOffBar = kOffPse + kPseBytes;
     // q_full, q_empty, k_full/k_empty[KS], v_full/v_empty[VS],
-    // s_full[2], p_full[2], pv_done[2], o_full[2], xch[2][4], pse_full[16]
-    static constexpr int kNumBar = 2 + 2 * kKStages + 2 * kVStages + 8 + 8 + 16;
+    // s_full[2], p_full[2], pv_done[2], o_full[2], pse_full[16]
+    static constexpr int kNumBar = 2 + 2 * kKStages + 2 * kVStages + 8 + 16;
     static constexpr int kUsed = kOffBar + kNumBar * 8 + 16;
     // Keep one CTA per SM (each CTA holds all 512 TMEM columns).
     static constexpr int kSmem = 1024 + (kUsed > 118 * 1024 ? kUsed : 118 * 1024);
@@ -150,9 +148,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     uint64_t *p_full = s_full + 2;          // [2]  P_X written (4 warps)
     uint64_t *pv_done = p_full + 2;         // [2]  PV_X done
     uint64_t *o_full = pv_done + 2;         // [2]  last PV_X of the pair done
-    uint64_t *xch = o_full + 2;             // [2][4] max / sum exchange (2 warps)
-    uint64_t *pse_full = xch + 8;           // [16] per softmax warp (pse mode)
-    float *xbuf = reinterpret_cast<float *>(smem + Cfg::kOffX);
+    uint64_t *pse_full = o_full + 2;        // [16] per softmax warp (pse mode)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + Cfg::kNumBar);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -177,7 +173,6 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             mbar_init(&pv_done[x], 1);
             mbar_init(&o_full[x], 1);
         }
-        for (int x = 0; x < 8; ++x) mbar_init(&xch[x], 2);
         for (int x = 0; x < 16; ++x) mbar_init(&pse_full[x], 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -452,52 +447,40 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         }
     } else {
         // ------------------------------------------------------------ softmax + epilogue
-        // 8 warps per tile: warp (quadrant q, half h) owns query rows
-        // 32q..32q+31 (its TMEM lanes) and key columns 64h..64h+63 of S.
+        // 8 warps per tile: warp (quadrant q, sub-block u) owns query rows
+        // 32q + 16u .. +15 (TMEM lanes); lane t holds row 32q + 16u + (t & 15)
+        // and key columns 64h .. 64h + 63 of S with h = t >> 4.
         const int sw = warp - 2;
         const int X = sw >> 3;                     // which tile of the pair
-        const int half = (sw >> 2) & 1;            // which 64 columns
+        const int sub = (sw >> 2) & 1;             // which 16 rows of the quadrant
         const int quad = warp & 3;
-        const int row = quad * 32 + lane;
-        const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
-        const uint32_t scol = t_lane + Cfg::col_s(X) + 64 * half;      // S columns
-        const uint32_t pcol = t_lane + Cfg::col_s(X) + 32 * half;      // P columns (2 keys each)
-        constexpr int DH = D / 2;                                      // O columns per warp
-        const uint32_t ocol = t_lane + Cfg::col_o(X) + DH * half;
-        uint64_t *xb = &xch[X * 4 + quad];
-        float *xmine = xbuf + ((X * 4 + quad) * 2 + half) * 32 + lane;     // + parity * 512
-        const float *xpeer = xbuf + ((X * 4 + quad) * 2 + (half ^ 1)) * 32 + lane;
+        const int half = lane >> 4;                // which 64 key columns (per lane)
+        const int row = quad * 32 + sub * 16 + (lane & 15);
+        const uint32_t t_lane = tmem + ((uint32_t)(quad * 32 + sub * 16) << 16);
+        const uint32_t scol = t_lane + Cfg::col_s(X);                  // S (+64 for h = 1)
+        constexpr int DH = D / 2;                                      // O columns per lane
+        const uint32_t ocol = t_lane + Cfg::col_o(X);                  // O (+DH for h = 1)
         const bool causal = (a.c.mask_type == 9 || a.c.mask_type == 3);
         const float sl2 = a.c.scale_log2;
         // plain mode with a positive scale: mask raw scores and fold the scale
         // into the exponent (one FFMA per element)
         const bool fold = (MODE == kModePlain) && (sl2 > 0.f);
-        uint32_t s_it = 0, p_it = 0, o_it = 0, x_it = 0, ps_it = 0;
+        uint32_t s_it = 0, p_it = 0, o_it = 0, ps_it = 0;
         T *outp = reinterpret_cast<T *>(a.c.out);
         const bool pse_tma = (MODE == kModePse) && a.c.pse_tma;
         uint8_t *pslot = smem + Cfg::kOffPse + sw * 4096;
         uint64_t *pbar = &pse_full[sw];
-        // lane 0 fetches this warp's pse box (32 rows x 64 keys) of key tile jt
+        // lane 0 fetches this warp's two pse boxes (16 rows x 64 keys each) of
+        // key tile jt
         auto pse_fetch = [&](const PairGeom &g2, const SubGeom &s2, int jt) {
             if (lane == 0) {
                 mbar_arrive_expect_tx(pbar, 4096);
-                tma_load_3d(pslot, &tp, pbar, jt * kPrefillBN + 64 * half, s2.q0 + 32 * quad,
-                            g2.b * a.c.H + s2.h);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh)
+                    tma_load_3d(pslot + hh * 2048, &tp, pbar, jt * kPrefillBN + 64 * hh,
+                                s2.q0 + 32 * quad + 16 * sub, g2.b * a.c.H + s2.h);
             }
         };
-
-        // Exchange one float per row with the partner warp (bounded wait).
-#define FIA_EXCHANGE(val, out)                                                            \
-    do {                                                                                  \
-        const int _par = x_it & 1;                                                        \
-        xmine[_par * 512] = (val);                                                        \
-        __syncwarp();                                                                     \
-        if (lane == 0) mbar_arrive(xb);                                                   \
-        FIA_WAIT(xb, x_it & 1, 33);                                                       \
-        __syncwarp();                                                                     \
-        (out) = xpeer[_par * 512];                                                        \
-        ++x_it;                                                                           \
-    } while (0)
 
         for (idx = it_begin; idx < it_end; ++idx) {
             const PairGeom gm = pair_geom(a, items, seqs, idx);
@@ -528,14 +511,14 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             if (pse_tma) pse_fetch(gm, sg, 0);
             for (int j = 0; j < sg.n; ++j) {
                 dbg_j = j;
-                const int tb = j * kPrefillBN + 64 * half;     // first key of this warp
+                const int tb = j * kPrefillBN + 64 * half;     // first key of this lane
                 FIA_WAIT(&s_full[X], s_it & 1, 30);
                 ++s_it;
                 __syncwarp();          // tcgen05.ld/st below are warp-collective (.aligned)
                 tc_fence_after();
                 uint32_t sr[2][32];
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) tmem_ld32(scol + cc * 32, sr[cc]);
+                for (int cc = 0; cc < 2; ++cc) tmem_ld16x2_32<64>(scol + cc * 32, sr[cc]);
                 tmem_ld_wait();
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) reg_fence32(sr[cc]);
@@ -552,16 +535,17 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                             sr[cc][x] = __float_as_uint(fmaf(__uint_as_float(sr[cc][x]), sl2, bias));
                         }
                 } else if (MODE == kModePse && pse_tma) {
-                    // this warp's pse box for tile j, 128-byte swizzled rows
+                    // this lane's row of pse box `half` for tile j (128-byte swizzle)
                     FIA_WAIT(pbar, ps_it & 1, 34);
                     ++ps_it;
-                    const uint32_t prow = smem_u32(pslot) + lane * 128;
+                    const int r16 = lane & 15;
+                    const uint32_t prow = smem_u32(pslot) + half * 2048 + r16 * 128;
 #pragma unroll
                     for (int c16 = 0; c16 < 8; ++c16) {
                         uint32_t w4[4];
                         asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
                                      : "=r"(w4[0]), "=r"(w4[1]), "=r"(w4[2]), "=r"(w4[3])
-                                     : "r"(prow + ((c16 ^ (lane & 7)) << 4)));
+                                     : "r"(prow + ((c16 ^ (r16 & 7)) << 4)));
                         const T *pv = reinterpret_cast<const T *>(w4);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
@@ -571,7 +555,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                                 fmaf(__uint_as_float(sr[col >> 5][col & 31]), sl2, bias));
                         }
                     }
-                    // the slot is free: fetch the next tile's box (generic-proxy
+                    // the slot is free: fetch the next tile's boxes (generic-proxy
                     // reads ordered before the async-proxy write)
                     fence_proxy_async_smem();
                     __syncwarp();
@@ -617,7 +601,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                             if (!keep) sr[cc][x] = __float_as_uint(-INFINITY);
                         }
                 }
-                // tree max over this warp's 64 columns, then with the partner's
+                // tree max over this lane's 64 columns, then with lane t ^ 16
 #define FIA_EL(e) __uint_as_float(sr[(e) >> 5][(e) & 31])
                 float mx4[4];
 #pragma unroll
@@ -628,12 +612,8 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                     for (int k = 0; k < 4; ++k) mx4[k] = fmax3(mx4[k], FIA_EL(e + k), FIA_EL(e + 4 + k));
 #undef FIA_EL
                 float mx = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
                 if (fold) mx = (mx == -INFINITY) ? -INFINITY : mx * sl2;
-                {
-                    float mp;
-                    FIA_EXCHANGE(mx, mp);
-                    mx = fmaxf(mx, mp);
-                }
 
                 // running max: exact on the first tile, afterwards raised only
                 // when it grows by more than 2^8 (O and l stay consistent with m)
@@ -650,7 +630,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 }
                 const float mu = (m == -INFINITY) ? 0.f : m;
 
-                // P = 2^(s - m) in the input dtype over this warp's part of S
+                // P = 2^(s - m) in the input dtype over this lane's half row
                 const uint64_t negmu2 = f2pack(-mu, -mu);
                 const uint64_t sl2x2 = f2pack(sl2, sl2);
                 uint64_t acc2[4];
@@ -672,7 +652,8 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                         f2unpack(pp, p0, p1);
                         pk[x] = pack2<T>(p0, p1);
                     }
-                    tmem_st16(pcol + cc * 16, pk);
+                    // packed P columns 32h + 16cc .. +15 (keys 64h + 32cc ..)
+                    tmem_st16x2_16<32>(scol + cc * 16, pk);
                 }
                 {
                     const uint64_t s01 = fadd2(fadd2(acc2[0], acc2[1]), fadd2(acc2[2], acc2[3]));
@@ -681,10 +662,10 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                     l += l0 + l1;
                 }
 
-                // Rescale this warp's half of O (rare).  The previous PV of this
-                // tile must be done with O first.  (The softmax warps cannot
-                // drift apart: S for the next key tile is only produced after
-                // all eight warps have signalled this P.)
+                // Rescale this lane's half of its O row (rare).  The previous PV
+                // of this tile must be done with O first.  (The softmax warps
+                // cannot drift apart: S for the next key tile is only produced
+                // after all eight warps have signalled this P.)
                 if (__any_sync(0xffffffffu, need)) {
                     if (j > 0) {
                         FIA_WAIT(&pv_done[X], (p_it - 1) & 1, 31);
@@ -694,13 +675,13 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
 #pragma unroll
                     for (int cc = 0; cc < DH / 32; ++cc) {
                         uint32_t orr[32];
-                        tmem_ld32(ocol + cc * 32, orr);
+                        tmem_ld16x2_32<DH>(ocol + cc * 32, orr);
                         tmem_ld_wait();
                         reg_fence32(orr);
 #pragma unroll
                         for (int x = 0; x < 32; ++x)
                             orr[x] = __float_as_uint(__uint_as_float(orr[x]) * alpha);
-                        tmem_st32(ocol + cc * 32, orr);
+                        tmem_st16x2_32<DH>(ocol + cc * 32, orr);
                     }
                 }
                 tmem_st_wait();
@@ -710,13 +691,9 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 ++p_it;
             }
 
-            // ---- epilogue: O / l (+ sink), lse; this warp writes D/2 columns ----
+            // ---- epilogue: O / l (+ sink), lse; each lane writes D/2 columns ----
             dbg_j = sg.n;
-            {
-                float lp;
-                FIA_EXCHANGE(l, lp);
-                l += lp;
-            }
+            l += __shfl_xor_sync(0xffffffffu, l, 16);
             FIA_WAIT(&o_full[X], o_it & 1, 32);
             ++o_it;
             __syncwarp();
@@ -732,7 +709,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
 #pragma unroll
             for (int cc = 0; cc < DH / 32; ++cc) {
                 uint32_t orr[32];
-                tmem_ld32(ocol + cc * 32, orr);
+                tmem_ld16x2_32<DH>(ocol + cc * 32, orr);
                 tmem_ld_wait();
                 reg_fence32(orr);
                 if (valid) {
@@ -752,7 +729,6 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             tc_fence_before();
             __syncwarp();
         }
-#undef FIA_EXCHANGE
     }
 done:
     tc_fence_before();
