@@ -45,6 +45,10 @@ namespace fia {
 
 enum { kModePlain = 0, kModeAlibi = 1, kModePse = 2 };
 
+// 128 rows x 128 bytes of zeros (static storage starts zeroed): copied by the
+// bulk-copy engine over the V rows past kvSeqLen of a ragged last key tile.
+static __device__ __align__(128) uint8_t g_zero_rows[kPrefillBN * 128];
+
 template <int D, int MODE = kModePlain>
 struct PrefillCfg {
     static constexpr int kHalves = D / 64;                 // 128-byte column groups
@@ -62,8 +66,8 @@ struct PrefillCfg {
     static constexpr int kPseBytes = (MODE == kModePse) ? 16 * 4096 : 0;
     static constexpr int kOffBar = kOffPse + kPseBytes;
     // q_full, q_empty, k_full/k_empty[KS], v_full/v_empty[VS],
-    // s_full[2], p_full[2], pv_done[2], o_full[2], pse_full[16]
-    static constexpr int kNumBar = 2 + 2 * kKStages + 2 * kVStages + 8 + 16;
+    // s_full[2], p_full[2], pv_done[2], o_full[2], pse_full[16], vz_full
+    static constexpr int kNumBar = 2 + 2 * kKStages + 2 * kVStages + 8 + 16 + 1;
     static constexpr int kUsed = kOffBar + kNumBar * 8 + 16;
     // Keep one CTA per SM (each CTA holds all 512 TMEM columns).
     static constexpr int kSmem = 1024 + (kUsed > 118 * 1024 ? kUsed : 118 * 1024);
@@ -149,6 +153,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     uint64_t *pv_done = p_full + 2;         // [2]  PV_X done
     uint64_t *o_full = pv_done + 2;         // [2]  last PV_X of the pair done
     uint64_t *pse_full = o_full + 2;        // [16] per softmax warp (pse mode)
+    uint64_t *vz_full = pse_full + 16;      // zero rows copied over a ragged V tile
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + Cfg::kNumBar);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -174,6 +179,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             mbar_init(&o_full[x], 1);
         }
         for (int x = 0; x < 16; ++x) mbar_init(&pse_full[x], 1);
+        mbar_init(vz_full, 1);
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tq);
@@ -254,11 +260,14 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ UMMA issuer
-        uint32_t q_it = 0, kv_it = 0, p_it[2] = {0, 0};
+        // One lane runs this role; the other 31 go straight to the teardown.
         // The issuing warp shares its SM sub-partition with four busy softmax
-        // warps, so it is starved of issue slots: every block of MMAs is
-        // issued from one asm statement, with its descriptors prepared before
-        // the wait that precedes it (off the critical path).
+        // warps and is starved of issue slots, so every instruction here is
+        // expensive: no warp-level syncs, each block of MMAs issued from one
+        // asm statement with descriptors prepared before the wait that
+        // precedes it.
+        if (lane != 0) goto done;
+        uint32_t q_it = 0, kv_it = 0, p_it[2] = {0, 0}, vz_it = 0;
         constexpr int NKQ = D / 16;                     // K-steps of QK^T
         constexpr uint32_t kHi = umma_desc_hi_sw128(1024);
         constexpr uint32_t kTileStep = Cfg::kTileBytes >> 4;
@@ -277,6 +286,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) d[kk] = ((uint64_t)kHi << 32) | (lo + kk * (2048 >> 4));
         };
+        // TMEM addresses of P (the PV A operand) of tile x
         auto ptmem = [&](int x, uint32_t (&d)[8]) {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) d[kk] = tmem + Cfg::col_s(x) + kk * 8;
@@ -291,6 +301,8 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             const PairGeom gm = pair_geom(a, items, seqs, idx);
             if (gm.nB == 0) continue;
             dbg_j = -1;
+            // descriptors are rebuilt before each wait rather than kept live:
+            // registers are scarce (96 per thread) and the softmax roles need them
             uint64_t qd[NKQ], kd[NKQ], vd[8];
             uint32_t pa[8];
             FIA_WAIT(q_full, q_it & 1, 20);
@@ -301,21 +313,17 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 const int ks = kv_base % KS;
                 kmajor(k_lo + ks * kTileStep, kd);
                 FIA_WAIT(&k_full[ks], (kv_base / KS) & 1, 21);
-                __syncwarp();
                 tc_fence_after();
-                if (lane == 0) {
-                    if (gm.nA > 0) {
-                        kmajor(q_lo, qd);
-                        qk(0, qd, kd);
-                        umma_commit(&s_full[0]);
-                    }
-                    kmajor(q_lo + kTileStep, qd);
-                    qk(1, qd, kd);
-                    umma_commit(&s_full[1]);
-                    umma_commit(&k_empty[ks]);
-                    if (gm.nB == 1) umma_commit(q_empty);
+                if (gm.nA > 0) {
+                    kmajor(q_lo, qd);
+                    qk(0, qd, kd);
+                    umma_commit(&s_full[0]);
                 }
-                __syncwarp();
+                kmajor(q_lo + kTileStep, qd);
+                qk(1, qd, kd);
+                umma_commit(&s_full[1]);
+                umma_commit(&k_empty[ks]);
+                if (gm.nB == 1) umma_commit(q_empty);
             }
             for (int j = 0; j < gm.nB; ++j) {
                 dbg_j = j;
@@ -327,27 +335,24 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 vmajor(v_lo + vs * kTileStep, vd);
                 kmajor(k_lo + ksn * kTileStep, kd);
                 FIA_WAIT(&v_full[vs], (kvi / VS) & 1, 24);
-                __syncwarp();
                 const int valid = gm.kvlen - j * kPrefillBN;
                 if (valid < kPrefillBN) {
-                    // rows past kvSeqLen: P is 0 there, but the slots may
-                    // hold anything (NaN * 0 = NaN in the MMA) -> zero them.
+                    // rows past kvSeqLen: P is 0 there, but the slots may hold
+                    // anything (NaN * 0 = NaN in the MMA): the bulk-copy engine
+                    // writes zeros over them after the V tile has landed.
                     uint8_t *vdst = smem + Cfg::kOffV + vs * Cfg::kTileBytes;
-                    const int nbytes = (kPrefillBN - valid) * 128;
-                    for (int hv = 0; hv < Cfg::kHalves; ++hv) {
-                        uint4 *p = reinterpret_cast<uint4 *>(vdst + hv * Cfg::kGroupBytes + valid * 128);
-                        for (int x = lane; x < nbytes / 16; x += 32) p[x] = make_uint4(0, 0, 0, 0);
-                    }
-                    fence_proxy_async_smem();
-                    __syncwarp();
+                    const uint32_t nbytes = (uint32_t)(kPrefillBN - valid) * 128u;
+                    mbar_arrive_expect_tx(vz_full, nbytes * Cfg::kHalves);
+                    for (int hv = 0; hv < Cfg::kHalves; ++hv)
+                        bulk_load(vdst + hv * Cfg::kGroupBytes + valid * 128, g_zero_rows, nbytes,
+                                  vz_full);
+                    FIA_WAIT(vz_full, vz_it & 1, 27);
+                    ++vz_it;
                 }
                 if constexpr (KS >= 2) {
                     // Every wait comes before a block, so each tile's PV(j) and
-                    // QK(j+1) go out back to back from one thread with only
-                    // commits between them (the issuing warp is starved of
-                    // issue slots by the softmax warps beside it, so any
-                    // instruction between two blocks leaves the tensor pipe
-                    // idle).  K(j+1) was requested a whole key tile earlier:
+                    // QK(j+1) go out back to back with only commits between
+                    // them.  K(j+1) was requested a whole key tile earlier:
                     // waiting for it up front almost never waits.
                     if (more) FIA_WAIT(&k_full[ksn], (kn / KS) & 1, 22);
                     if (j < gm.nA) {
@@ -355,40 +360,32 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                         kmajor(q_lo, qd);
                         FIA_WAIT(&p_full[0], p_it[0] & 1, 23);
                         ++p_it[0];
-                        __syncwarp();
                         tc_fence_after();
-                        if (lane == 0) {
-                            umma_ts_x8(tmem + Cfg::col_o(0), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
-                            umma_commit(&pv_done[0]);
-                            if (j + 1 < gm.nA) {
-                                qk(0, qd, kd);
-                                umma_commit(&s_full[0]);
-                            } else {
-                                umma_commit(&o_full[0]);
-                            }
+                        umma_ts_x8(tmem + Cfg::col_o(0), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
+                        umma_commit(&pv_done[0]);
+                        if (j + 1 < gm.nA) {
+                            qk(0, qd, kd);
+                            umma_commit(&s_full[0]);
+                        } else {
+                            umma_commit(&o_full[0]);
                         }
-                        __syncwarp();
                     }
                     ptmem(1, pa);
                     kmajor(q_lo + kTileStep, qd);
                     FIA_WAIT(&p_full[1], p_it[1] & 1, 25);
                     ++p_it[1];
-                    __syncwarp();
                     tc_fence_after();
-                    if (lane == 0) {
-                        umma_ts_x8(tmem + Cfg::col_o(1), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
-                        umma_commit(&pv_done[1]);
-                        umma_commit(&v_empty[vs]);
-                        if (more) {
-                            qk(1, qd, kd);
-                            umma_commit(&s_full[1]);
-                            umma_commit(&k_empty[ksn]);
-                            if (j + 1 == gm.nB - 1) umma_commit(q_empty);
-                        } else {
-                            umma_commit(&o_full[1]);
-                        }
+                    umma_ts_x8(tmem + Cfg::col_o(1), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
+                    umma_commit(&pv_done[1]);
+                    umma_commit(&v_empty[vs]);
+                    if (more) {
+                        qk(1, qd, kd);
+                        umma_commit(&s_full[1]);
+                        umma_commit(&k_empty[ksn]);
+                        if (j + 1 == gm.nB - 1) umma_commit(q_empty);
+                    } else {
+                        umma_commit(&o_full[1]);
                     }
-                    __syncwarp();
                 } else {
                     // One K stage: K(j+1) is loaded only after QK(j) of both
                     // tiles, so it is waited for between the PV and QK blocks.
@@ -397,49 +394,33 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                         kmajor(q_lo, qd);
                         FIA_WAIT(&p_full[0], p_it[0] & 1, 23);
                         ++p_it[0];
-                        __syncwarp();
                         tc_fence_after();
-                        if (lane == 0) {
-                            umma_ts_x8(tmem + Cfg::col_o(0), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
-                            umma_commit(&pv_done[0]);
-                            if (j == gm.nA - 1) umma_commit(&o_full[0]);
-                        }
-                        __syncwarp();
+                        umma_ts_x8(tmem + Cfg::col_o(0), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
+                        umma_commit(&pv_done[0]);
+                        if (j == gm.nA - 1) umma_commit(&o_full[0]);
                         if (j + 1 < gm.nA) {
                             FIA_WAIT(&k_full[ksn], (kn / KS) & 1, 22);
-                            __syncwarp();
                             tc_fence_after();
-                            if (lane == 0) {
-                                qk(0, qd, kd);
-                                umma_commit(&s_full[0]);
-                            }
-                            __syncwarp();
+                            qk(0, qd, kd);
+                            umma_commit(&s_full[0]);
                         }
                     }
                     ptmem(1, pa);
                     kmajor(q_lo + kTileStep, qd);
                     FIA_WAIT(&p_full[1], p_it[1] & 1, 25);
                     ++p_it[1];
-                    __syncwarp();
                     tc_fence_after();
-                    if (lane == 0) {
-                        umma_ts_x8(tmem + Cfg::col_o(1), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
-                        umma_commit(&pv_done[1]);
-                        umma_commit(&v_empty[vs]);
-                        if (j == gm.nB - 1) umma_commit(&o_full[1]);
-                    }
-                    __syncwarp();
+                    umma_ts_x8(tmem + Cfg::col_o(1), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
+                    umma_commit(&pv_done[1]);
+                    umma_commit(&v_empty[vs]);
+                    if (j == gm.nB - 1) umma_commit(&o_full[1]);
                     if (more) {
                         FIA_WAIT(&k_full[ksn], (kn / KS) & 1, 26);
-                        __syncwarp();
                         tc_fence_after();
-                        if (lane == 0) {
-                            qk(1, qd, kd);
-                            umma_commit(&s_full[1]);
-                            umma_commit(&k_empty[ksn]);
-                            if (j + 1 == gm.nB - 1) umma_commit(q_empty);
-                        }
-                        __syncwarp();
+                        qk(1, qd, kd);
+                        umma_commit(&s_full[1]);
+                        umma_commit(&k_empty[ksn]);
+                        if (j + 1 == gm.nB - 1) umma_commit(q_empty);
                     }
                 }
             }
@@ -526,13 +507,25 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 // ---- scores (log2 units unless folded), bias, masks ----
                 const bool edge = (tb + 64 > gm.kvlen) || (causal && tb + 63 > qpos);
                 if constexpr (MODE == kModeAlibi) {
-                    const float base = slope2 * (float)(tb - qpos);
+                    // bias slope * (t - qpos) in log2 units, two keys at a time:
+                    // the key offset pair is carried as exact floats (integers
+                    // below 2^24), so each bias is one rounding of slope * offset
+                    const float t0 = (float)(tb - qpos);
+                    const uint64_t sp2 = f2pack(slope2, slope2), sl2x2 = f2pack(sl2, sl2);
+                    const uint64_t two2 = f2pack(2.f, 2.f);
+                    uint64_t off2 = f2pack(t0, t0 + 1.f);
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc)
 #pragma unroll
-                        for (int x = 0; x < 32; ++x) {
-                            const float bias = fmaf(slope2, (float)(cc * 32 + x), base);
-                            sr[cc][x] = __float_as_uint(fmaf(__uint_as_float(sr[cc][x]), sl2, bias));
+                        for (int x = 0; x < 16; ++x) {
+                            const uint64_t s2 = f2pack(__uint_as_float(sr[cc][2 * x]),
+                                                       __uint_as_float(sr[cc][2 * x + 1]));
+                            const uint64_t y2 = ffma2(s2, sl2x2, fmul2(sp2, off2));
+                            float y0, y1;
+                            f2unpack(y2, y0, y1);
+                            sr[cc][2 * x] = __float_as_uint(y0);
+                            sr[cc][2 * x + 1] = __float_as_uint(y1);
+                            off2 = fadd2(off2, two2);
                         }
                 } else if (MODE == kModePse && pse_tma) {
                     // this lane's row of pse box `half` for tile j (128-byte swizzle)
@@ -734,6 +727,7 @@ done:
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
+        __syncwarp();          // lanes 1-31 left the issuer role early; dealloc is .aligned
         tc_fence_after();
         tmem_dealloc(tmem, Cfg::kTmemCols);
     }
