@@ -8,24 +8,25 @@
 // (O, m, l), and a second kernel merges the splits with the lse rule of the
 // V3 "lse" bullet (max, rescaled exponent sums, log of the sum added back).
 //
-// Kernel 1, fia_decode_kernel: one CTA per split unit (b, kvh, [t0, t1)).
-//   * K/V rows of the unit stream through a STAGES-deep ring of shared-memory
-//     tiles (64 keys each) filled by TMA: one 3-D box per (block run, 128-byte
-//     column group), the physical row coming from the block table, so every
-//     cached byte is fetched once, 128-byte swizzled for conflict-free reads.
-//   * 4 warps split each tile 16 keys apiece.  The g*qlen query rows of the
-//     group form the 16-row A operand of m16n8k16 tensor-core MMAs:
-//     S = Q K^T (keys as N), online softmax in fp32 on the accumulator
-//     fragments, then O += P V with P fed straight from registers.
-//   * int8 caches are widened to f16 in registers by placing each byte (+128)
-//     under the f16 exponent pattern for 1024, i.e. the exact value 1152 + x;
-//     the 1152 bias is removed afterwards (for K from the per-row constant,
-//     for V through a per-row sum of P from one extra MMA against ones).  The
-//     per-channel K scale is folded into q (with a power-of-two range fix), the
-//     K offset becomes one additive constant per row, and the V scale/offset
-//     are applied once in the combine.
-//   * Warps merge their (m, l, O) in shared memory and the CTA writes one
-//     partial per unit.
+// Kernel 1 (one CTA per split unit (b, kvh, [t0, t1))).  K/V rows of the unit
+// stream through a ring of shared-memory tiles (64 keys each) filled by TMA:
+// one 3-D box per (block run, 128-byte column group), the physical row coming
+// from the block table, so every cached byte is fetched once, 128-byte
+// swizzled.  4 warps split each tile 16 keys apiece and run m16n8k16
+// tensor-core MMAs; warps merge their (m, l, O) in shared memory and the CTA
+// writes one partial per unit.
+//   * fia_decode_kernel (fp16/bf16 cache): the g*qlen query rows of the
+//     group form the 16-row A operand; S = Q K^T (keys as N), online softmax
+//     in fp32 on the accumulator fragments, O += P V with P from registers.
+//   * fia_decode_i8_kernel (int8 cache): keys are the 16-row A operand and
+//     the query rows the N = 8 columns (S^T = K Q'^T, O^T = V^T P^T), so no
+//     MMA row is padding.  Bytes are widened to f16 in registers by placing
+//     each byte (+128) under the f16 exponent pattern for 1024, i.e. the
+//     exact value 1152 + x; the 1152 bias is removed afterwards (for K from
+//     the per-row constant, for V through a per-row sum of P from one extra
+//     MMA against ones).  The per-channel K scale is folded into q (with a
+//     power-of-two range fix), the K offset becomes one additive constant per
+//     row, and the V scale/offset are applied once in the combine.
 // Kernel 2, fia_combine_kernel: one CTA per (b, kvh, row); merges the unit
 //   partials in fixed logical order (deterministic), adds the learnable sink
 //   to the denominator, applies int8 V dequantisation, writes out and lse.
@@ -42,9 +43,9 @@
 
 namespace fia {
 
-template <int D, bool INT8>
+template <int D>
 struct DecodeCfg {
-    static constexpr int kRowBytes = D * (INT8 ? 1 : 2);
+    static constexpr int kRowBytes = D * 2;
     static constexpr int kHalves = kRowBytes / 128;               // 128-byte column groups
     static constexpr int kTileBytes = kDecodeTile * kRowBytes;    // one of K or V
     static constexpr int kStages = (2 * kTileBytes >= 32768) ? 3 : 4;
@@ -56,20 +57,17 @@ struct DecodeCfg {
     static_assert(kRowBytes % 128 == 0, "row must be a whole number of 128-byte groups");
 };
 
-int decode_smem_bytes(int D, bool kv_int8) {
-    if (D == 64) return kv_int8 ? -1 : DecodeCfg<64, false>::kSmem;
-    if (D == 128) return kv_int8 ? DecodeCfg<128, true>::kSmem : DecodeCfg<128, false>::kSmem;
-    return -1;
-}
+struct DecodeI8Cfg;
+int decode_smem_bytes(int D, bool kv_int8);
 
-template <typename T, int D, bool INT8>
-__global__ void __launch_bounds__(128, INT8 ? 3 : 2)
+template <typename T, int D>
+__global__ void __launch_bounds__(128, 2)
 fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv) {
-    using Cfg = DecodeCfg<D, INT8>;
+    using Cfg = DecodeCfg<D>;
     constexpr int STAGES = Cfg::kStages;
     constexpr int KT = D / 16;           // k-steps of the QK^T MMA
-    constexpr bool MMA_BF16 = INT8 ? false : MmaType<T>::bf16;
+    constexpr bool MMA_BF16 = MmaType<T>::bf16;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -118,7 +116,7 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
             const int prow = blk * a.c.bs + (t % a.c.bs);
             for (int hv = 0; hv < Cfg::kHalves; ++hv) {
                 const int off = hv * kDecodeTile * 128 + bi * br * 128;
-                const int col = INT8 ? hv * 128 : hv * 64;
+                const int col = hv * 64;
                 tma_load_3d(kst + off, &tk, &full[s], col, u.kvh, prow);
                 tma_load_3d(vst + off, &tv, &full[s], col, u.kvh, prow);
             }
@@ -141,80 +139,15 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
     const T *qb_ptr = qp + ((int64_t)(si.cu_q + qi_b) * a.c.H + head_b) * D;
 
     uint32_t qf[KT][4];
-    float sc_a = a.c.scale_log2, sc_b = a.c.scale_log2;   // multiplies the raw accumulator
-    float add_a = 0.f, add_b = 0.f;                       // per-row additive term (log2 units)
-    if constexpr (!INT8) {
+    const float sc_a = a.c.scale_log2, sc_b = a.c.scale_log2;   // multiplies the raw accumulator
+    const float add_a = 0.f, add_b = 0.f;                       // per-row additive term (log2 units)
 #pragma unroll
-        for (int kk = 0; kk < KT; ++kk) {
-            const int d0 = kk * 16 + 2 * c;
-            qf[kk][0] = va ? *reinterpret_cast<const uint32_t *>(qa_ptr + d0) : 0u;
-            qf[kk][1] = vb ? *reinterpret_cast<const uint32_t *>(qb_ptr + d0) : 0u;
-            qf[kk][2] = va ? *reinterpret_cast<const uint32_t *>(qa_ptr + d0 + 8) : 0u;
-            qf[kk][3] = vb ? *reinterpret_cast<const uint32_t *>(qb_ptr + d0 + 8) : 0u;
-        }
-    } else {
-        // q'_d = q_d * kScale_d (fp32).  This thread holds dims 16kk+4c+{0..3};
-        // the same order is used for the int8 key words below.
-        const float *ks = a.k_scale + u.kvh * D;
-        const float *ko = a.k_offset ? a.k_offset + u.kvh * D : nullptr;
-        float qa[KT][4], qb[KT][4];
-        float mx_a = 0.f, mx_b = 0.f, cs_a = 0.f, cs_b = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < KT; ++kk) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int d = kk * 16 + 4 * c + e;
-                const float s = ks[d];
-                const float o = ko ? ko[d] : 0.f;
-                qa[kk][e] = va ? to_f32<T>(qa_ptr[d]) * s : 0.f;
-                qb[kk][e] = vb ? to_f32<T>(qb_ptr[d]) * s : 0.f;
-                mx_a = fmaxf(mx_a, fabsf(qa[kk][e]));
-                mx_b = fmaxf(mx_b, fabsf(qb[kk][e]));
-                cs_a = fmaf(qa[kk][e], o, cs_a);
-                cs_b = fmaf(qb[kk][e], o, cs_b);
-            }
-        }
-#pragma unroll
-        for (int x = 1; x <= 2; x <<= 1) {
-            mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, x));
-            mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, x));
-            cs_a += __shfl_xor_sync(0xffffffffu, cs_a, x);
-            cs_b += __shfl_xor_sync(0xffffffffu, cs_b, x);
-        }
-        // Scale each row by a power of two so that max|q'| lands below 2^11
-        // (well inside f16 range), then undo it on the fp32 accumulator.
-        int ea = 0, eb = 0;
-        if (mx_a > 0.f) { frexpf(mx_a, &ea); ea = 11 - ea; }
-        if (mx_b > 0.f) { frexpf(mx_b, &eb); eb = 11 - eb; }
-#pragma unroll
-        for (int kk = 0; kk < KT; ++kk) {
-            qf[kk][0] = pack2<__half>(ldexpf(qa[kk][0], ea), ldexpf(qa[kk][1], ea));
-            qf[kk][1] = pack2<__half>(ldexpf(qb[kk][0], eb), ldexpf(qb[kk][1], eb));
-            qf[kk][2] = pack2<__half>(ldexpf(qa[kk][2], ea), ldexpf(qa[kk][3], ea));
-            qf[kk][3] = pack2<__half>(ldexpf(qb[kk][2], eb), ldexpf(qb[kk][3], eb));
-        }
-        sc_a = ldexpf(a.c.scale_log2, -ea);
-        sc_b = ldexpf(a.c.scale_log2, -eb);
-        // The MMA sees each key byte as the f16 value 1152 + k (see the QK loop),
-        // so the raw score carries 1152 * sum_d q'_d, with q' exactly as the MMA
-        // saw it (f16): remove it here, together with the key offset term.
-        float sq_a = 0.f, sq_b = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < KT; ++kk) {
-            const float2 fa0 = __half22float2(*reinterpret_cast<const __half2 *>(&qf[kk][0]));
-            const float2 fa1 = __half22float2(*reinterpret_cast<const __half2 *>(&qf[kk][2]));
-            const float2 fb0 = __half22float2(*reinterpret_cast<const __half2 *>(&qf[kk][1]));
-            const float2 fb1 = __half22float2(*reinterpret_cast<const __half2 *>(&qf[kk][3]));
-            sq_a += (fa0.x + fa0.y) + (fa1.x + fa1.y);
-            sq_b += (fb0.x + fb0.y) + (fb1.x + fb1.y);
-        }
-#pragma unroll
-        for (int x = 1; x <= 2; x <<= 1) {
-            sq_a += __shfl_xor_sync(0xffffffffu, sq_a, x);
-            sq_b += __shfl_xor_sync(0xffffffffu, sq_b, x);
-        }
-        add_a = cs_a * a.c.scale_log2 - 1152.0f * sq_a * sc_a;
-        add_b = cs_b * a.c.scale_log2 - 1152.0f * sq_b * sc_b;
+    for (int kk = 0; kk < KT; ++kk) {
+        const int d0 = kk * 16 + 2 * c;
+        qf[kk][0] = va ? *reinterpret_cast<const uint32_t *>(qa_ptr + d0) : 0u;
+        qf[kk][1] = vb ? *reinterpret_cast<const uint32_t *>(qb_ptr + d0) : 0u;
+        qf[kk][2] = va ? *reinterpret_cast<const uint32_t *>(qa_ptr + d0 + 8) : 0u;
+        qf[kk][3] = vb ? *reinterpret_cast<const uint32_t *>(qb_ptr + d0 + 8) : 0u;
     }
     const bool causal = (a.c.mask_type == 9 || a.c.mask_type == 3);
     const bool alibi = a.c.mask_type == 3;
@@ -228,9 +161,6 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
     }
 
     float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
-    // int8: sum of the (f16-rounded) P each row fed to the MMA, to remove the
-    // 1152 bias of the value operand (see the PV loop)
-    float osum[4] = {0.f, 0.f, 0.f, 0.f};
     float o[D / 8][4];
 #pragma unroll
     for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
@@ -248,7 +178,7 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
         float sacc[2][4];
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
-        if constexpr (!INT8) {
+        {
             const int mi = lane >> 3;
             const int tok = warp * 16 + (mi >> 1) * 8 + (lane & 7);
 #pragma unroll
@@ -259,20 +189,6 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
                 ldsm_x4(addr, b00, b01, b10, b11);
                 mma_16816<MMA_BF16>(sacc[0], qf[kk], b00, b01);
                 mma_16816<MMA_BF16>(sacc[1], qf[kk], b10, b11);
-            }
-        } else {
-#pragma unroll
-            for (int kk = 0; kk < KT; ++kk) {
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    const int tok = warp * 16 + nt * 8 + r;
-                    // bytes biased to 128 + k under the f16 exponent pattern:
-                    // f16 values 1152 + k, exact; the 1152 * sum(q') term is
-                    // removed from the row constant above
-                    const uint32_t w = lds32(kst + swz128(tok, kk) + 4 * c) ^ 0x80808080u;
-                    mma_16816<false>(sacc[nt], qf[kk], prmt(w, 0x64646464u, 0x4140u),
-                                     prmt(w, 0x64646464u, 0x4342u));
-                }
             }
         }
 
@@ -351,22 +267,17 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
                 o[jj][0] *= al_a; o[jj][1] *= al_a;
                 o[jj][2] *= al_b; o[jj][3] *= al_b;
             }
-            if constexpr (INT8) {
-                osum[0] *= al_a; osum[1] *= al_a;
-                osum[2] *= al_b; osum[3] *= al_b;
-            }
         }
-        using PT = typename std::conditional<INT8, __half, T>::type;
         uint32_t pa[4];
-        pa[0] = pack2<PT>(sv[0][0], sv[0][1]);
-        pa[1] = pack2<PT>(sv[0][2], sv[0][3]);
-        pa[2] = pack2<PT>(sv[1][0], sv[1][1]);
-        pa[3] = pack2<PT>(sv[1][2], sv[1][3]);
+        pa[0] = pack2<T>(sv[0][0], sv[0][1]);
+        pa[1] = pack2<T>(sv[0][2], sv[0][3]);
+        pa[2] = pack2<T>(sv[1][0], sv[1][1]);
+        pa[3] = pack2<T>(sv[1][2], sv[1][3]);
 
         // ---- O += P V ----  (V rows past the unit's end are zeroed: P is 0
         // there but the slots may hold NaN garbage)
         const bool tail = (tw + 16 > u.t_end);
-        if constexpr (!INT8) {
+        {
             uint32_t mk0 = 0xffffffffu, mk1 = 0xffffffffu;
             if (tail) {
                 const int t0 = tw + 2 * c;
@@ -389,36 +300,6 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
             };
             if (tail) pv_tile(std::true_type{});
             else pv_tile(std::false_type{});
-        } else {
-            const int tk0 = warp * 16 + 2 * c;
-            const int tg = tw + 2 * c;
-            const uint32_t z0 = (tail && tg >= u.t_end) ? 0u : 0xffffffffu;
-            const uint32_t z1 = (tail && tg + 1 >= u.t_end) ? 0u : 0xffffffffu;
-            const uint32_t z2 = (tail && tg + 8 >= u.t_end) ? 0u : 0xffffffffu;
-            const uint32_t z3 = (tail && tg + 9 >= u.t_end) ? 0u : 0xffffffffu;
-#pragma unroll
-            for (int i = 0; i < D / 32; ++i) {
-                const int chunk = 2 * i + (r >> 2);
-                const int wo = 4 * (r & 3);
-                uint32_t w0 = lds32(vst + swz128(tk0, chunk) + wo);
-                uint32_t w1 = lds32(vst + swz128(tk0 + 1, chunk) + wo);
-                uint32_t w2 = lds32(vst + swz128(tk0 + 8, chunk) + wo);
-                uint32_t w3 = lds32(vst + swz128(tk0 + 9, chunk) + wo);
-                if (tail) { w0 &= z0; w1 &= z1; w2 &= z2; w3 &= z3; }
-                const uint32_t x01 = prmt(w0, w1, 0x5140u) ^ 0x80808080u;
-                const uint32_t x23 = prmt(w0, w1, 0x7362u) ^ 0x80808080u;
-                const uint32_t y01 = prmt(w2, w3, 0x5140u) ^ 0x80808080u;
-                const uint32_t y23 = prmt(w2, w3, 0x7362u) ^ 0x80808080u;
-                // values as f16 (1152 + v), exact; the bias is removed at the end
-                const uint32_t F = 0x64646464u;
-                mma_16816<false>(o[4 * i + 0], pa, prmt(x01, F, 0x4140u), prmt(y01, F, 0x4140u));
-                mma_16816<false>(o[4 * i + 1], pa, prmt(x01, F, 0x4342u), prmt(y01, F, 0x4342u));
-                mma_16816<false>(o[4 * i + 2], pa, prmt(x23, F, 0x4140u), prmt(y23, F, 0x4140u));
-                mma_16816<false>(o[4 * i + 3], pa, prmt(x23, F, 0x4342u), prmt(y23, F, 0x4342u));
-            }
-            // sum_t p~_t per row with the same rounding and accumulation as O
-            const uint32_t ones = 0x3C003C00u;   // f16x2 (1, 1)
-            mma_16816<false>(osum, pa, ones, ones);
         }
 
         __syncwarp();
@@ -445,25 +326,432 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
     for (int jj = 0; jj < D / 8; ++jj) {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            int d;
-            if constexpr (!INT8) {
-                d = jj * 8 + 2 * c + e;
-            } else {
-                // n-tile jj = 4i + q covers dims 32i + 4n + q for column n
-                d = (jj >> 2) * 32 + 4 * (2 * c + e) + (jj & 3);
-            }
-            if constexpr (INT8) {
-                oww[ra * D + d] = fmaf(-1152.0f, osum[0], o[jj][e]);
-                oww[rb * D + d] = fmaf(-1152.0f, osum[2], o[jj][2 + e]);
-            } else {
-                oww[ra * D + d] = o[jj][e];
-                oww[rb * D + d] = o[jj][2 + e];
-            }
+            const int d = jj * 8 + 2 * c + e;
+            oww[ra * D + d] = o[jj][e];
+            oww[rb * D + d] = o[jj][2 + e];
         }
     }
     if (c == 0) {
         mlw[warp * kDecodeRows + ra] = make_float2(m_a, l_a);
         mlw[warp * kDecodeRows + rb] = make_float2(m_b, l_b);
+    }
+    __syncthreads();
+    float *po = a.part_o + (int64_t)u.slot * kDecodeRows * D;
+    float2 *pml = a.part_ml + (int64_t)u.slot * kDecodeRows;
+    for (int idx = tid; idx < R * D; idx += blockDim.x) {
+        const int row = idx / D, d = idx % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, mlw[w * kDecodeRows + row].x);
+        float acc = 0.f, L = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float2 ml = mlw[w * kDecodeRows + row];
+                const float f = ex2(ml.x - M);
+                acc = fmaf(ow[(w * kDecodeRows + row) * D + d], f, acc);
+                L = fmaf(ml.y, f, L);
+            }
+        }
+        po[row * D + d] = acc;
+        if (d == 0) pml[row] = make_float2(M, L);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// int8 KV decode with the keys as the MMA row dimension.
+//
+// S^T = K Q'^T and O^T = V^T P^T: the 16 keys of a warp are the 16-row A
+// operand (widened from int8 in registers) and the query rows of the group
+// (g heads x qlen tokens) are the N = 8 column tiles (NT of them).  No MMA row
+// is padding, each (key, row) exponential is computed once, and the O^T
+// accumulator is 32 floats per thread per column tile, so four CTAs fit an SM.
+//   * K (A of S^T): key rows r and r + 8 of the warp; k-step kk = 4G + i
+//     covers dims 64G + 16c + 4i + {0..3} for thread column c, so one 16-byte
+//     shared load per key row brings four k-steps.  Q'^T (B) uses the same
+//     dims for query row 8nt + r.
+//   * P^T (B of O^T): the S^T accumulator packed to f16 and transposed in
+//     registers with movmatrix (keys x rows -> rows x keys).
+//   * V^T (A of O^T): M tile mt, row rho holds output dim
+//     64 (rho >> 3) + 8 (rho & 7) + mt, so a thread's dims of one key row are
+//     two runs of 8 contiguous bytes (two 8-byte shared loads).
+struct DecodeI8Cfg {
+    static constexpr int D = 128;
+    static constexpr int kTileBytes = kDecodeTile * D;          // one of K or V
+    static constexpr int kStageBytes = 2 * kTileBytes;
+    static constexpr int kStages = 3;
+    static constexpr int kMergeBytes = 4 * kDecodeRows * D * 4 + 4 * kDecodeRows * 8;
+    static constexpr int kDataBytes =
+        (kStages * kStageBytes > kMergeBytes) ? kStages * kStageBytes : kMergeBytes;
+    static constexpr int kSmem = 1024 /*align slack*/ + kDataBytes + 2 * kStages * 8 + 16;
+};
+
+int decode_smem_bytes(int D, bool kv_int8) {
+    if (kv_int8) return D == 128 ? DecodeI8Cfg::kSmem : -1;
+    if (D == 64) return DecodeCfg<64>::kSmem;
+    if (D == 128) return DecodeCfg<128>::kSmem;
+    return -1;
+}
+
+template <typename T, int NT>
+__global__ void __launch_bounds__(128, 4)
+fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ CUtensorMap tk,
+                     const __grid_constant__ CUtensorMap tv) {
+    using Cfg = DecodeI8Cfg;
+    constexpr int D = Cfg::D;
+    constexpr int STAGES = Cfg::kStages;
+    constexpr int KT = D / 16;                 // k-steps of S^T
+    constexpr int MT = D / 16;                 // M tiles of O^T
+    constexpr uint32_t F = 0x64646464u;        // f16 exponent bytes of 1024
+    static_assert(KT % 4 == 0, "keys are read 64 dims (4 k-steps) at a time");
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + Cfg::kDataBytes);
+    uint64_t *empty = full + STAGES;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + STAGES);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int r = lane >> 2;       // fragment row group
+    const int c = lane & 3;        // fragment column pair
+
+    const DecodeUnit u = a.units[blockIdx.x];
+    const SeqInfo si = a.c.seq[u.b];
+    const int g = a.c.g;
+    const int R = si.qlen * g;
+    const int n_tiles = (u.t_end - u.t_begin + kDecodeTile - 1) / kDecodeTile;
+
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 4);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tk);
+        tma_prefetch_desc(&tv);
+    }
+    __syncthreads();
+
+    const int32_t *bt_row = a.c.bt + (int64_t)u.b * a.c.bt_stride;
+    auto issue = [&](int j) {
+        const int s = j % STAGES;
+        const int t0 = u.t_begin + j * kDecodeTile;
+        const int t1 = min(t0 + kDecodeTile, u.t_end);
+        const int br = a.c.box_rows;
+        const int nbox = (t1 - t0 + br - 1) / br;
+        uint8_t *kst = smem + s * Cfg::kStageBytes;
+        uint8_t *vst = kst + Cfg::kTileBytes;
+        mbar_arrive_expect_tx(&full[s], (uint32_t)(nbox * br * 128 * 2));
+        for (int bi = 0; bi < nbox; ++bi) {
+            const int t = t0 + bi * br;
+            const int prow = bt_row[t / a.c.bs] * a.c.bs + (t % a.c.bs);
+            tma_load_3d(kst + bi * br * 128, &tk, &full[s], 0, u.kvh, prow);
+            tma_load_3d(vst + bi * br * 128, &tv, &full[s], 0, u.kvh, prow);
+        }
+    };
+    if (tid == 0) {
+        for (int j = 0; j < STAGES && j < n_tiles; ++j) issue(j);
+    }
+
+    // ---- Q'^T fragments: this thread holds query row nb = 8nt + r ----
+    // q'_d = q_d * kScale_d, scaled per row by a power of two so that
+    // max |q'| lands below 2^11 (inside f16 range); sc undoes it on the
+    // accumulator.  add = qkScale * sum_d q_d sK_d oK_d (key offset) minus
+    // 1152 * sum_d q'_d (the bias of the widened key bytes), in log2 units.
+    uint32_t qb[NT][KT][2];
+    float sc_b[NT], add_b[NT];
+    {
+        const T *qp = reinterpret_cast<const T *>(a.c.q);
+        const float *ks = a.k_scale + u.kvh * D;
+        const float *ko = a.k_offset ? a.k_offset + u.kvh * D : nullptr;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int nb = 8 * nt + r;
+            const bool vr = nb < R;
+            const int qi = vr ? nb / g : 0;
+            const int head = vr ? u.kvh * g + nb % g : 0;
+            const T *qrow = qp + ((int64_t)(si.cu_q + qi) * a.c.H + head) * D;
+            float qv[KT][4];
+            float mx = 0.f, cs = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < KT; ++kk) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int d = (kk >> 2) * 64 + 16 * c + 4 * (kk & 3) + e;
+                    const float o = ko ? ko[d] : 0.f;
+                    qv[kk][e] = vr ? to_f32<T>(qrow[d]) * ks[d] : 0.f;
+                    mx = fmaxf(mx, fabsf(qv[kk][e]));
+                    cs = fmaf(qv[kk][e], o, cs);
+                }
+            }
+#pragma unroll
+            for (int x = 1; x <= 2; x <<= 1) {
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, x));
+                cs += __shfl_xor_sync(0xffffffffu, cs, x);
+            }
+            int ex = 0;
+            if (mx > 0.f) { frexpf(mx, &ex); ex = 11 - ex; }
+            float sq = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < KT; ++kk) {
+                qb[nt][kk][0] = pack2<__half>(ldexpf(qv[kk][0], ex), ldexpf(qv[kk][1], ex));
+                qb[nt][kk][1] = pack2<__half>(ldexpf(qv[kk][2], ex), ldexpf(qv[kk][3], ex));
+                const float2 f0 = __half22float2(*reinterpret_cast<const __half2 *>(&qb[nt][kk][0]));
+                const float2 f1 = __half22float2(*reinterpret_cast<const __half2 *>(&qb[nt][kk][1]));
+                sq += (f0.x + f0.y) + (f1.x + f1.y);
+            }
+#pragma unroll
+            for (int x = 1; x <= 2; x <<= 1) sq += __shfl_xor_sync(0xffffffffu, sq, x);
+            sc_b[nt] = ldexpf(a.c.scale_log2, -ex);
+            add_b[nt] = cs * a.c.scale_log2 - 1152.0f * sq * sc_b[nt];
+        }
+    }
+
+    // ---- accumulator columns: this thread holds query rows 8nt + 2c + e ----
+    const bool causal = (a.c.mask_type == 9 || a.c.mask_type == 3);
+    const bool alibi = a.c.mask_type == 3;
+    float sc[NT][2], add[NT][2], slope[NT][2];
+    int qpos[NT][2];
+    bool vrow[NT][2];
+    const T *pse_row[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int n = 8 * nt + 2 * c + e;
+            // the B-layout thread holding row n is lane 4 (2c + e) of the column tile
+            sc[nt][e] = __shfl_sync(0xffffffffu, sc_b[nt], 4 * (2 * c + e));
+            add[nt][e] = __shfl_sync(0xffffffffu, add_b[nt], 4 * (2 * c + e));
+            vrow[nt][e] = n < R;
+            const int qi = vrow[nt][e] ? n / g : 0;
+            const int head = vrow[nt][e] ? u.kvh * g + n % g : 0;
+            qpos[nt][e] = si.kvlen - si.qlen + qi;
+            slope[nt][e] = (alibi && vrow[nt][e]) ? a.c.slopes[head] * kLog2e : 0.f;
+            pse_row[nt][e] = nullptr;
+            if (a.c.pse && vrow[nt][e])
+                pse_row[nt][e] = reinterpret_cast<const T *>(a.c.pse) +
+                                 (((int64_t)u.b * a.c.H + head) * a.c.pse_q + qi) * a.c.pse_kv;
+        }
+    }
+
+    float m[NT][2], l[NT][2];
+    float o[NT][MT][4];
+    float osum[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        m[nt][0] = m[nt][1] = -INFINITY;
+        l[nt][0] = l[nt][1] = 0.f;
+        osum[nt][0] = osum[nt][1] = osum[nt][2] = osum[nt][3] = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
+    }
+    const uint32_t ones = 0x3C003C00u;          // f16x2 (1, 1)
+    const uint32_t ones4[4] = {ones, ones, ones, ones};
+
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+        const int s = j % STAGES;
+        if (!mbar_wait(&full[s], (j / STAGES) & 1, abort_flag, a.c.err, 1)) { ok = false; break; }
+        __syncwarp();      // movmatrix / mma.sync below are warp-collective (.aligned)
+        const uint32_t kst = smem_u32(smem + s * Cfg::kStageBytes);
+        const uint32_t vst = kst + Cfg::kTileBytes;
+        const int tw = u.t_begin + j * kDecodeTile + warp * 16;   // first key of this warp
+
+        // ---- S^T = K Q'^T over this warp's 16 keys ----
+        float sacc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+        {
+            const int ka = warp * 16 + r, kb = ka + 8;
+#pragma unroll
+            for (int G = 0; G < KT / 4; ++G) {
+                uint32_t wa[4], wb[4];
+                lds128(kst + swz128(ka, 4 * G + c), wa);
+                lds128(kst + swz128(kb, 4 * G + c), wb);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    // bytes biased to 128 + k under the f16 exponent pattern:
+                    // f16 values 1152 + k, exact (the bias is in add)
+                    const uint32_t xa = wa[i] ^ 0x80808080u, xb = wb[i] ^ 0x80808080u;
+                    const uint32_t A[4] = {prmt(xa, F, 0x4140u), prmt(xb, F, 0x4140u),
+                                           prmt(xa, F, 0x4342u), prmt(xb, F, 0x4342u)};
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        mma_16816<false>(sacc[nt], A, qb[nt][4 * G + i][0], qb[nt][4 * G + i][1]);
+                }
+            }
+        }
+
+        // ---- scores, masks, online softmax (columns = query rows) ----
+        // accumulator element q of column tile nt: key tw + r + 8 (q >> 1),
+        // row 8nt + 2c + (q & 1)
+        const bool simple = !alibi && !a.c.pse && (tw + 16 <= u.t_end) &&
+                            (!causal || tw + 15 <= si.kvlen - si.qlen);
+        float sv[NT][4];
+        float mx[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int e = q & 1;
+                float x = fmaf(sacc[nt][q], sc[nt][e], add[nt][e]);
+                if (!simple) {
+                    const int t = tw + r + 8 * (q >> 1);
+                    const bool in = t < u.t_end;
+                    if (alibi) x = fmaf(slope[nt][e], (float)(t - qpos[nt][e]), x);
+                    if (pse_row[nt][e] && in) x = fmaf(to_f32<T>(pse_row[nt][e][t]), kLog2e, x);
+                    const bool keep = in && vrow[nt][e] && !(causal && t > qpos[nt][e]);
+                    x = keep ? x : -INFINITY;
+                }
+                sv[nt][q] = x;
+            }
+            mx[nt][0] = fmaxf(sv[nt][0], sv[nt][2]);
+            mx[nt][1] = fmaxf(sv[nt][1], sv[nt][3]);
+        }
+        if (!simple) __syncwarp();     // reconverge after the per-key pse loads
+#pragma unroll
+        for (int x = 4; x <= 16; x <<= 1)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                mx[nt][0] = fmaxf(mx[nt][0], __shfl_xor_sync(0xffffffffu, mx[nt][0], x));
+                mx[nt][1] = fmaxf(mx[nt][1], __shfl_xor_sync(0xffffffffu, mx[nt][1], x));
+            }
+        // Running max raised only when it grows by more than 2^8 (P stays
+        // <= 2^8, fine for f16); O, l and m stay mutually consistent.
+        bool up_any = false;
+        float al[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float mn = fmaxf(m[nt][e], mx[nt][e]);
+                al[nt][e] = 1.0f;
+                if (mn > m[nt][e] + 8.0f) {
+                    al[nt][e] = ex2(m[nt][e] - mn);
+                    m[nt][e] = mn;
+                    up_any = true;
+                }
+            }
+        }
+        __syncwarp();      // movmatrix and mma.sync below are .aligned
+        uint32_t pb[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const float mu0 = (m[nt][0] == -INFINITY) ? 0.f : m[nt][0];
+            const float mu1 = (m[nt][1] == -INFINITY) ? 0.f : m[nt][1];
+            const float p0 = ex2(sv[nt][0] - mu0), p1 = ex2(sv[nt][1] - mu1);
+            const float p2 = ex2(sv[nt][2] - mu0), p3 = ex2(sv[nt][3] - mu1);
+            l[nt][0] = fmaf(l[nt][0], al[nt][0], p0 + p2);
+            l[nt][1] = fmaf(l[nt][1], al[nt][1], p1 + p3);
+            // P^T fragments: (keys x rows) f16 tiles transposed to (rows x keys)
+            pb[nt][0] = movmatrix_trans(pack2<__half>(p0, p1));     // keys 2c, 2c+1
+            pb[nt][1] = movmatrix_trans(pack2<__half>(p2, p3));     // keys 2c+8, 2c+9
+        }
+        if (__any_sync(0xffffffffu, up_any)) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    o[nt][mt][0] *= al[nt][0]; o[nt][mt][1] *= al[nt][1];
+                    o[nt][mt][2] *= al[nt][0]; o[nt][mt][3] *= al[nt][1];
+                }
+                osum[nt][0] *= al[nt][0]; osum[nt][1] *= al[nt][1];
+                osum[nt][2] *= al[nt][0]; osum[nt][3] *= al[nt][1];
+            }
+        }
+
+        // ---- O^T += V^T P^T ----  (V rows past the unit's end are zeroed: P
+        // is 0 there but the slots may hold NaN garbage)
+        {
+            const int k0 = warp * 16 + 2 * c;
+            const int tg = tw + 2 * c;
+            const bool tail = (tw + 16 > u.t_end);
+            // dims 8r .. 8r+7 (rows rho = r) and 64 + 8r .. (rows rho = r + 8)
+            const uint32_t lo_off = ((uint32_t)(r >> 1) << 4), hi_off = ((uint32_t)(4 + (r >> 1)) << 4);
+            const uint32_t in8 = 8u * (uint32_t)(r & 1);
+            uint2 vl[4], vh[4];     // key rows k0, k0+1, k0+8, k0+9
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq) {
+                const int kr = k0 + (kq & 1) + 8 * (kq >> 1);
+                const uint32_t rowb = vst + (uint32_t)kr * 128u;
+                const uint32_t sw = (uint32_t)(kr & 7) << 4;
+                vl[kq] = lds64(rowb + (lo_off ^ sw) + in8);
+                vh[kq] = lds64(rowb + (hi_off ^ sw) + in8);
+                if (tail && tg + (kq & 1) + 8 * (kq >> 1) >= u.t_end) {
+                    vl[kq] = make_uint2(0u, 0u);
+                    vh[kq] = make_uint2(0u, 0u);
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {           // M tiles 4h .. 4h+3
+                const uint32_t a0 = h ? vl[0].y : vl[0].x, a1 = h ? vl[1].y : vl[1].x;
+                const uint32_t b0 = h ? vh[0].y : vh[0].x, b1 = h ? vh[1].y : vh[1].x;
+                const uint32_t c0 = h ? vl[2].y : vl[2].x, c1 = h ? vl[3].y : vl[3].x;
+                const uint32_t d0 = h ? vh[2].y : vh[2].x, d1 = h ? vh[3].y : vh[3].x;
+                // key pairs interleaved byte by byte, then biased (+128)
+                const uint32_t xa01 = prmt(a0, a1, 0x5140u) ^ 0x80808080u;   // rho r, keys 2c/2c+1
+                const uint32_t xa23 = prmt(a0, a1, 0x7362u) ^ 0x80808080u;
+                const uint32_t xb01 = prmt(b0, b1, 0x5140u) ^ 0x80808080u;   // rho r+8
+                const uint32_t xb23 = prmt(b0, b1, 0x7362u) ^ 0x80808080u;
+                const uint32_t xc01 = prmt(c0, c1, 0x5140u) ^ 0x80808080u;   // rho r, keys 2c+8/+9
+                const uint32_t xc23 = prmt(c0, c1, 0x7362u) ^ 0x80808080u;
+                const uint32_t xd01 = prmt(d0, d1, 0x5140u) ^ 0x80808080u;   // rho r+8
+                const uint32_t xd23 = prmt(d0, d1, 0x7362u) ^ 0x80808080u;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {       // M tile mt = 4h + q: byte q of each word
+                    const uint32_t sel = (q & 1) ? 0x4342u : 0x4140u;
+                    const uint32_t A[4] = {prmt((q < 2) ? xa01 : xa23, F, sel),
+                                           prmt((q < 2) ? xb01 : xb23, F, sel),
+                                           prmt((q < 2) ? xc01 : xc23, F, sel),
+                                           prmt((q < 2) ? xd01 : xd23, F, sel)};
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        mma_16816<false>(o[nt][4 * h + q], A, pb[nt][0], pb[nt][1]);
+                }
+            }
+            // sum_k p~ per row with the same rounding and accumulation as O
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_16816<false>(osum[nt], ones4, pb[nt][0], pb[nt][1]);
+        }
+
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        if (tid == 0 && j + STAGES < n_tiles) {
+            if (!mbar_wait(&empty[s], (j / STAGES) & 1, abort_flag, a.c.err, 2)) { ok = false; break; }
+            issue(j + STAGES);
+        }
+        __syncwarp();
+    }
+    (void)ok;
+
+    // ---- merge the 4 warps' (m, l, O) and write this unit's partial ----
+#pragma unroll
+    for (int x = 4; x <= 16; x <<= 1)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            l[nt][0] += __shfl_xor_sync(0xffffffffu, l[nt][0], x);
+            l[nt][1] += __shfl_xor_sync(0xffffffffu, l[nt][1], x);
+        }
+    __syncthreads();   // every warp is done with the stage buffers
+    float *ow = reinterpret_cast<float *>(smem);                               // [4][16][D]
+    float2 *mlw = reinterpret_cast<float2 *>(smem + 4 * kDecodeRows * D * 4);  // [4][16]
+    float *oww = ow + warp * kDecodeRows * D;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int n = 8 * nt + 2 * c + e;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                oww[n * D + 8 * r + mt] = fmaf(-1152.0f, osum[nt][e], o[nt][mt][e]);
+                oww[n * D + 64 + 8 * r + mt] = fmaf(-1152.0f, osum[nt][e], o[nt][mt][2 + e]);
+            }
+            if (r == 0) mlw[warp * kDecodeRows + n] = make_float2(m[nt][e], l[nt][e]);
+        }
     }
     __syncthreads();
     float *po = a.part_o + (int64_t)u.slot * kDecodeRows * D;
@@ -536,11 +824,22 @@ fia_combine_kernel(const __grid_constant__ CombineArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-template <typename T, int D, bool INT8>
+template <typename T, int D>
 static cudaError_t launch_decode_t(const DecodeArgs &a, const CUtensorMap &tk,
                                    const CUtensorMap &tv, int grid, cudaStream_t s) {
-    auto kern = fia_decode_kernel<T, D, INT8>;
-    const int smem = DecodeCfg<D, INT8>::kSmem;
+    auto kern = fia_decode_kernel<T, D>;
+    const int smem = DecodeCfg<D>::kSmem;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, 128, smem, s>>>(a, tk, tv);
+    return cudaGetLastError();
+}
+
+template <typename T, int NT>
+static cudaError_t launch_decode_i8_t(const DecodeArgs &a, const CUtensorMap &tk,
+                                      const CUtensorMap &tv, int grid, cudaStream_t s) {
+    auto kern = fia_decode_i8_kernel<T, NT>;
+    const int smem = DecodeI8Cfg::kSmem;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, 128, smem, s>>>(a, tk, tv);
@@ -551,14 +850,20 @@ cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap &tk, const CUte
                           int q_dtype, bool kv_int8, int grid, cudaStream_t s) {
     const bool bf = (q_dtype == 1);
     if (a.c.D == 128) {
-        if (kv_int8) return bf ? launch_decode_t<__nv_bfloat16, 128, true>(a, tk, tv, grid, s)
-                               : launch_decode_t<__half, 128, true>(a, tk, tv, grid, s);
-        return bf ? launch_decode_t<__nv_bfloat16, 128, false>(a, tk, tv, grid, s)
-                  : launch_decode_t<__half, 128, false>(a, tk, tv, grid, s);
+        if (kv_int8) {
+            // query rows per KV head: one or two N = 8 column tiles
+            if (a.max_rows <= 8)
+                return bf ? launch_decode_i8_t<__nv_bfloat16, 1>(a, tk, tv, grid, s)
+                          : launch_decode_i8_t<__half, 1>(a, tk, tv, grid, s);
+            return bf ? launch_decode_i8_t<__nv_bfloat16, 2>(a, tk, tv, grid, s)
+                      : launch_decode_i8_t<__half, 2>(a, tk, tv, grid, s);
+        }
+        return bf ? launch_decode_t<__nv_bfloat16, 128>(a, tk, tv, grid, s)
+                  : launch_decode_t<__half, 128>(a, tk, tv, grid, s);
     }
     if (a.c.D == 64 && !kv_int8)
-        return bf ? launch_decode_t<__nv_bfloat16, 64, false>(a, tk, tv, grid, s)
-                  : launch_decode_t<__half, 64, false>(a, tk, tv, grid, s);
+        return bf ? launch_decode_t<__nv_bfloat16, 64>(a, tk, tv, grid, s)
+                  : launch_decode_t<__half, 64>(a, tk, tv, grid, s);
     return cudaErrorInvalidValue;
 }
 

@@ -47,6 +47,7 @@ struct fia_op {
     size_t off_part_ml = 0, off_part_o = 0;
     uint64_t ws_size = 0;
     int32_t grid = 0, grid2 = 0;
+    int32_t max_rows = 0;           // decode: max seqLen * g
     int64_t work_items = 0;
     int32_t split_tokens = 0;
     cudaEvent_t ev_start = nullptr, ev_stop = nullptr;
@@ -359,6 +360,7 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
     std::vector<uint8_t> host;
     if (decode) {
         o->path = 1;
+        o->max_rows = (int32_t)(max_q * g);
         const bool causal = (maskType != FIA_MASK_NONE);
         (void)causal;
         int64_t total = 0;
@@ -543,6 +545,7 @@ fia_status fia_run(void *workspace, uint64_t workspaceSize, fia_op *op, void *st
         d.k_scale = op->k_scale;
         d.k_offset = op->k_offset;
         d.n_units = op->grid;
+        d.max_rows = op->max_rows;
         if (op->grid > 0) e = launch_decode(d, op->tk, op->tv, op->q_dtype, op->kv_int8, op->grid, s);
         if (e == cudaSuccess && op->grid2 > 0) {
             CombineArgs cb{};
@@ -634,6 +637,7 @@ fia_status fia_decode_run_static(fia_op *op, void *stream_ptr) {
     d.k_scale = op->k_scale;
     d.k_offset = op->k_offset;
     d.n_units = op->grid;
+    d.max_rows = op->max_rows;
     cudaError_t e = cudaSuccess;
     if (op->grid > 0) e = launch_decode(d, op->tk, op->tv, op->q_dtype, op->kv_int8, op->grid, s);
     if (e == cudaSuccess && op->grid2 > 0) {

@@ -67,6 +67,7 @@ struct DecodeArgs {
     float2 *part_ml;        // [slots][16] (m in log2 units, l)
     const float *k_scale, *k_offset;   // int8 only
     int32_t n_units;
+    int32_t max_rows;       // max over sequences of seqLen * g (<= kDecodeRows)
 };
 
 struct CombineArgs {
