@@ -174,7 +174,8 @@ def make_op(p, t):
                      [int(x) for x in p.seq_len], [int(x) for x in p.kv_seq_len], p.head_num,
                      p.kv_head_num, p.qk_scale, mask_type=p.mask_type, slopes=t["slopes"],
                      pse=t["pse"], sink=t["sink"], k_scale=t["k_scale"], k_offset=t["k_offset"],
-                     v_scale=t["v_scale"], v_offset=t["v_offset"], want_lse=p.want_lse)
+                     v_scale=t["v_scale"], v_offset=t["v_offset"], want_lse=p.want_lse,
+                     kv_layout=p.kv_layout)
 
 
 def time_op(op, steps, warmup, flush):
@@ -398,7 +399,9 @@ def main():
                          ("int8_long_decode", W.int8_long_decode),
                          ("alibi_prefill", lambda: W.alibi_prefill(False)),
                          ("alibi_prefill_pse", lambda: W.alibi_prefill(True)),
-                         ("tiny_decode", W.tiny_decode)):
+                         ("tiny_decode", W.tiny_decode),
+                         ("decode_large_batch_bnnbsd", W.decode_large_batch_bnnbsd),
+                         ("prefill_prefix_bnnbsd", W.prefill_prefix_bnnbsd)):
             q = fn()
             td = to_dev(q, dev)
             o2 = make_op(q, td)

@@ -83,6 +83,15 @@ typedef enum {
 } fia_mask_type;
 
 /* Optional extensions; the struct pointer and every field may be NULL. */
+/* Paged KV cache layout (aclnnFusedInferAttentionScoreV3, paged attention
+   constraints: the cache may be BnBsH or BnNBsD, BnNBsD being the one the page
+   recommends for performance).  key and value use the same layout.
+     FIA_KV_BNBSH   [numBlocks, blockSize, kvHeadNum, headSize] (4-D) or
+                    [numBlocks, blockSize, kvHeadNum * headSize] (3-D)
+     FIA_KV_BNNBSD  [numBlocks, kvHeadNum, blockSize, headSize] (4-D only): the
+                    rows of one (block, KV head) are contiguous. */
+typedef enum { FIA_KV_BNBSH = 0, FIA_KV_BNNBSD = 1 } fia_kv_layout;
+
 typedef struct {
     /* pse-shift bias [batch, headNum, maxQ, maxKV], the query's dtype, added to
        the scaled scores: s += pse[b][h][i][t] for new token i and key position t
@@ -105,6 +114,9 @@ typedef struct {
     /* lse output [nTokens, headNum] f32 (V3 "lse" bullet): m + log(sum exp(s - m)).
        Rows with no visible key get +inf. */
     fia_tensor *lse;
+    /* KV cache layout, a fia_kv_layout value (0, the default, is BnBsH).  A
+       zero-initialised fia_ext keeps the default. */
+    int32_t kvLayout;
 } fia_ext;
 
 typedef struct fia_op fia_op;

@@ -60,9 +60,9 @@ def _load():
             lib = ctypes.CDLL(_LIB_PATH)
             common = [_P, _I, _P, _P, _I, _I64, _I, _P, _I, _P, _P, _I, _I, _I, _I, _D, _I, _P,
                       _P, _I, _I, _I, _P, _P, _P, _P, _P]
-            lib.fia_oracle_attention.argtypes = common + [_P, _I64, _I, _P, _P]
+            lib.fia_oracle_attention.argtypes = common + [_P, _I64, _I, _P, _P, _I]
             lib.fia_oracle_attention.restype = _I
-            lib.fia_oracle_row_probs.argtypes = common + [_I, _I, _I, _P, _P, _P]
+            lib.fia_oracle_row_probs.argtypes = common + [_I, _I, _I, _P, _P, _P, _I]
             lib.fia_oracle_row_probs.restype = _I
             lib.fia_oracle_max_threads.restype = _I
             _lib = lib
@@ -78,6 +78,11 @@ def _ptr(t: Optional[torch.Tensor]):
         return None
     assert t.device.type == "cpu" and t.is_contiguous()
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _layout(p) -> int:
+    """KV cache layout of problem p: 0 BnBsH (default), 1 BnNBsD."""
+    return int(getattr(p, "kv_layout", 0))
 
 
 def _common(p, keep):
@@ -96,7 +101,9 @@ def _common(p, keep):
     pse_dt = _DT[pse.dtype] if pse is not None else 0
     pse_q = pse.shape[2] if pse is not None else 0
     pse_kv = pse.shape[3] if pse is not None else 0
-    return [_ptr(q), _DT[q.dtype], _ptr(kc), _ptr(vc), _DT[kc.dtype], kc.shape[0], kc.shape[1],
+    # block size: [numBlocks, blockSize, KVH, D] (BnBsH) or [numBlocks, KVH, blockSize, D]
+    bs = kc.shape[2] if _layout(p) == 1 else kc.shape[1]
+    return [_ptr(q), _DT[q.dtype], _ptr(kc), _ptr(vc), _DT[kc.dtype], kc.shape[0], bs,
             _ptr(bt), bt.shape[1], _ptr(sl), _ptr(kl), sl.shape[0],
             p.head_num, p.kv_head_num, q.shape[2], float(p.qk_scale), int(p.mask_type),
             _ptr(slopes), _ptr(pse), pse_dt, pse_q, pse_kv, _ptr(sink),
@@ -127,7 +134,7 @@ def attention(p, rows: Optional[Sequence[Tuple[int, int]]] = None,
     rc = lib.fia_oracle_attention(*args,
                                   rows_arr.ctypes.data_as(_P) if rows_arr is not None else None,
                                   n_rows, int(threads),
-                                  out.ctypes.data_as(_P), lse.ctypes.data_as(_P))
+                                  out.ctypes.data_as(_P), lse.ctypes.data_as(_P), _layout(p))
     if rc != 0:
         raise ValueError("oracle rejected the problem (code %d)" % rc)
     return out, lse
@@ -144,7 +151,7 @@ def row_probs(p, b: int, i: int, h: int) -> Tuple[np.ndarray, np.ndarray, float]
     out = np.zeros((p.query.shape[2],), dtype=np.float64)
     lse = np.zeros((1,), dtype=np.float64)
     rc = lib.fia_oracle_row_probs(*args, b, i, h, probs.ctypes.data_as(_P),
-                                  out.ctypes.data_as(_P), lse.ctypes.data_as(_P))
+                                  out.ctypes.data_as(_P), lse.ctypes.data_as(_P), _layout(p))
     if rc != 0:
         raise ValueError("oracle rejected the row (code %d)" % rc)
     return probs[:kvlen], out, float(lse[0])

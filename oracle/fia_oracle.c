@@ -21,7 +21,9 @@
  *                                                      seqLen[b] cache entries)
  *   2. for every logical kv position t < kvSeqLen[b]:
  *        blk = blockTables[b][t / blockSize], off = t % blockSize
- *        k_t = key[blk][off][kvh][:],  v_t = value[blk][off][kvh][:]
+ *        k_t = key[blk][off][kvh][:],  v_t = value[blk][off][kvh][:]   (BnBsH)
+ *        k_t = key[blk][kvh][off][:],  v_t = value[blk][kvh][off][:]   (BnNBsD;
+ *        V3 paged attention constraints: the cache is BnBsH or BnNBsD)
  *        int8 cache: k^ = kScale * (k + kOffset), v^ = vScale * (v + vOffset)
  *        per (kvh, d) channel; no offset given -> offset 0 (symmetric).
  *   3. causal (maskType 9, and 3 = ALiBi which includes causal): skip t > qpos
@@ -92,7 +94,15 @@ typedef struct {
     const void *pse; int pse_dtype; int pse_maxq; int pse_maxkv; /* or NULL    */
     const float *sink;                          /* [H] or NULL                 */
     const float *k_scale, *k_offset, *v_scale, *v_offset; /* [KVH, D] or NULL  */
+    int kv_layout;                              /* 0 BnBsH, 1 BnNBsD           */
 } oracle_args;
+
+/* Element offset of cache row (blk, off) of KV head kvh. */
+static int64_t cache_row(const oracle_args *a, int64_t blk, int off, int kvh) {
+    if (a->kv_layout == 1)
+        return ((blk * a->KVH + kvh) * a->bs + off) * (int64_t)a->D;
+    return ((blk * a->bs + off) * a->KVH + kvh) * (int64_t)a->D;
+}
 
 /* One (b, i, h) row.  probs (optional) receives the normalised weight of each
  * logical position t < kvSeqLen[b] (0 where masked).  Returns the number of
@@ -119,7 +129,7 @@ static int64_t oracle_row(const oracle_args *a, int b, int i, int h, int64_t tok
         if (causal && t > qpos) continue;
         int32_t blk = a->block_tables[(int64_t)b * a->max_blocks + t / a->bs];
         if (blk < 0 || blk >= a->num_blocks) { free(qv); free(s); free(keep); return -1; }
-        int64_t row = (((int64_t)blk * a->bs + t % a->bs) * a->KVH + kvh) * (int64_t)D;
+        int64_t row = cache_row(a, blk, t % a->bs, kvh);
         double dot = 0.0;
         for (int d = 0; d < D; ++d) {
             double kd = load_elem(a->k, a->kv_dtype, row + d);
@@ -158,7 +168,7 @@ static int64_t oracle_row(const oracle_args *a, int b, int i, int h, int64_t tok
         s[t] = p;
         l += p;
         int32_t blk = a->block_tables[(int64_t)b * a->max_blocks + t / a->bs];
-        int64_t row = (((int64_t)blk * a->bs + t % a->bs) * a->KVH + kvh) * (int64_t)D;
+        int64_t row = cache_row(a, blk, t % a->bs, kvh);
         for (int d = 0; d < D; ++d) {
             double vd = load_elem(a->v, a->kv_dtype, row + d);
             if (a->kv_dtype == OR_I8) {
@@ -190,14 +200,15 @@ int fia_oracle_attention(
     int H, int KVH, int D, double qk_scale, int mask_type, const float *slopes,
     const void *pse, int pse_dtype, int pse_maxq, int pse_maxkv, const float *sink,
     const float *k_scale, const float *k_offset, const float *v_scale, const float *v_offset,
-    const int64_t *rows, int64_t n_rows, int n_threads, double *out, double *lse) {
+    const int64_t *rows, int64_t n_rows, int n_threads, double *out, double *lse, int kv_layout) {
     if (H <= 0 || KVH <= 0 || H % KVH != 0 || D <= 0 || bs <= 0) return -2;
+    if (kv_layout != 0 && kv_layout != 1) return -2;
     if (kv_dtype == OR_I8 && (!k_scale || !v_scale)) return -2;
     if (mask_type == 3 && !slopes) return -2;
     oracle_args a = {q, q_dtype, k, v, kv_dtype, num_blocks, bs, block_tables, max_blocks,
                      seq_len, kv_seq_len, batch, H, KVH, D, qk_scale, mask_type, slopes,
                      pse, pse_dtype, pse_maxq, pse_maxkv, sink,
-                     k_scale, k_offset, v_scale, v_offset};
+                     k_scale, k_offset, v_scale, v_offset, kv_layout};
     /* token -> (b, i) */
     int64_t n_tokens = 0;
     for (int b = 0; b < batch; ++b) n_tokens += seq_len[b];
@@ -235,12 +246,13 @@ int fia_oracle_row_probs(
     int H, int KVH, int D, double qk_scale, int mask_type, const float *slopes,
     const void *pse, int pse_dtype, int pse_maxq, int pse_maxkv, const float *sink,
     const float *k_scale, const float *k_offset, const float *v_scale, const float *v_offset,
-    int b, int i, int h, double *probs, double *out, double *lse) {
+    int b, int i, int h, double *probs, double *out, double *lse, int kv_layout) {
     if (H <= 0 || KVH <= 0 || H % KVH != 0 || b < 0 || b >= batch) return -2;
+    if (kv_layout != 0 && kv_layout != 1) return -2;
     oracle_args a = {q, q_dtype, k, v, kv_dtype, num_blocks, bs, block_tables, max_blocks,
                      seq_len, kv_seq_len, batch, H, KVH, D, qk_scale, mask_type, slopes,
                      pse, pse_dtype, pse_maxq, pse_maxkv, sink,
-                     k_scale, k_offset, v_scale, v_offset};
+                     k_scale, k_offset, v_scale, v_offset, kv_layout};
     int64_t token = 0;
     for (int bb = 0; bb < b; ++bb) token += seq_len[bb];
     token += i;

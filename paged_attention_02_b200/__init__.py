@@ -17,11 +17,11 @@ from typing import Optional, Sequence
 import torch
 
 from . import _lib
-from ._lib import (FIA_MASK_ALIBI, FIA_MASK_CAUSAL, FIA_MASK_NONE, FiaError, fia_ext,
-                   fia_plan_info, fia_tensor)
+from ._lib import (FIA_KV_BNBSH, FIA_KV_BNNBSD, FIA_MASK_ALIBI, FIA_MASK_CAUSAL, FIA_MASK_NONE,
+                   FiaError, fia_ext, fia_plan_info, fia_tensor)
 
 __all__ = ["FiaOp", "fused_infer_attention", "FIA_MASK_NONE", "FIA_MASK_ALIBI",
-           "FIA_MASK_CAUSAL", "FiaError", "tensor_desc"]
+           "FIA_MASK_CAUSAL", "FIA_KV_BNBSH", "FIA_KV_BNNBSD", "FiaError", "tensor_desc"]
 
 _DT = {torch.float16: _lib.FIA_F16, torch.bfloat16: _lib.FIA_BF16, torch.float32: _lib.FIA_F32,
        torch.int8: _lib.FIA_I8, torch.int32: _lib.FIA_I32}
@@ -52,7 +52,8 @@ class FiaOp:
     """One planned call (phase 1 done); ``run()`` enqueues phase 2.
 
     Arguments follow ``fia_get_workspace_size``: query ``[nTokens, H, D]``,
-    key/value caches ``[numBlocks, blockSize, kvHeadNum, D]``, block table
+    key/value caches ``[numBlocks, blockSize, kvHeadNum, D]`` (``kv_layout=
+    FIA_KV_BNNBSD``: ``[numBlocks, kvHeadNum, blockSize, D]``), block table
     ``[batch, maxBlockNum]`` int32 (all on the same CUDA device), host
     sequence lengths.  ``out`` / ``lse`` are allocated when not given
     (``want_lse=False`` skips lse).  Tensors are referenced, not copied: keep
@@ -63,7 +64,7 @@ class FiaOp:
                  kv_seq_len: Sequence[int], head_num: int, kv_head_num: int, qk_scale: float,
                  mask_type: int = FIA_MASK_NONE, slopes=None, pse=None, sink=None, k_scale=None,
                  k_offset=None, v_scale=None, v_offset=None, out=None, lse=None,
-                 want_lse: bool = True):
+                 want_lse: bool = True, kv_layout: int = FIA_KV_BNBSH):
         dev = query.device
         self.out = out if out is not None else torch.empty_like(query)
         if lse is None and want_lse:
@@ -77,7 +78,7 @@ class FiaOp:
                         out=self.out, lse=self.lse).items()}
         self._ext = fia_ext(_ptr(self._d["pse"]), _ptr(self._d["sink"]), _ptr(self._d["ks"]),
                             _ptr(self._d["ko"]), _ptr(self._d["vs"]), _ptr(self._d["vo"]),
-                            _ptr(self._d["lse"]))
+                            _ptr(self._d["lse"]), int(kv_layout))
         b = len(seq_len)
         self._sl = (ctypes.c_int32 * max(b, 1))(*[int(x) for x in seq_len])
         self._kl = (ctypes.c_int32 * max(b, 1))(*[int(x) for x in kv_seq_len])
@@ -163,11 +164,11 @@ class FiaOp:
 def fused_infer_attention(query, key, value, block_tables, seq_len, kv_seq_len, head_num,
                           kv_head_num, qk_scale, mask_type=FIA_MASK_NONE, slopes=None, pse=None,
                           sink=None, k_scale=None, k_offset=None, v_scale=None, v_offset=None,
-                          want_lse=True):
+                          want_lse=True, kv_layout=FIA_KV_BNBSH):
     """One-shot call: plan, run on the current stream, return (out, lse)."""
     op = FiaOp(query, key, value, block_tables, seq_len, kv_seq_len, head_num, kv_head_num,
                qk_scale, mask_type, slopes, pse, sink, k_scale, k_offset, v_scale, v_offset,
-               want_lse=want_lse)
+               want_lse=want_lse, kv_layout=kv_layout)
     out, lse = op.run()
     op._keep.append(op.workspace)
     return out, lse

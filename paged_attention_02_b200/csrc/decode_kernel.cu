@@ -112,13 +112,13 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
         mbar_arrive_expect_tx(&full[s], (uint32_t)(nbox * br * 128 * Cfg::kHalves * 2));
         for (int bi = 0; bi < nbox; ++bi) {
             const int t = t0 + bi * br;
-            const int blk = bt_row[t / a.c.bs];
-            const int prow = blk * a.c.bs + (t % a.c.bs);
+            int y, z;
+            kv_box_yz(a.c, u.kvh, bt_row[t / a.c.bs], t % a.c.bs, y, z);
             for (int hv = 0; hv < Cfg::kHalves; ++hv) {
                 const int off = hv * kDecodeTile * 128 + bi * br * 128;
                 const int col = hv * 64;
-                tma_load_3d(kst + off, &tk, &full[s], col, u.kvh, prow);
-                tma_load_3d(vst + off, &tv, &full[s], col, u.kvh, prow);
+                tma_load_3d(kst + off, &tk, &full[s], col, y, z);
+                tma_load_3d(vst + off, &tv, &full[s], col, y, z);
             }
         }
     };
@@ -448,9 +448,10 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
         mbar_arrive_expect_tx(&full[s], (uint32_t)(nbox * br * 128 * 2));
         for (int bi = 0; bi < nbox; ++bi) {
             const int t = t0 + bi * br;
-            const int prow = bt_row[t / a.c.bs] * a.c.bs + (t % a.c.bs);
-            tma_load_3d(kst + bi * br * 128, &tk, &full[s], 0, u.kvh, prow);
-            tma_load_3d(vst + bi * br * 128, &tv, &full[s], 0, u.kvh, prow);
+            int y, z;
+            kv_box_yz(a.c, u.kvh, bt_row[t / a.c.bs], t % a.c.bs, y, z);
+            tma_load_3d(kst + bi * br * 128, &tk, &full[s], 0, y, z);
+            tma_load_3d(vst + bi * br * 128, &tv, &full[s], 0, y, z);
         }
     };
     if (tid == 0) {

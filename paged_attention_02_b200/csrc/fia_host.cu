@@ -82,14 +82,16 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 3-D tiled map over a row-major [rows, mid, inner] tensor, 128-byte swizzle.
+// 3-D tiled map over a row-major [rows, mid, inner] tensor, 128-byte swizzle;
+// the box is box_inner x box_mid x box_rows.
 bool encode_3d(CUtensorMap *m, CUtensorMapDataType dt, int esize, void *base, uint64_t inner,
-               uint64_t mid, uint64_t rows, uint32_t box_inner, uint32_t box_rows) {
+               uint64_t mid, uint64_t rows, uint32_t box_inner, uint32_t box_rows,
+               uint32_t box_mid = 1) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {inner, mid, rows};
     cuuint64_t strides[2] = {inner * esize, inner * mid * esize};
-    cuuint32_t box[3] = {box_inner, 1, box_rows};
+    cuuint32_t box[3] = {box_inner, box_mid, box_rows};
     cuuint32_t es[3] = {1, 1, 1};
     CUresult r = fn(m, dt, 3, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -168,15 +170,24 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
     if (numel(attnOut) != n_tokens * headNum * D || attnOut->dims[0] != n_tokens)
         return FIA_ERR_SHAPE;
     int64_t nb = 0, bs = 0;
-    if (key->ndim == 4) {
-        if (key->dims[2] != kvHeadNum || key->dims[3] != D) return FIA_ERR_SHAPE;
-    } else if (key->ndim == 3) {
-        if (key->dims[2] != (int64_t)kvHeadNum * D) return FIA_ERR_SHAPE;
+    const int32_t kv_layout = ext ? ext->kvLayout : (int32_t)FIA_KV_BNBSH;
+    if (kv_layout == FIA_KV_BNNBSD) {
+        if (key->ndim != 4 || key->dims[1] != kvHeadNum || key->dims[3] != D) return FIA_ERR_SHAPE;
+        nb = key->dims[0];
+        bs = key->dims[2];
+    } else if (kv_layout == FIA_KV_BNBSH) {
+        if (key->ndim == 4) {
+            if (key->dims[2] != kvHeadNum || key->dims[3] != D) return FIA_ERR_SHAPE;
+        } else if (key->ndim == 3) {
+            if (key->dims[2] != (int64_t)kvHeadNum * D) return FIA_ERR_SHAPE;
+        } else {
+            return FIA_ERR_SHAPE;
+        }
+        nb = key->dims[0];
+        bs = key->dims[1];
     } else {
-        return FIA_ERR_SHAPE;
+        return FIA_ERR_PARAM;
     }
-    nb = key->dims[0];
-    bs = key->dims[1];
     if (value->ndim != key->ndim) return FIA_ERR_SHAPE;
     for (int i = 0; i < key->ndim; ++i)
         if (value->dims[i] != key->dims[i]) return FIA_ERR_SHAPE;
@@ -301,6 +312,7 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
     c.g = g;
     c.D = (int32_t)D;
     c.bs = (int32_t)bs;
+    c.kv_layout = kv_layout;
     c.mask_type = maskType;
     c.scale_log2 = qkScale * 1.4426950408889634f;
     if (kv_int8) {
@@ -318,8 +330,18 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
     const uint32_t box_inner = kv_int8 ? 128u : 64u;
     const int box_rows = decode ? gcd_int((int)bs, kDecodeTile) : gcd_int((int)bs, kPrefillBN);
     c.box_rows = box_rows;
-    bool enc_ok = encode_3d(&o->tk, kdt, kv_es, key->data, D, kvHeadNum, nb * bs, box_inner, box_rows) &&
-                  encode_3d(&o->tv, kdt, kv_es, value->data, D, kvHeadNum, nb * bs, box_inner, box_rows);
+    // K/V maps: {D, KVH, blocks*bs} (BnBsH, box of one head x rows) or
+    // {D, bs, blocks*KVH} (BnNBsD, box of rows x one head); both land in
+    // shared memory as `rows` consecutive 128-byte rows
+    bool enc_ok;
+    if (kv_layout == FIA_KV_BNNBSD)
+        enc_ok = encode_3d(&o->tk, kdt, kv_es, key->data, D, bs, nb * kvHeadNum, box_inner, 1,
+                           box_rows) &&
+                 encode_3d(&o->tv, kdt, kv_es, value->data, D, bs, nb * kvHeadNum, box_inner, 1,
+                           box_rows);
+    else
+        enc_ok = encode_3d(&o->tk, kdt, kv_es, key->data, D, kvHeadNum, nb * bs, box_inner, box_rows) &&
+                 encode_3d(&o->tv, kdt, kv_es, value->data, D, kvHeadNum, nb * bs, box_inner, box_rows);
     if (!decode)
         enc_ok = enc_ok && encode_3d(&o->tq, tdt, 2, query->data, D, headNum, n_tokens, 64, kPrefillBM);
     if (!decode && pse && (pse->dims[3] % 8) == 0 && aligned16(pse->data)) {

@@ -57,8 +57,23 @@ struct CommonArgs {
     int32_t mask_type;
     int32_t pse_vec;        // pse rows 16-byte aligned (vector loads allowed)
     int32_t pse_tma;        // prefill: pse boxes fetched by TMA (tensor map tp)
+    int32_t kv_layout;      // 0: [blocks, bs, KVH, D]; 1: [blocks, KVH, bs, D]
     float scale_log2;       // qkScale * log2(e)
 };
+
+// TMA coordinates (y, z) of cache row `off` of block `blk`, KV head kvh, in
+// the K/V tensor maps: {D, KVH, blocks*bs} for layout 0, {D, bs, blocks*KVH}
+// for layout 1 (the box is one head x rows, or rows x one head).
+__device__ __forceinline__ void kv_box_yz(const CommonArgs &c, int kvh, int blk, int off, int &y,
+                                          int &z) {
+    if (c.kv_layout) {
+        y = off;
+        z = blk * c.KVH + kvh;
+    } else {
+        y = kvh;
+        z = blk * c.bs + off;
+    }
+}
 
 struct DecodeArgs {
     CommonArgs c;

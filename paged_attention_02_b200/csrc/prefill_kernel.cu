@@ -240,20 +240,22 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                     mbar_arrive_expect_tx(&k_full[ks], bytes);
                     for (int bi = 0; bi < nbox; ++bi) {
                         const int t = t0 + bi * br;
-                        const int prow = bt_row[t / a.c.bs] * a.c.bs + (t % a.c.bs);
+                        int y, z;
+                        kv_box_yz(a.c, gm.kvh, bt_row[t / a.c.bs], t % a.c.bs, y, z);
                         for (int hv = 0; hv < Cfg::kHalves; ++hv)
                             tma_load_3d(kd + hv * Cfg::kGroupBytes + bi * br * 128, &tk, &k_full[ks],
-                                        hv * 64, gm.kvh, prow);
+                                        hv * 64, y, z);
                     }
                     FIA_WAIT(&v_empty[vs], ((kv_it / VS) & 1) ^ 1, 12);
                     uint8_t *vd = smem + Cfg::kOffV + vs * Cfg::kTileBytes;
                     mbar_arrive_expect_tx(&v_full[vs], bytes);
                     for (int bi = 0; bi < nbox; ++bi) {
                         const int t = t0 + bi * br;
-                        const int prow = bt_row[t / a.c.bs] * a.c.bs + (t % a.c.bs);
+                        int y, z;
+                        kv_box_yz(a.c, gm.kvh, bt_row[t / a.c.bs], t % a.c.bs, y, z);
                         for (int hv = 0; hv < Cfg::kHalves; ++hv)
                             tma_load_3d(vd + hv * Cfg::kGroupBytes + bi * br * 128, &tv, &v_full[vs],
-                                        hv * 64, gm.kvh, prow);
+                                        hv * 64, y, z);
                     }
                 }
             }

@@ -60,7 +60,8 @@ def _call(**kw):
             args[k] = v
     d = {k: tensor_desc(v) for k, v in t.items()}
     P = lambda x: ctypes.pointer(x) if x is not None else None
-    ext = fia_ext(P(d["pse"]), P(d["sink"]), P(d["ks"]), None, P(d["vs"]), None, P(d["lse"]))
+    ext = fia_ext(P(d["pse"]), P(d["sink"]), P(d["ks"]), None, P(d["vs"]), None, P(d["lse"]),
+                  int(args.get("layout", 0)))
     n = max(len(args["seq"]), 1)
     sl = (ctypes.c_int32 * n)(*args["seq"])
     kl = (ctypes.c_int32 * n)(*args["kv"])
@@ -135,3 +136,21 @@ def test_run_rejects_null_op_and_missing_workspace():
     assert L.fia_run(None, 0, None, None) == L.FIA_ERR_NULLPTR
     assert L.fia_op_set_timing_events(None, None, None) == L.FIA_ERR_NULLPTR
     assert L.fia_op_get_plan_info(None, None) == L.FIA_ERR_NULLPTR
+
+
+def test_phase1_kv_layout_rules():
+    """BnNBsD cache [numBlocks, kvHeadNum, blockSize, headSize] (V3 paged
+    attention constraints: BnBsH or BnNBsD): validated by phase 1."""
+    from paged_attention_02_b200 import _lib as L
+    bn = lambda: torch.zeros(8, 2, 16, 128, dtype=torch.bfloat16)
+    assert _call(layout=2) == L.FIA_ERR_PARAM                                     # unknown layout
+    assert _call(layout=1) == L.FIA_ERR_SHAPE                                     # BnBsH dims given
+    assert _call(layout=1, k=torch.zeros(8, 16, 256, dtype=torch.bfloat16),
+                 v=torch.zeros(8, 16, 256, dtype=torch.bfloat16)) == L.FIA_ERR_SHAPE  # 3-D
+    assert _call(layout=1, k=bn(), v=torch.zeros(8, 2, 16, 64, dtype=torch.bfloat16)) == \
+        L.FIA_ERR_SHAPE                                                            # k != v
+    # valid BnNBsD inputs pass validation; without a GPU, phase 1 stops at the
+    # tensor-map encoding
+    assert _call(layout=1, k=bn(), v=bn()) in (L.FIA_ERR_CUDA, L.FIA_OK)
+    # the table must cover kvSeqLen with the BnNBsD block size (dims[2] = 16)
+    assert _call(layout=1, k=bn(), v=bn(), kv=[20, 80]) == L.FIA_ERR_SHAPE

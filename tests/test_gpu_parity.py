@@ -236,3 +236,45 @@ def test_config_alibi_prefill_and_pse_agree():
 def test_config_int8_long_decode_full():
     p = W.int8_long_decode()
     _full_size(p, 256, 4)
+
+
+# BnNBsD cache layout [numBlocks, kvHeadNum, blockSize, headSize] (V3 paged
+# attention constraints: BnBsH or BnNBsD, the latter recommended): the kernels
+# read each (block, KV head) run as one TMA box.  Checked against the oracle on
+# the same cache, and bitwise against the BnBsH run of the same problem (the
+# layout only changes where rows come from).
+BNNBSD_CASES = {
+    "decode_gqa4_bs16_ragged": dict(seq_len=[1] * 4, kv_seq_len=[1, 15, 700, 1000], head_num=16,
+                                    kv_head_num=4, head_size=128, block_size=16),
+    "decode_bs128_sink_f16": dict(seq_len=[1, 1], kv_seq_len=[513, 2049], head_num=16,
+                                  kv_head_num=2, head_size=128, block_size=128, dtype="f16",
+                                  sink=True),
+    "decode_int8_offsets_sink": dict(seq_len=[1, 1, 2], kv_seq_len=[300, 1025, 64], head_num=16,
+                                     kv_head_num=2, head_size=128, block_size=64, kv_dtype="i8",
+                                     sink=True),
+    "decode_mtp_causal_d64": dict(seq_len=[3, 1], kv_seq_len=[45, 260], head_num=8, kv_head_num=2,
+                                  head_size=64, block_size=32, mask_type=W.MASK_CAUSAL),
+    "prefill_causal_gqa_bs64": dict(seq_len=[130, 300], kv_seq_len=[130, 700], head_num=8,
+                                    kv_head_num=2, head_size=128, block_size=64,
+                                    mask_type=W.MASK_CAUSAL),
+    "prefill_alibi_mha_bs32_f16": dict(seq_len=[200], kv_seq_len=[333], head_num=4, kv_head_num=4,
+                                       head_size=128, block_size=32, dtype="f16",
+                                       mask_type=W.MASK_ALIBI, alibi_slopes=True),
+    "prefill_pse_causal_bs128": dict(seq_len=[140], kv_seq_len=[400], head_num=4, kv_head_num=2,
+                                     head_size=128, block_size=128, mask_type=W.MASK_CAUSAL,
+                                     pse=True),
+    "prefill_nomask_d64_bs16": dict(seq_len=[129, 40], kv_seq_len=[129, 90], head_num=4,
+                                    kv_head_num=1, head_size=64, block_size=16),
+}
+
+
+@pytest.mark.parametrize("name", sorted(BNNBSD_CASES))
+def test_bnnbsd_layout(name):
+    p = W.make_problem(name=name, seed=zlib.crc32(name.encode()) % 10000, spare_blocks=3,
+                       **BNNBSD_CASES[name])
+    q = W.to_bnnbsd(p)
+    _, out_q, lse_q = run_gpu(q)
+    ref_out, ref_lse = oracle.attention(q)
+    compare(out_q, lse_q, ref_out, ref_lse, name)
+    _, out_p, lse_p = run_gpu(p)
+    assert np.array_equal(out_q, out_p) and np.array_equal(lse_q, lse_p)

@@ -41,7 +41,7 @@ class Problem:
 
     name: str
     query: torch.Tensor                 # [nTokens, H, D]  f16 | bf16
-    key_cache: torch.Tensor             # [numBlocks, bs, KVH, D]  f16 | bf16 | i8
+    key_cache: torch.Tensor             # [numBlocks, bs, KVH, D] (kv_layout 1: [numBlocks, KVH, bs, D])
     value_cache: torch.Tensor           # same shape / dtype as key_cache
     block_tables: torch.Tensor          # [B, maxBlockNum] int32
     seq_len: np.ndarray                 # [B] int32 (host)
@@ -58,6 +58,7 @@ class Problem:
     v_scale: Optional[torch.Tensor] = None    # [KVH, D] f32
     v_offset: Optional[torch.Tensor] = None   # [KVH, D] f32
     want_lse: bool = True
+    kv_layout: int = 0                        # 0 BnBsH, 1 BnNBsD
 
     @property
     def batch(self) -> int:
@@ -69,7 +70,7 @@ class Problem:
 
     @property
     def block_size(self) -> int:
-        return int(self.key_cache.shape[1])
+        return int(self.key_cache.shape[2 if self.kv_layout == 1 else 1])
 
     @property
     def n_tokens(self) -> int:
@@ -115,6 +116,7 @@ def make_problem(
     int8_offsets: bool = True,
     want_lse: bool = True,
     max_blocks: Optional[int] = None,
+    kv_layout: int = 0,
 ) -> Problem:
     """Draw a seeded problem.
 
@@ -126,6 +128,8 @@ def make_problem(
       sequence's last block (e.g. NaN) to prove they are never read.
     * ALiBi slopes are ``2**(-8(h+1)/H)`` (caller-supplied, as the
       PrefixEncoder ``slopes`` parameter is).
+    * ``kv_layout=1``: the same cache stored BnNBsD ``[numBlocks, KVH, bs, D]``
+      (drawn as above, then transposed).
     * ``pse``: the ALiBi bias written out as a full ``[B, H, maxQ, maxKV]``
       tensor of the query dtype, ``pse[b,h,i,t] = slope_h * (t - qpos_i)``
       with ``qpos_i = kvSeqLen_b - seqLen_b + i``.
@@ -198,13 +202,24 @@ def make_problem(
             ko = torch.from_numpy((0.1 * rng.standard_normal((KVH, D))).astype(np.float32))
             vo = torch.from_numpy((0.1 * rng.standard_normal((KVH, D))).astype(np.float32))
 
-    return Problem(
+    p = Problem(
         name=name, query=query, key_cache=kc, value_cache=vc,
         block_tables=torch.from_numpy(bt), seq_len=seq_len, kv_seq_len=kv_seq_len,
         head_num=H, kv_head_num=KVH, qk_scale=float(qk_scale), mask_type=mask_type,
         slopes=slopes_t if mask_type == MASK_ALIBI else None, pse=pse_t, sink=sink_t,
         k_scale=ks, k_offset=ko, v_scale=vs, v_offset=vo, want_lse=want_lse,
     )
+    return to_bnnbsd(p) if kv_layout == 1 else p
+
+
+def to_bnnbsd(p: Problem) -> Problem:
+    """The same problem with its K/V pool stored BnNBsD ``[numBlocks, KVH, bs, D]``
+    (a pure transpose of the BnBsH pool; the block table is unchanged)."""
+    if p.kv_layout == 1:
+        return p
+    return dataclasses.replace(p, key_cache=p.key_cache.transpose(1, 2).contiguous(),
+                               value_cache=p.value_cache.transpose(1, 2).contiguous(),
+                               kv_layout=1)
 
 
 # ---------------------------------------------------------------------------
@@ -263,6 +278,16 @@ def int8_long_decode() -> Problem:
                         sink=True)
 
 
+def decode_large_batch_bnnbsd() -> Problem:
+    """decode_large_batch with its pool stored BnNBsD [numBlocks, KVH, bs, D]."""
+    return dataclasses.replace(to_bnnbsd(decode_large_batch()), name="decode_large_batch_bnnbsd")
+
+
+def prefill_prefix_bnnbsd() -> Problem:
+    """prefill_prefix with its pool stored BnNBsD [numBlocks, KVH, bs, D]."""
+    return dataclasses.replace(to_bnnbsd(prefill_prefix()), name="prefill_prefix_bnnbsd")
+
+
 NAMED = {
     "tiny_decode": tiny_decode,
     "prefill_prefix": prefill_prefix,
@@ -270,6 +295,8 @@ NAMED = {
     "alibi_prefill": lambda: alibi_prefill(False),
     "alibi_prefill_pse": lambda: alibi_prefill(True),
     "int8_long_decode": int8_long_decode,
+    "decode_large_batch_bnnbsd": decode_large_batch_bnnbsd,
+    "prefill_prefix_bnnbsd": prefill_prefix_bnnbsd,
 }
 
 
