@@ -92,6 +92,10 @@ typedef enum {
                     rows of one (block, KV head) are contiguous. */
 typedef enum { FIA_KV_BNBSH = 0, FIA_KV_BNNBSD = 1 } fia_kv_layout;
 
+/* int8 KV dequantisation modes (V3 fake-quantization: per-channel mode, and
+   per-token mode with scale/offset of shape (B, S) or (1, B, S), f32). */
+typedef enum { FIA_ANTIQUANT_PER_CHANNEL = 0, FIA_ANTIQUANT_PER_TOKEN = 1 } fia_antiquant_mode;
+
 typedef struct {
     /* pse-shift bias [batch, headNum, maxQ, maxKV], the query's dtype, added to
        the scaled scores: s += pse[b][h][i][t] for new token i and key position t
@@ -103,10 +107,18 @@ typedef struct {
        not scaled by qkScale, that joins the softmax denominator with no value
        row.  lse includes it. */
     const fia_tensor *sink;
-    /* int8 K/V dequantisation, per (kvHead, channel): [kvHeadNum, headSize] f32
-       (V3 fake-quantization bullets, per-channel mode).  The cache value x
-       stands for scale * (x + offset).  kScale and vScale are required when
-       key/value are FIA_I8; a NULL offset means 0 (symmetric). */
+    /* int8 K/V dequantisation (V3 fake-quantization bullets).  The cache value
+       x stands for scale * (x + offset).  kScale and vScale are required when
+       key/value are FIA_I8; a NULL offset means 0 (symmetric).  Per key / value
+       mode (kAntiquantMode / vAntiquantMode below):
+         FIA_ANTIQUANT_PER_CHANNEL  [kvHeadNum, headSize] f32: one pair per
+                                    (KV head, channel);
+         FIA_ANTIQUANT_PER_TOKEN    [batch, S] or [1, batch, S] f32 with
+                                    S >= max kvSeqLen: one pair per (sequence,
+                                    cached token position), shared by every
+                                    KV head and channel of that token.
+       Scale and offset of one operand use the same mode; K and V may differ
+       (e.g. per-channel keys with per-token values). */
     const fia_tensor *kScale;
     const fia_tensor *kOffset;
     const fia_tensor *vScale;
@@ -117,6 +129,10 @@ typedef struct {
     /* KV cache layout, a fia_kv_layout value (0, the default, is BnBsH).  A
        zero-initialised fia_ext keeps the default. */
     int32_t kvLayout;
+    /* int8 dequantisation modes of K and V, fia_antiquant_mode values (0, the
+       default, is per-channel). */
+    int32_t kAntiquantMode;
+    int32_t vAntiquantMode;
 } fia_ext;
 
 typedef struct fia_op fia_op;

@@ -60,9 +60,9 @@ def _load():
             lib = ctypes.CDLL(_LIB_PATH)
             common = [_P, _I, _P, _P, _I, _I64, _I, _P, _I, _P, _P, _I, _I, _I, _I, _D, _I, _P,
                       _P, _I, _I, _I, _P, _P, _P, _P, _P]
-            lib.fia_oracle_attention.argtypes = common + [_P, _I64, _I, _P, _P, _I]
+            lib.fia_oracle_attention.argtypes = common + [_P, _I64, _I, _P, _P, _I, _I, _I, _I64, _I64]
             lib.fia_oracle_attention.restype = _I
-            lib.fia_oracle_row_probs.argtypes = common + [_I, _I, _I, _P, _P, _P, _I]
+            lib.fia_oracle_row_probs.argtypes = common + [_I, _I, _I, _P, _P, _P, _I, _I, _I, _I64, _I64]
             lib.fia_oracle_row_probs.restype = _I
             lib.fia_oracle_max_threads.restype = _I
             _lib = lib
@@ -83,6 +83,15 @@ def _ptr(t: Optional[torch.Tensor]):
 def _layout(p) -> int:
     """KV cache layout of problem p: 0 BnBsH (default), 1 BnNBsD."""
     return int(getattr(p, "kv_layout", 0))
+
+
+def _quant_modes(p):
+    """(k_mode, v_mode, k_row_stride, v_row_stride): per-channel (0) or
+    per-token (1) int8 dequantisation; per-token tensors are [B, S]."""
+    km, vm = int(getattr(p, "k_antiquant_mode", 0)), int(getattr(p, "v_antiquant_mode", 0))
+    ks = p.k_scale.shape[-1] if (km == 1 and p.k_scale is not None) else 0
+    vs = p.v_scale.shape[-1] if (vm == 1 and p.v_scale is not None) else 0
+    return [km, vm, int(ks), int(vs)]
 
 
 def _common(p, keep):
@@ -134,7 +143,8 @@ def attention(p, rows: Optional[Sequence[Tuple[int, int]]] = None,
     rc = lib.fia_oracle_attention(*args,
                                   rows_arr.ctypes.data_as(_P) if rows_arr is not None else None,
                                   n_rows, int(threads),
-                                  out.ctypes.data_as(_P), lse.ctypes.data_as(_P), _layout(p))
+                                  out.ctypes.data_as(_P), lse.ctypes.data_as(_P), _layout(p),
+                                  *_quant_modes(p))
     if rc != 0:
         raise ValueError("oracle rejected the problem (code %d)" % rc)
     return out, lse
@@ -151,7 +161,8 @@ def row_probs(p, b: int, i: int, h: int) -> Tuple[np.ndarray, np.ndarray, float]
     out = np.zeros((p.query.shape[2],), dtype=np.float64)
     lse = np.zeros((1,), dtype=np.float64)
     rc = lib.fia_oracle_row_probs(*args, b, i, h, probs.ctypes.data_as(_P),
-                                  out.ctypes.data_as(_P), lse.ctypes.data_as(_P), _layout(p))
+                                  out.ctypes.data_as(_P), lse.ctypes.data_as(_P), _layout(p),
+                                  *_quant_modes(p))
     if rc != 0:
         raise ValueError("oracle rejected the row (code %d)" % rc)
     return probs[:kvlen], out, float(lse[0])

@@ -25,7 +25,9 @@
  *        k_t = key[blk][kvh][off][:],  v_t = value[blk][kvh][off][:]   (BnNBsD;
  *        V3 paged attention constraints: the cache is BnBsH or BnNBsD)
  *        int8 cache: k^ = kScale * (k + kOffset), v^ = vScale * (v + vOffset)
- *        per (kvh, d) channel; no offset given -> offset 0 (symmetric).
+ *        per (kvh, d) channel (per-channel mode) or per (b, t) cached token
+ *        (per-token mode, scale/offset [B, S], V3 fake-quantization
+ *        bullets; K and V modes may differ); no offset given -> offset 0.
  *   3. causal (maskType 9, and 3 = ALiBi which includes causal): skip t > qpos
  *   4. s_t = qkScale * sum_d q_d k_td
  *        + slope_h * (t - qpos)          (maskType 3)
@@ -95,7 +97,18 @@ typedef struct {
     const float *sink;                          /* [H] or NULL                 */
     const float *k_scale, *k_offset, *v_scale, *v_offset; /* [KVH, D] or NULL  */
     int kv_layout;                              /* 0 BnBsH, 1 BnNBsD           */
+    int k_mode, v_mode;                         /* 0 per-channel, 1 per-token  */
+    int64_t k_tok_stride, v_tok_stride;         /* per-token: row stride S     */
 } oracle_args;
+
+/* int8 dequantisation of cache value x of (sequence b, position t, channel
+ * d, KV head kvh): scale * (x + offset) with scale/offset chosen by mode. */
+static double dequant(const float *scale, const float *offset, int mode, int64_t tok_stride,
+                      int b, int64_t t, int kvh, int D, int d, double x) {
+    int64_t idx = mode == 1 ? (int64_t)b * tok_stride + t : (int64_t)kvh * D + d;
+    double off = offset ? (double)offset[idx] : 0.0;
+    return (double)scale[idx] * (x + off);
+}
 
 /* Element offset of cache row (blk, off) of KV head kvh. */
 static int64_t cache_row(const oracle_args *a, int64_t blk, int off, int kvh) {
@@ -133,10 +146,8 @@ static int64_t oracle_row(const oracle_args *a, int b, int i, int h, int64_t tok
         double dot = 0.0;
         for (int d = 0; d < D; ++d) {
             double kd = load_elem(a->k, a->kv_dtype, row + d);
-            if (a->kv_dtype == OR_I8) {
-                double off = a->k_offset ? a->k_offset[kvh * D + d] : 0.0;
-                kd = (double)a->k_scale[kvh * D + d] * (kd + off);
-            }
+            if (a->kv_dtype == OR_I8)
+                kd = dequant(a->k_scale, a->k_offset, a->k_mode, a->k_tok_stride, b, t, kvh, D, d, kd);
             dot += qv[d] * kd;
         }
         double st = a->qk_scale * dot;
@@ -171,10 +182,8 @@ static int64_t oracle_row(const oracle_args *a, int b, int i, int h, int64_t tok
         int64_t row = cache_row(a, blk, t % a->bs, kvh);
         for (int d = 0; d < D; ++d) {
             double vd = load_elem(a->v, a->kv_dtype, row + d);
-            if (a->kv_dtype == OR_I8) {
-                double off = a->v_offset ? a->v_offset[kvh * D + d] : 0.0;
-                vd = (double)a->v_scale[kvh * D + d] * (vd + off);
-            }
+            if (a->kv_dtype == OR_I8)
+                vd = dequant(a->v_scale, a->v_offset, a->v_mode, a->v_tok_stride, b, t, kvh, D, d, vd);
             out[d] += p * vd;
         }
     }
@@ -200,15 +209,18 @@ int fia_oracle_attention(
     int H, int KVH, int D, double qk_scale, int mask_type, const float *slopes,
     const void *pse, int pse_dtype, int pse_maxq, int pse_maxkv, const float *sink,
     const float *k_scale, const float *k_offset, const float *v_scale, const float *v_offset,
-    const int64_t *rows, int64_t n_rows, int n_threads, double *out, double *lse, int kv_layout) {
+    const int64_t *rows, int64_t n_rows, int n_threads, double *out, double *lse, int kv_layout,
+    int k_mode, int v_mode, int64_t k_tok_stride, int64_t v_tok_stride) {
     if (H <= 0 || KVH <= 0 || H % KVH != 0 || D <= 0 || bs <= 0) return -2;
     if (kv_layout != 0 && kv_layout != 1) return -2;
+    if (k_mode < 0 || k_mode > 1 || v_mode < 0 || v_mode > 1) return -2;
     if (kv_dtype == OR_I8 && (!k_scale || !v_scale)) return -2;
     if (mask_type == 3 && !slopes) return -2;
     oracle_args a = {q, q_dtype, k, v, kv_dtype, num_blocks, bs, block_tables, max_blocks,
                      seq_len, kv_seq_len, batch, H, KVH, D, qk_scale, mask_type, slopes,
                      pse, pse_dtype, pse_maxq, pse_maxkv, sink,
-                     k_scale, k_offset, v_scale, v_offset, kv_layout};
+                     k_scale, k_offset, v_scale, v_offset, kv_layout,
+                     k_mode, v_mode, k_tok_stride, v_tok_stride};
     /* token -> (b, i) */
     int64_t n_tokens = 0;
     for (int b = 0; b < batch; ++b) n_tokens += seq_len[b];
@@ -246,13 +258,16 @@ int fia_oracle_row_probs(
     int H, int KVH, int D, double qk_scale, int mask_type, const float *slopes,
     const void *pse, int pse_dtype, int pse_maxq, int pse_maxkv, const float *sink,
     const float *k_scale, const float *k_offset, const float *v_scale, const float *v_offset,
-    int b, int i, int h, double *probs, double *out, double *lse, int kv_layout) {
+    int b, int i, int h, double *probs, double *out, double *lse, int kv_layout,
+    int k_mode, int v_mode, int64_t k_tok_stride, int64_t v_tok_stride) {
     if (H <= 0 || KVH <= 0 || H % KVH != 0 || b < 0 || b >= batch) return -2;
     if (kv_layout != 0 && kv_layout != 1) return -2;
+    if (k_mode < 0 || k_mode > 1 || v_mode < 0 || v_mode > 1) return -2;
     oracle_args a = {q, q_dtype, k, v, kv_dtype, num_blocks, bs, block_tables, max_blocks,
                      seq_len, kv_seq_len, batch, H, KVH, D, qk_scale, mask_type, slopes,
                      pse, pse_dtype, pse_maxq, pse_maxkv, sink,
-                     k_scale, k_offset, v_scale, v_offset, kv_layout};
+                     k_scale, k_offset, v_scale, v_offset, kv_layout,
+                     k_mode, v_mode, k_tok_stride, v_tok_stride};
     int64_t token = 0;
     for (int bb = 0; bb < b; ++bb) token += seq_len[bb];
     token += i;

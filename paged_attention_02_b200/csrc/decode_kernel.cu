@@ -393,7 +393,7 @@ int decode_smem_bytes(int D, bool kv_int8) {
     return -1;
 }
 
-template <typename T, int NT>
+template <typename T, int NT, bool KTOK, bool VTOK>
 __global__ void __launch_bounds__(128, 4)
 fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv) {
@@ -459,16 +459,20 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
     }
 
     // ---- Q'^T fragments: this thread holds query row nb = 8nt + r ----
-    // q'_d = q_d * kScale_d, scaled per row by a power of two so that
-    // max |q'| lands below 2^11 (inside f16 range); sc undoes it on the
-    // accumulator.  add = qkScale * sum_d q_d sK_d oK_d (key offset) minus
+    // Per-channel K: q'_d = q_d * kScale_d, scaled per row by a power of two
+    // so that max |q'| lands below 2^11 (inside f16 range); sc undoes it on
+    // the accumulator.  add = qkScale * sum_d q_d sK_d oK_d (key offset) minus
     // 1152 * sum_d q'_d (the bias of the widened key bytes), in log2 units.
+    // Per-token K (scale sK_t, offset oK_t per cached token): q' = q, and a
+    // score is qkScale * sK_t * (sum_d q_d k_td + oK_t * sum_d q_d): sc and add
+    // stay in raw units and qs = sum_d q_d; sK_t and oK_t join per key.
+    constexpr bool ktok = KTOK, vtok = VTOK;     // per-token K / V (else per-channel)
     uint32_t qb[NT][KT][2];
-    float sc_b[NT], add_b[NT];
+    float sc_b[NT], add_b[NT], qs_b[NT];
     {
         const T *qp = reinterpret_cast<const T *>(a.c.q);
-        const float *ks = a.k_scale + u.kvh * D;
-        const float *ko = a.k_offset ? a.k_offset + u.kvh * D : nullptr;
+        const float *ks = ktok ? nullptr : a.k_scale + u.kvh * D;
+        const float *ko = (!ktok && a.k_offset) ? a.k_offset + u.kvh * D : nullptr;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const int nb = 8 * nt + r;
@@ -483,8 +487,8 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int d = (kk >> 2) * 64 + 16 * c + 4 * (kk & 3) + e;
-                    const float o = ko ? ko[d] : 0.f;
-                    qv[kk][e] = vr ? to_f32<T>(qrow[d]) * ks[d] : 0.f;
+                    const float o = ktok ? 1.f : (ko ? ko[d] : 0.f);
+                    qv[kk][e] = vr ? to_f32<T>(qrow[d]) * (ktok ? 1.f : ks[d]) : 0.f;
                     mx = fmaxf(mx, fabsf(qv[kk][e]));
                     cs = fmaf(qv[kk][e], o, cs);
                 }
@@ -507,15 +511,22 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
             }
 #pragma unroll
             for (int x = 1; x <= 2; x <<= 1) sq += __shfl_xor_sync(0xffffffffu, sq, x);
-            sc_b[nt] = ldexpf(a.c.scale_log2, -ex);
-            add_b[nt] = cs * a.c.scale_log2 - 1152.0f * sq * sc_b[nt];
+            if (ktok) {
+                sc_b[nt] = ldexpf(1.0f, -ex);
+                add_b[nt] = -1152.0f * sq * sc_b[nt];
+                qs_b[nt] = cs;
+            } else {
+                sc_b[nt] = ldexpf(a.c.scale_log2, -ex);
+                add_b[nt] = cs * a.c.scale_log2 - 1152.0f * sq * sc_b[nt];
+                qs_b[nt] = 0.f;
+            }
         }
     }
 
     // ---- accumulator columns: this thread holds query rows 8nt + 2c + e ----
     const bool causal = (a.c.mask_type == 9 || a.c.mask_type == 3);
     const bool alibi = a.c.mask_type == 3;
-    float sc[NT][2], add[NT][2], slope[NT][2];
+    float sc[NT][2], add[NT][2], qs[NT][2], slope[NT][2];
     int qpos[NT][2];
     bool vrow[NT][2];
     const T *pse_row[NT][2];
@@ -527,6 +538,7 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
             // the B-layout thread holding row n is lane 4 (2c + e) of the column tile
             sc[nt][e] = __shfl_sync(0xffffffffu, sc_b[nt], 4 * (2 * c + e));
             add[nt][e] = __shfl_sync(0xffffffffu, add_b[nt], 4 * (2 * c + e));
+            qs[nt][e] = ktok ? __shfl_sync(0xffffffffu, qs_b[nt], 4 * (2 * c + e)) : 0.f;
             vrow[nt][e] = n < R;
             const int qi = vrow[nt][e] ? n / g : 0;
             const int head = vrow[nt][e] ? u.kvh * g + n % g : 0;
@@ -542,8 +554,15 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
     float m[NT][2], l[NT][2];
     float o[NT][MT][4];
     float osum[NT][4];
+    float voff[NT][2];      // per-token V: sum_t p_t sV_t oV_t per row
+    // per-token scale / offset rows of this sequence
+    const float *ksr = ktok ? a.k_scale + (int64_t)u.b * a.k_tok_stride : nullptr;
+    const float *kor = (ktok && a.k_offset) ? a.k_offset + (int64_t)u.b * a.k_tok_stride : nullptr;
+    const float *vsr = vtok ? a.v_scale + (int64_t)u.b * a.v_tok_stride : nullptr;
+    const float *vor = (vtok && a.v_offset) ? a.v_offset + (int64_t)u.b * a.v_tok_stride : nullptr;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
+        voff[nt][0] = voff[nt][1] = 0.f;
         m[nt][0] = m[nt][1] = -INFINITY;
         l[nt][0] = l[nt][1] = 0.f;
         osum[nt][0] = osum[nt][1] = osum[nt][2] = osum[nt][3] = 0.f;
@@ -594,12 +613,27 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
                             (!causal || tw + 15 <= si.kvlen - si.qlen);
         float sv[NT][4];
         float mx[NT][2];
+        // per-token K of this thread's keys tw + r and tw + r + 8 (keys past
+        // the unit's end are masked below and never read)
+        float kf[2] = {1.f, 1.f}, kof[2] = {0.f, 0.f};
+        if constexpr (KTOK) {
+#pragma unroll
+            for (int hk = 0; hk < 2; ++hk) {
+                const int t = tw + r + 8 * hk;
+                if (t < u.t_end) {
+                    kf[hk] = ksr[t] * a.c.scale_log2;
+                    kof[hk] = kor ? kor[t] : 0.f;
+                }
+            }
+        }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int e = q & 1;
-                float x = fmaf(sacc[nt][q], sc[nt][e], add[nt][e]);
+                float x = ktok ? fmaf(sacc[nt][q], sc[nt][e], fmaf(kof[q >> 1], qs[nt][e], add[nt][e])) *
+                                     kf[q >> 1]
+                               : fmaf(sacc[nt][q], sc[nt][e], add[nt][e]);
                 if (!simple) {
                     const int t = tw + r + 8 * (q >> 1);
                     const bool in = t < u.t_end;
@@ -638,16 +672,32 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
                 }
             }
         }
+        // per-token V of this thread's keys: P is scaled by sV_t before it
+        // meets the value bytes, and sum_t p_t sV_t oV_t is kept per row
+        float vf[2] = {1.f, 1.f}, vof[2] = {0.f, 0.f};
+        if constexpr (VTOK) {
+#pragma unroll
+            for (int hk = 0; hk < 2; ++hk) {
+                const int t = tw + r + 8 * hk;
+                vf[hk] = (t < u.t_end) ? vsr[t] : 0.f;
+                vof[hk] = (vor && t < u.t_end) ? vor[t] : 0.f;
+            }
+        }
         __syncwarp();      // movmatrix and mma.sync below are .aligned
         uint32_t pb[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const float mu0 = (m[nt][0] == -INFINITY) ? 0.f : m[nt][0];
             const float mu1 = (m[nt][1] == -INFINITY) ? 0.f : m[nt][1];
-            const float p0 = ex2(sv[nt][0] - mu0), p1 = ex2(sv[nt][1] - mu1);
-            const float p2 = ex2(sv[nt][2] - mu0), p3 = ex2(sv[nt][3] - mu1);
+            float p0 = ex2(sv[nt][0] - mu0), p1 = ex2(sv[nt][1] - mu1);
+            float p2 = ex2(sv[nt][2] - mu0), p3 = ex2(sv[nt][3] - mu1);
             l[nt][0] = fmaf(l[nt][0], al[nt][0], p0 + p2);
             l[nt][1] = fmaf(l[nt][1], al[nt][1], p1 + p3);
+            if constexpr (VTOK) {
+                p0 *= vf[0]; p1 *= vf[0]; p2 *= vf[1]; p3 *= vf[1];
+                voff[nt][0] = fmaf(voff[nt][0], al[nt][0], fmaf(p0, vof[0], p2 * vof[1]));
+                voff[nt][1] = fmaf(voff[nt][1], al[nt][1], fmaf(p1, vof[0], p3 * vof[1]));
+            }
             // P^T fragments: (keys x rows) f16 tiles transposed to (rows x keys)
             pb[nt][0] = movmatrix_trans(pack2<__half>(p0, p1));     // keys 2c, 2c+1
             pb[nt][1] = movmatrix_trans(pack2<__half>(p2, p3));     // keys 2c+8, 2c+9
@@ -736,6 +786,10 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
         for (int nt = 0; nt < NT; ++nt) {
             l[nt][0] += __shfl_xor_sync(0xffffffffu, l[nt][0], x);
             l[nt][1] += __shfl_xor_sync(0xffffffffu, l[nt][1], x);
+            if constexpr (VTOK) {
+                voff[nt][0] += __shfl_xor_sync(0xffffffffu, voff[nt][0], x);
+                voff[nt][1] += __shfl_xor_sync(0xffffffffu, voff[nt][1], x);
+            }
         }
     __syncthreads();   // every warp is done with the stage buffers
     float *ow = reinterpret_cast<float *>(smem);                               // [4][16][D]
@@ -747,9 +801,11 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
         for (int e = 0; e < 2; ++e) {
             const int n = 8 * nt + 2 * c + e;
 #pragma unroll
+            // per-token V: + sum_t p_t sV_t oV_t (exactly 0 otherwise)
             for (int mt = 0; mt < MT; ++mt) {
-                oww[n * D + 8 * r + mt] = fmaf(-1152.0f, osum[nt][e], o[nt][mt][e]);
-                oww[n * D + 64 + 8 * r + mt] = fmaf(-1152.0f, osum[nt][e], o[nt][mt][2 + e]);
+                oww[n * D + 8 * r + mt] = fmaf(-1152.0f, osum[nt][e], o[nt][mt][e]) + voff[nt][e];
+                oww[n * D + 64 + 8 * r + mt] =
+                    fmaf(-1152.0f, osum[nt][e], o[nt][mt][2 + e]) + voff[nt][e];
             }
             if (r == 0) mlw[warp * kDecodeRows + n] = make_float2(m[nt][e], l[nt][e]);
         }
@@ -809,9 +865,13 @@ fia_combine_kernel(const __grid_constant__ CombineArgs a) {
         }
         const float Lt = L + (a.c.sink ? ex2(sink2 - M2) : 0.f);
         if constexpr (INT8) {
-            const float vs = a.v_scale[it.kvh * D + d];
-            const float vo = a.v_offset ? a.v_offset[it.kvh * D + d] : 0.f;
-            acc = vs * fmaf(vo, L, acc);
+            // per-channel V: out_d = sV_d (sum_t p_t v_td + oV_d sum_t p_t) / L;
+            // per-token V was applied token by token in the partials
+            if (!a.v_mode) {
+                const float vs = a.v_scale[it.kvh * D + d];
+                const float vo = a.v_offset ? a.v_offset[it.kvh * D + d] : 0.f;
+                acc = vs * fmaf(vo, L, acc);
+            }
         }
         val = acc / Lt;
         lse = (M2 + log2f(Lt)) * kLn2;
@@ -836,15 +896,26 @@ static cudaError_t launch_decode_t(const DecodeArgs &a, const CUtensorMap &tk,
     return cudaGetLastError();
 }
 
-template <typename T, int NT>
-static cudaError_t launch_decode_i8_t(const DecodeArgs &a, const CUtensorMap &tk,
+template <typename T, int NT, bool KTOK, bool VTOK>
+static cudaError_t launch_decode_i8_m(const DecodeArgs &a, const CUtensorMap &tk,
                                       const CUtensorMap &tv, int grid, cudaStream_t s) {
-    auto kern = fia_decode_i8_kernel<T, NT>;
+    auto kern = fia_decode_i8_kernel<T, NT, KTOK, VTOK>;
     const int smem = DecodeI8Cfg::kSmem;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, 128, smem, s>>>(a, tk, tv);
     return cudaGetLastError();
+}
+
+// dequantisation modes as compile-time flags: the per-channel kernel carries
+// no per-token code
+template <typename T, int NT>
+static cudaError_t launch_decode_i8_t(const DecodeArgs &a, const CUtensorMap &tk,
+                                      const CUtensorMap &tv, int grid, cudaStream_t s) {
+    if (a.k_mode) return a.v_mode ? launch_decode_i8_m<T, NT, true, true>(a, tk, tv, grid, s)
+                                  : launch_decode_i8_m<T, NT, true, false>(a, tk, tv, grid, s);
+    return a.v_mode ? launch_decode_i8_m<T, NT, false, true>(a, tk, tv, grid, s)
+                    : launch_decode_i8_m<T, NT, false, false>(a, tk, tv, grid, s);
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, const CUtensorMap &tk, const CUtensorMap &tv,

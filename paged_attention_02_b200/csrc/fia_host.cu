@@ -48,6 +48,8 @@ struct fia_op {
     uint64_t ws_size = 0;
     int32_t grid = 0, grid2 = 0;
     int32_t max_rows = 0;           // decode: max seqLen * g
+    int32_t k_mode = 0, v_mode = 0;     // int8 dequant modes (fia_antiquant_mode)
+    int64_t k_tok_stride = 0, v_tok_stride = 0;
     int64_t work_items = 0;
     int32_t split_tokens = 0;
     cudaEvent_t ev_start = nullptr, ev_stop = nullptr;
@@ -237,17 +239,40 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
     }
     const fia_tensor *ks = ext ? ext->kScale : nullptr, *ko = ext ? ext->kOffset : nullptr;
     const fia_tensor *vs = ext ? ext->vScale : nullptr, *vo = ext ? ext->vOffset : nullptr;
+    const int32_t k_mode = ext ? ext->kAntiquantMode : (int32_t)FIA_ANTIQUANT_PER_CHANNEL;
+    const int32_t v_mode = ext ? ext->vAntiquantMode : (int32_t)FIA_ANTIQUANT_PER_CHANNEL;
+    if ((k_mode != FIA_ANTIQUANT_PER_CHANNEL && k_mode != FIA_ANTIQUANT_PER_TOKEN) ||
+        (v_mode != FIA_ANTIQUANT_PER_CHANNEL && v_mode != FIA_ANTIQUANT_PER_TOKEN))
+        return FIA_ERR_PARAM;
+    int64_t k_tok_stride = 0, v_tok_stride = 0;
     if (kv_int8) {
-        for (const fia_tensor *t : {ks, vs}) {
-            fia_status s = check_f32_vec(t, kvHeadNum, D);
-            if (s != FIA_OK) return s;
-        }
-        for (const fia_tensor *t : {ko, vo}) {
-            if (!t) continue;
-            fia_status s = check_f32_vec(t, kvHeadNum, D);
-            if (s != FIA_OK) return s;
-        }
-    } else if (ks || vs || ko || vo) {
+        // per-channel: [kvHeadNum, headSize]; per-token: [batch, S] or
+        // [1, batch, S] with S >= max kvSeqLen.  Returns the row stride S.
+        auto check_quant = [&](const fia_tensor *t, int32_t mode, int64_t *stride) -> fia_status {
+            if (mode == FIA_ANTIQUANT_PER_CHANNEL) return check_f32_vec(t, kvHeadNum, D);
+            if (!t || !t->data) return FIA_ERR_NULLPTR;
+            if (t->dtype != FIA_F32) return FIA_ERR_DTYPE;
+            int64_t bd, sd;
+            if (t->ndim == 2) {
+                bd = t->dims[0];
+                sd = t->dims[1];
+            } else if (t->ndim == 3 && t->dims[0] == 1) {
+                bd = t->dims[1];
+                sd = t->dims[2];
+            } else {
+                return FIA_ERR_SHAPE;
+            }
+            if (bd != batch || sd < std::max<int64_t>(max_kv, 1)) return FIA_ERR_SHAPE;
+            if (*stride != 0 && *stride != sd) return FIA_ERR_SHAPE;   // scale vs offset
+            *stride = sd;
+            return FIA_OK;
+        };
+        fia_status st;
+        if ((st = check_quant(ks, k_mode, &k_tok_stride)) != FIA_OK) return st;
+        if (ko && (st = check_quant(ko, k_mode, &k_tok_stride)) != FIA_OK) return st;
+        if ((st = check_quant(vs, v_mode, &v_tok_stride)) != FIA_OK) return st;
+        if (vo && (st = check_quant(vo, v_mode, &v_tok_stride)) != FIA_OK) return st;
+    } else if (ks || vs || ko || vo || k_mode != 0 || v_mode != 0) {
         return FIA_ERR_PARAM;
     }
 
@@ -316,6 +341,10 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
     c.mask_type = maskType;
     c.scale_log2 = qkScale * 1.4426950408889634f;
     if (kv_int8) {
+        o->k_mode = k_mode;
+        o->v_mode = v_mode;
+        o->k_tok_stride = k_tok_stride;
+        o->v_tok_stride = v_tok_stride;
         o->k_scale = reinterpret_cast<const float *>(ks->data);
         o->k_offset = ko ? reinterpret_cast<const float *>(ko->data) : nullptr;
         o->v_scale = reinterpret_cast<const float *>(vs->data);
@@ -566,6 +595,12 @@ fia_status fia_run(void *workspace, uint64_t workspaceSize, fia_op *op, void *st
         d.part_ml = reinterpret_cast<float2 *>(ws + op->off_part_ml);
         d.k_scale = op->k_scale;
         d.k_offset = op->k_offset;
+        d.v_scale = op->v_scale;
+        d.v_offset = op->v_offset;
+        d.k_tok_stride = op->k_tok_stride;
+        d.v_tok_stride = op->v_tok_stride;
+        d.k_mode = op->k_mode;
+        d.v_mode = op->v_mode;
         d.n_units = op->grid;
         d.max_rows = op->max_rows;
         if (op->grid > 0) e = launch_decode(d, op->tk, op->tv, op->q_dtype, op->kv_int8, op->grid, s);
@@ -577,6 +612,7 @@ fia_status fia_run(void *workspace, uint64_t workspaceSize, fia_op *op, void *st
             cb.part_ml = d.part_ml;
             cb.v_scale = op->v_scale;
             cb.v_offset = op->v_offset;
+            cb.v_mode = op->v_mode;
             cb.n_items = op->grid2;
             e = launch_combine(cb, op->q_dtype, op->kv_int8, op->grid2, s);
         }
@@ -658,6 +694,12 @@ fia_status fia_decode_run_static(fia_op *op, void *stream_ptr) {
     d.part_ml = reinterpret_cast<float2 *>(ws + op->off_part_ml);
     d.k_scale = op->k_scale;
     d.k_offset = op->k_offset;
+    d.v_scale = op->v_scale;
+    d.v_offset = op->v_offset;
+    d.k_tok_stride = op->k_tok_stride;
+    d.v_tok_stride = op->v_tok_stride;
+    d.k_mode = op->k_mode;
+    d.v_mode = op->v_mode;
     d.n_units = op->grid;
     d.max_rows = op->max_rows;
     cudaError_t e = cudaSuccess;
@@ -670,6 +712,7 @@ fia_status fia_decode_run_static(fia_op *op, void *stream_ptr) {
         cb.part_ml = d.part_ml;
         cb.v_scale = op->v_scale;
         cb.v_offset = op->v_offset;
+        cb.v_mode = op->v_mode;
         cb.n_items = op->grid2;
         e = launch_combine(cb, op->q_dtype, op->kv_int8, op->grid2, s);
     }

@@ -81,6 +81,9 @@ struct DecodeArgs {
     float *part_o;          // [slots][16][D]
     float2 *part_ml;        // [slots][16] (m in log2 units, l)
     const float *k_scale, *k_offset;   // int8 only
+    const float *v_scale, *v_offset;   // int8 only (used here in per-token mode)
+    int64_t k_tok_stride, v_tok_stride;   // per-token mode: row stride S of [B, S]
+    int32_t k_mode, v_mode;  // int8 dequant: 0 per (KV head, channel), 1 per (b, token)
     int32_t n_units;
     int32_t max_rows;       // max over sequences of seqLen * g (<= kDecodeRows)
 };
@@ -91,6 +94,7 @@ struct CombineArgs {
     const float *part_o;
     const float2 *part_ml;
     const float *v_scale, *v_offset;   // int8 only
+    int32_t v_mode;         // int8: 1 = per-token V, already applied in the partials
     int32_t n_items;
 };
 

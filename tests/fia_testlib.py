@@ -18,7 +18,9 @@ def run_gpu(p, device="cuda", **overrides):
     kw = dict(mask_type=p.mask_type, slopes=d(p.slopes), pse=d(p.pse), sink=d(p.sink),
               k_scale=d(p.k_scale), k_offset=d(p.k_offset), v_scale=d(p.v_scale),
               v_offset=d(p.v_offset), want_lse=p.want_lse,
-              kv_layout=int(getattr(p, "kv_layout", 0)))
+              kv_layout=int(getattr(p, "kv_layout", 0)),
+              k_antiquant_mode=int(getattr(p, "k_antiquant_mode", 0)),
+              v_antiquant_mode=int(getattr(p, "v_antiquant_mode", 0)))
     kw.update(overrides)
     op = fia.FiaOp(d(p.query), d(p.key_cache), d(p.value_cache), d(p.block_tables),
                    [int(x) for x in p.seq_len], [int(x) for x in p.kv_seq_len], p.head_num,

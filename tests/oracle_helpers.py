@@ -75,11 +75,18 @@ def dense_sdpa(p: Problem) -> np.ndarray:
     out = np.zeros((p.n_tokens, H, D), dtype=np.float64)
     kc = p.key_cache.to(torch.float64)
     vc = p.value_cache.to(torch.float64)
+    if getattr(p, "kv_layout", 0) == 1:          # BnNBsD -> BnBsH view
+        kc, vc = kc.transpose(1, 2), vc.transpose(1, 2)
+    km, vm = int(getattr(p, "k_antiquant_mode", 0)), int(getattr(p, "v_antiquant_mode", 0))
     if p.kv_is_int8:
-        ko = torch.zeros(KVH, D, dtype=torch.float64) if p.k_offset is None else p.k_offset.double()
-        vo = torch.zeros(KVH, D, dtype=torch.float64) if p.v_offset is None else p.v_offset.double()
-        kc = (kc + ko) * p.k_scale.double()
-        vc = (vc + vo) * p.v_scale.double()
+        # per-channel pairs are applied to the whole pool here; per-token
+        # pairs ([B, S]) after each sequence's gather below
+        if not km:
+            ko = torch.zeros(KVH, D, dtype=torch.float64) if p.k_offset is None else p.k_offset.double()
+            kc = (kc + ko) * p.k_scale.double()
+        if not vm:
+            vo = torch.zeros(KVH, D, dtype=torch.float64) if p.v_offset is None else p.v_offset.double()
+            vc = (vc + vo) * p.v_scale.double()
     for b in range(p.batch):
         ql, kl = int(p.seq_len[b]), int(p.kv_seq_len[b])
         if ql == 0:
@@ -88,6 +95,12 @@ def dense_sdpa(p: Problem) -> np.ndarray:
         blk = p.block_tables[b].long()[t // bs]
         kd = kc[blk, t % bs]                              # [kl, KVH, D]
         vd = vc[blk, t % bs]
+        if p.kv_is_int8 and km:
+            off = p.k_offset[b, :kl].double() if p.k_offset is not None else torch.zeros(kl, dtype=torch.float64)
+            kd = (kd + off[:, None, None]) * p.k_scale[b, :kl].double()[:, None, None]
+        if p.kv_is_int8 and vm:
+            off = p.v_offset[b, :kl].double() if p.v_offset is not None else torch.zeros(kl, dtype=torch.float64)
+            vd = (vd + off[:, None, None]) * p.v_scale[b, :kl].double()[:, None, None]
         q = p.query[cu[b]:cu[b + 1]].to(torch.float64)    # [ql, H, D]
         kd = kd.repeat_interleave(g, dim=1)               # GQA: head h -> kv head h // g
         vd = vd.repeat_interleave(g, dim=1)

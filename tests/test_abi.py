@@ -61,7 +61,7 @@ def _call(**kw):
     d = {k: tensor_desc(v) for k, v in t.items()}
     P = lambda x: ctypes.pointer(x) if x is not None else None
     ext = fia_ext(P(d["pse"]), P(d["sink"]), P(d["ks"]), None, P(d["vs"]), None, P(d["lse"]),
-                  int(args.get("layout", 0)))
+                  int(args.get("layout", 0)), int(args.get("kmode", 0)), int(args.get("vmode", 0)))
     n = max(len(args["seq"]), 1)
     sl = (ctypes.c_int32 * n)(*args["seq"])
     kl = (ctypes.c_int32 * n)(*args["kv"])
@@ -154,3 +154,25 @@ def test_phase1_kv_layout_rules():
     assert _call(layout=1, k=bn(), v=bn()) in (L.FIA_ERR_CUDA, L.FIA_OK)
     # the table must cover kvSeqLen with the BnNBsD block size (dims[2] = 16)
     assert _call(layout=1, k=bn(), v=bn(), kv=[20, 80]) == L.FIA_ERR_SHAPE
+
+
+def test_phase1_per_token_antiquant_rules():
+    """Per-token int8 dequantisation (V3 fake-quantization: scale/offset
+    (B, S) or (1, B, S), f32; K and V modes may differ)."""
+    from paged_attention_02_b200 import _lib as L
+    k8 = torch.zeros(8, 16, 2, 128, dtype=torch.int8)
+    ch = torch.ones(2, 128)                       # per-channel [KVH, D]
+    tok = torch.ones(2, 40)                       # per-token [B=2, S=40 >= max kvSeqLen 33]
+    ok = (L.FIA_ERR_CUDA, L.FIA_OK)               # valid: no GPU here, phase 1 stops at encoding
+    assert _call(k=k8, v=k8, ks=tok, vs=tok, kmode=1, vmode=1) in ok
+    assert _call(k=k8, v=k8, ks=ch, vs=tok, kmode=0, vmode=1) in ok
+    assert _call(k=k8, v=k8, ks=tok, vs=ch, kmode=1, vmode=0) in ok
+    assert _call(k=k8, v=k8, ks=tok[None], vs=tok[None], kmode=1, vmode=1) in ok      # (1, B, S)
+    assert _call(k=k8, v=k8, ks=tok, vs=tok, kmode=2) == L.FIA_ERR_PARAM              # unknown mode
+    assert _call(k=k8, v=k8, ks=tok, vs=tok, kmode=0, vmode=1) == L.FIA_ERR_SHAPE     # K expects [KVH, D]
+    assert _call(k=k8, v=k8, ks=torch.ones(3, 40), vs=tok, kmode=1, vmode=1) == L.FIA_ERR_SHAPE  # B
+    assert _call(k=k8, v=k8, ks=torch.ones(2, 30), vs=tok, kmode=1, vmode=1) == L.FIA_ERR_SHAPE  # S < 33
+    assert _call(k=k8, v=k8, ks=torch.ones(2, 40, dtype=torch.float16), vs=tok, kmode=1,
+                 vmode=1) == L.FIA_ERR_DTYPE
+    # a mode on a bf16 cache is a parameter error
+    assert _call(kmode=1) == L.FIA_ERR_PARAM

@@ -278,3 +278,34 @@ def test_bnnbsd_layout(name):
     compare(out_q, lse_q, ref_out, ref_lse, name)
     _, out_p, lse_p = run_gpu(p)
     assert np.array_equal(out_q, out_p) and np.array_equal(lse_q, lse_p)
+
+
+# Per-token int8 dequantisation (V3 fake-quantization: scale/offset per
+# (sequence, cached token), [B, S] f32; K and V modes may differ, e.g.
+# per-channel keys with per-token values).
+PER_TOKEN_CASES = {
+    "tok_kv_bf16_sink": dict(seq_len=[1, 1, 1], kv_seq_len=[300, 1025, 7], head_num=16,
+                             kv_head_num=2, head_size=128, block_size=64, kv_dtype="i8",
+                             sink=True, k_antiquant="token", v_antiquant="token"),
+    "k_channel_v_token_f16": dict(seq_len=[1, 1], kv_seq_len=[513, 64], head_num=8, kv_head_num=1,
+                                  head_size=128, block_size=16, dtype="f16", kv_dtype="i8",
+                                  k_antiquant="channel", v_antiquant="token"),
+    "k_token_v_channel_sym": dict(seq_len=[1, 1], kv_seq_len=[200, 4100], head_num=16,
+                                  kv_head_num=4, head_size=128, block_size=128, kv_dtype="i8",
+                                  int8_offsets=False, k_antiquant="token", v_antiquant="channel"),
+    "tok_mtp_causal_nt2": dict(seq_len=[2, 1, 2], kv_seq_len=[90, 33, 700], head_num=16,
+                               kv_head_num=2, head_size=128, block_size=32, kv_dtype="i8",
+                               mask_type=W.MASK_CAUSAL, k_antiquant="token", v_antiquant="token"),
+    "tok_bnnbsd": dict(seq_len=[1, 1], kv_seq_len=[777, 129], head_num=16, kv_head_num=2,
+                       head_size=128, block_size=64, kv_dtype="i8", sink=True,
+                       k_antiquant="token", v_antiquant="token", kv_layout=1),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PER_TOKEN_CASES))
+def test_int8_per_token_antiquant(name):
+    p = W.make_problem(name=name, seed=zlib.crc32(name.encode()) % 10000, spare_blocks=2,
+                       **PER_TOKEN_CASES[name])
+    _, out, lse = run_gpu(p)
+    ref_out, ref_lse = oracle.attention(p)
+    compare(out, lse, ref_out, ref_lse, name)

@@ -292,3 +292,55 @@ def test_oracle_bnnbsd_layout_matches_bnbsh(kind):
     swapped = dataclasses.replace(q, key_cache=q.key_cache.flip(1).contiguous())
     o3, _ = oracle.attention(swapped)
     assert not np.allclose(o1, o3)
+
+
+def _int8_problem(k_antiquant="token", v_antiquant="token", **kw):
+    cfg = dict(seq_len=[1, 2, 1], kv_seq_len=[70, 33, 5], head_num=8, kv_head_num=2,
+               head_size=128, block_size=16, kv_dtype="i8", sink=True)
+    cfg.update(kw)
+    return W.make_problem(seed=zlib.crc32((k_antiquant + v_antiquant).encode()) % 1000,
+                          k_antiquant=k_antiquant, v_antiquant=v_antiquant, **cfg)
+
+
+@pytest.mark.parametrize("km,vm", [(1, 1), (1, 0), (0, 1)])
+def test_oracle_per_token_reduces_to_per_channel_for_constant_scales(km, vm):
+    """V3 fake-quantization modes: per-token (scale/offset per (b, t), [B, S])
+    and per-channel ([KVH, D]) are the same dequantisation when every scale
+    (offset) is one constant: the results agree bitwise, in any mix of K/V
+    modes."""
+    p = _int8_problem()
+    S = p.k_scale.shape[1]
+    def with_modes(pp, mk, mv):
+        ks = (p.batch, S) if mk else (p.kv_head_num, p.head_size)
+        vs = (p.batch, S) if mv else (p.kv_head_num, p.head_size)
+        return dataclasses.replace(pp, k_scale=torch.full(ks, 0.0125), k_offset=torch.full(ks, 0.25),
+                                   v_scale=torch.full(vs, 0.015625), v_offset=torch.full(vs, -0.5),
+                                   k_antiquant_mode=mk, v_antiquant_mode=mv)
+    o0, l0 = oracle.attention(with_modes(p, 0, 0))
+    o1, l1 = oracle.attention(with_modes(p, km, vm))
+    assert np.array_equal(o0, o1) and np.array_equal(l0, l1)
+
+
+def test_oracle_per_token_uses_each_tokens_own_scale():
+    """Per-token scales are indexed by (sequence, cached position): against
+    torch SDPA on the pool dequantised token by token; doubling every V scale
+    doubles the output exactly and leaves lse alone; scales of positions past
+    kvSeqLen are never read."""
+    p = _int8_problem(sink=False)
+    out, lse = oracle.attention(p)
+    ref_out = dense_sdpa(p)
+    assert np.abs(out - ref_out).max() < 1e-9
+    p2 = dataclasses.replace(p, v_scale=p.v_scale * 2, v_offset=p.v_offset)
+    out2, lse2 = oracle.attention(p2)
+    assert np.array_equal(out2, 2 * out) and np.array_equal(lse2, lse)
+    ks = p.k_scale.clone()
+    for b in range(p.batch):
+        ks[b, int(p.kv_seq_len[b]):] = float("nan")      # never read
+    out3, lse3 = oracle.attention(dataclasses.replace(p, k_scale=ks))
+    assert np.array_equal(out3, out) and np.array_equal(lse3, lse)
+    ks2 = p.k_scale.clone()
+    ks2[1, 3] *= 3.0                                      # a read position of sequence 1
+    out4, _ = oracle.attention(dataclasses.replace(p, k_scale=ks2))
+    rows_seq1 = slice(int(p.seq_len[0]), int(p.seq_len[0] + p.seq_len[1]))
+    assert not np.allclose(out4[rows_seq1], out[rows_seq1])
+    assert np.array_equal(out4[:int(p.seq_len[0])], out[:int(p.seq_len[0])])

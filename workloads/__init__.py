@@ -59,6 +59,8 @@ class Problem:
     v_offset: Optional[torch.Tensor] = None   # [KVH, D] f32
     want_lse: bool = True
     kv_layout: int = 0                        # 0 BnBsH, 1 BnNBsD
+    k_antiquant_mode: int = 0                 # int8: 0 per-channel [KVH, D], 1 per-token [B, S]
+    v_antiquant_mode: int = 0
 
     @property
     def batch(self) -> int:
@@ -117,6 +119,8 @@ def make_problem(
     want_lse: bool = True,
     max_blocks: Optional[int] = None,
     kv_layout: int = 0,
+    k_antiquant: str = "channel",
+    v_antiquant: str = "channel",
 ) -> Problem:
     """Draw a seeded problem.
 
@@ -128,6 +132,10 @@ def make_problem(
       sequence's last block (e.g. NaN) to prove they are never read.
     * ALiBi slopes are ``2**(-8(h+1)/H)`` (caller-supplied, as the
       PrefixEncoder ``slopes`` parameter is).
+    * int8 scales ``U(0.005, 0.02)`` and offsets ``N(0, 0.1)``, per
+      ``k_antiquant`` / ``v_antiquant``: ``"channel"`` ``[KVH, D]`` or
+      ``"token"`` ``[B, S]`` with ``S = max kvSeqLen + 3`` (a row stride
+      longer than any sequence).
     * ``kv_layout=1``: the same cache stored BnNBsD ``[numBlocks, KVH, bs, D]``
       (drawn as above, then transposed).
     * ``pse``: the ALiBi bias written out as a full ``[B, H, maxQ, maxKV]``
@@ -195,12 +203,17 @@ def make_problem(
         sink_t = torch.from_numpy(rng.standard_normal(H, dtype=np.float32))
 
     ks = ko = vs = vo = None
+    modes = {"channel": 0, "token": 1}
+    km, vm = modes[k_antiquant], modes[v_antiquant]
     if kv_dtype == "i8":
-        ks = torch.from_numpy(rng.uniform(0.005, 0.02, (KVH, D)).astype(np.float32))
-        vs = torch.from_numpy(rng.uniform(0.005, 0.02, (KVH, D)).astype(np.float32))
+        S = int(kv_seq_len.max()) + 3 if B else 3
+        kshape = (B, S) if km else (KVH, D)
+        vshape = (B, S) if vm else (KVH, D)
+        ks = torch.from_numpy(rng.uniform(0.005, 0.02, kshape).astype(np.float32))
+        vs = torch.from_numpy(rng.uniform(0.005, 0.02, vshape).astype(np.float32))
         if int8_offsets:
-            ko = torch.from_numpy((0.1 * rng.standard_normal((KVH, D))).astype(np.float32))
-            vo = torch.from_numpy((0.1 * rng.standard_normal((KVH, D))).astype(np.float32))
+            ko = torch.from_numpy((0.1 * rng.standard_normal(kshape)).astype(np.float32))
+            vo = torch.from_numpy((0.1 * rng.standard_normal(vshape)).astype(np.float32))
 
     p = Problem(
         name=name, query=query, key_cache=kc, value_cache=vc,
@@ -208,6 +221,8 @@ def make_problem(
         head_num=H, kv_head_num=KVH, qk_scale=float(qk_scale), mask_type=mask_type,
         slopes=slopes_t if mask_type == MASK_ALIBI else None, pse=pse_t, sink=sink_t,
         k_scale=ks, k_offset=ko, v_scale=vs, v_offset=vo, want_lse=want_lse,
+        k_antiquant_mode=km if kv_dtype == "i8" else 0,
+        v_antiquant_mode=vm if kv_dtype == "i8" else 0,
     )
     return to_bnnbsd(p) if kv_layout == 1 else p
 
