@@ -176,7 +176,7 @@ def make_op(p, t):
                      pse=t["pse"], sink=t["sink"], k_scale=t["k_scale"], k_offset=t["k_offset"],
                      v_scale=t["v_scale"], v_offset=t["v_offset"], want_lse=p.want_lse,
                      kv_layout=p.kv_layout, k_antiquant_mode=p.k_antiquant_mode,
-                     v_antiquant_mode=p.v_antiquant_mode)
+                     v_antiquant_mode=p.v_antiquant_mode, band=p.band)
 
 
 def time_op(op, steps, warmup, flush):

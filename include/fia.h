@@ -96,6 +96,9 @@ typedef enum { FIA_KV_BNBSH = 0, FIA_KV_BNNBSD = 1 } fia_kv_layout;
    per-token mode with scale/offset of shape (B, S) or (1, B, S), f32). */
 typedef enum { FIA_ANTIQUANT_PER_CHANNEL = 0, FIA_ANTIQUANT_PER_TOKEN = 1 } fia_antiquant_mode;
 
+/* sparse modes (V3 sparseMode): 0 = mask from maskType, 4 = band */
+typedef enum { FIA_SPARSE_NONE = 0, FIA_SPARSE_BAND = 4 } fia_sparse_mode;
+
 typedef struct {
     /* pse-shift bias [batch, headNum, maxQ, maxKV], the query's dtype, added to
        the scaled scores: s += pse[b][h][i][t] for new token i and key position t
@@ -133,6 +136,17 @@ typedef struct {
        default, is per-channel). */
     int32_t kAntiquantMode;
     int32_t vAntiquantMode;
+    /* Band mask (V3 sparseMode 4 with preTokens / nextTokens): with
+       sparseMode = FIA_SPARSE_BAND, new token i (absolute position qpos =
+       kvSeqLen - seqLen + i) sees the cached keys t with
+       qpos - preTokens <= t <= qpos + nextTokens (and t < kvSeqLen);
+       maskType must then be FIA_MASK_NONE, and preTokens + nextTokens >= 0.
+       A row whose band holds no key gets out 0 and lse +inf.  The default
+       (0) leaves masking to maskType.  Sliding-window attention is the band
+       with nextTokens = 0. */
+    int32_t sparseMode;
+    int64_t preTokens;
+    int64_t nextTokens;
 } fia_ext;
 
 typedef struct fia_op fia_op;

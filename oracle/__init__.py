@@ -60,9 +60,11 @@ def _load():
             lib = ctypes.CDLL(_LIB_PATH)
             common = [_P, _I, _P, _P, _I, _I64, _I, _P, _I, _P, _P, _I, _I, _I, _I, _D, _I, _P,
                       _P, _I, _I, _I, _P, _P, _P, _P, _P]
-            lib.fia_oracle_attention.argtypes = common + [_P, _I64, _I, _P, _P, _I, _I, _I, _I64, _I64]
+            lib.fia_oracle_attention.argtypes = common + [_P, _I64, _I, _P, _P, _I, _I, _I, _I64, _I64,
+                                                          _I, _I64, _I64]
             lib.fia_oracle_attention.restype = _I
-            lib.fia_oracle_row_probs.argtypes = common + [_I, _I, _I, _P, _P, _P, _I, _I, _I, _I64, _I64]
+            lib.fia_oracle_row_probs.argtypes = common + [_I, _I, _I, _P, _P, _P, _I, _I, _I, _I64, _I64,
+                                                          _I, _I64, _I64]
             lib.fia_oracle_row_probs.restype = _I
             lib.fia_oracle_max_threads.restype = _I
             _lib = lib
@@ -92,6 +94,14 @@ def _quant_modes(p):
     ks = p.k_scale.shape[-1] if (km == 1 and p.k_scale is not None) else 0
     vs = p.v_scale.shape[-1] if (vm == 1 and p.v_scale is not None) else 0
     return [km, vm, int(ks), int(vs)]
+
+
+def _band(p):
+    """(band, preTokens, nextTokens) of problem p (band mask, V3 sparseMode 4)."""
+    if getattr(p, "band", None) is None:
+        return [0, 0, 0]
+    pre, nxt = p.band
+    return [1, int(pre), int(nxt)]
 
 
 def _common(p, keep):
@@ -144,7 +154,7 @@ def attention(p, rows: Optional[Sequence[Tuple[int, int]]] = None,
                                   rows_arr.ctypes.data_as(_P) if rows_arr is not None else None,
                                   n_rows, int(threads),
                                   out.ctypes.data_as(_P), lse.ctypes.data_as(_P), _layout(p),
-                                  *_quant_modes(p))
+                                  *_quant_modes(p), *_band(p))
     if rc != 0:
         raise ValueError("oracle rejected the problem (code %d)" % rc)
     return out, lse
@@ -162,7 +172,7 @@ def row_probs(p, b: int, i: int, h: int) -> Tuple[np.ndarray, np.ndarray, float]
     lse = np.zeros((1,), dtype=np.float64)
     rc = lib.fia_oracle_row_probs(*args, b, i, h, probs.ctypes.data_as(_P),
                                   out.ctypes.data_as(_P), lse.ctypes.data_as(_P), _layout(p),
-                                  *_quant_modes(p))
+                                  *_quant_modes(p), *_band(p))
     if rc != 0:
         raise ValueError("oracle rejected the row (code %d)" % rc)
     return probs[:kvlen], out, float(lse[0])

@@ -29,6 +29,7 @@
  *        (per-token mode, scale/offset [B, S], V3 fake-quantization
  *        bullets; K and V modes may differ); no offset given -> offset 0.
  *   3. causal (maskType 9, and 3 = ALiBi which includes causal): skip t > qpos
+ *      band (V3 sparseMode 4): skip t < qpos - preTokens and t > qpos + nextTokens
  *   4. s_t = qkScale * sum_d q_d k_td
  *        + slope_h * (t - qpos)          (maskType 3)
  *        + pse[b][h][i][t]               (when a pse tensor is given)
@@ -99,6 +100,7 @@ typedef struct {
     int kv_layout;                              /* 0 BnBsH, 1 BnNBsD           */
     int k_mode, v_mode;                         /* 0 per-channel, 1 per-token  */
     int64_t k_tok_stride, v_tok_stride;         /* per-token: row stride S     */
+    int band; int64_t pre_tokens, next_tokens;  /* band mask (sparseMode 4)    */
 } oracle_args;
 
 /* int8 dequantisation of cache value x of (sequence b, position t, channel
@@ -140,6 +142,7 @@ static int64_t oracle_row(const oracle_args *a, int b, int i, int h, int64_t tok
     for (int64_t t = 0; t < kvlen; ++t) {
         keep[t] = 0;
         if (causal && t > qpos) continue;
+        if (a->band && (t < qpos - a->pre_tokens || t > qpos + a->next_tokens)) continue;
         int32_t blk = a->block_tables[(int64_t)b * a->max_blocks + t / a->bs];
         if (blk < 0 || blk >= a->num_blocks) { free(qv); free(s); free(keep); return -1; }
         int64_t row = cache_row(a, blk, t % a->bs, kvh);
@@ -210,17 +213,23 @@ int fia_oracle_attention(
     const void *pse, int pse_dtype, int pse_maxq, int pse_maxkv, const float *sink,
     const float *k_scale, const float *k_offset, const float *v_scale, const float *v_offset,
     const int64_t *rows, int64_t n_rows, int n_threads, double *out, double *lse, int kv_layout,
-    int k_mode, int v_mode, int64_t k_tok_stride, int64_t v_tok_stride) {
+    int k_mode, int v_mode, int64_t k_tok_stride, int64_t v_tok_stride,
+    int band, int64_t pre_tokens, int64_t next_tokens) {
     if (H <= 0 || KVH <= 0 || H % KVH != 0 || D <= 0 || bs <= 0) return -2;
     if (kv_layout != 0 && kv_layout != 1) return -2;
     if (k_mode < 0 || k_mode > 1 || v_mode < 0 || v_mode > 1) return -2;
     if (kv_dtype == OR_I8 && (!k_scale || !v_scale)) return -2;
     if (mask_type == 3 && !slopes) return -2;
-    oracle_args a = {q, q_dtype, k, v, kv_dtype, num_blocks, bs, block_tables, max_blocks,
-                     seq_len, kv_seq_len, batch, H, KVH, D, qk_scale, mask_type, slopes,
-                     pse, pse_dtype, pse_maxq, pse_maxkv, sink,
-                     k_scale, k_offset, v_scale, v_offset, kv_layout,
-                     k_mode, v_mode, k_tok_stride, v_tok_stride};
+    oracle_args a = {.q = q, .q_dtype = q_dtype, .k = k, .v = v, .kv_dtype = kv_dtype,
+                     .num_blocks = num_blocks, .bs = bs, .block_tables = block_tables,
+                     .max_blocks = max_blocks, .seq_len = seq_len, .kv_seq_len = kv_seq_len,
+                     .batch = batch, .H = H, .KVH = KVH, .D = D, .qk_scale = qk_scale,
+                     .mask_type = mask_type, .slopes = slopes, .pse = pse, .pse_dtype = pse_dtype,
+                     .pse_maxq = pse_maxq, .pse_maxkv = pse_maxkv, .sink = sink,
+                     .k_scale = k_scale, .k_offset = k_offset, .v_scale = v_scale,
+                     .v_offset = v_offset, .kv_layout = kv_layout, .k_mode = k_mode,
+                     .v_mode = v_mode, .k_tok_stride = k_tok_stride, .v_tok_stride = v_tok_stride,
+                     .band = band, .pre_tokens = pre_tokens, .next_tokens = next_tokens};
     /* token -> (b, i) */
     int64_t n_tokens = 0;
     for (int b = 0; b < batch; ++b) n_tokens += seq_len[b];
@@ -259,15 +268,21 @@ int fia_oracle_row_probs(
     const void *pse, int pse_dtype, int pse_maxq, int pse_maxkv, const float *sink,
     const float *k_scale, const float *k_offset, const float *v_scale, const float *v_offset,
     int b, int i, int h, double *probs, double *out, double *lse, int kv_layout,
-    int k_mode, int v_mode, int64_t k_tok_stride, int64_t v_tok_stride) {
+    int k_mode, int v_mode, int64_t k_tok_stride, int64_t v_tok_stride,
+    int band, int64_t pre_tokens, int64_t next_tokens) {
     if (H <= 0 || KVH <= 0 || H % KVH != 0 || b < 0 || b >= batch) return -2;
     if (kv_layout != 0 && kv_layout != 1) return -2;
     if (k_mode < 0 || k_mode > 1 || v_mode < 0 || v_mode > 1) return -2;
-    oracle_args a = {q, q_dtype, k, v, kv_dtype, num_blocks, bs, block_tables, max_blocks,
-                     seq_len, kv_seq_len, batch, H, KVH, D, qk_scale, mask_type, slopes,
-                     pse, pse_dtype, pse_maxq, pse_maxkv, sink,
-                     k_scale, k_offset, v_scale, v_offset, kv_layout,
-                     k_mode, v_mode, k_tok_stride, v_tok_stride};
+    oracle_args a = {.q = q, .q_dtype = q_dtype, .k = k, .v = v, .kv_dtype = kv_dtype,
+                     .num_blocks = num_blocks, .bs = bs, .block_tables = block_tables,
+                     .max_blocks = max_blocks, .seq_len = seq_len, .kv_seq_len = kv_seq_len,
+                     .batch = batch, .H = H, .KVH = KVH, .D = D, .qk_scale = qk_scale,
+                     .mask_type = mask_type, .slopes = slopes, .pse = pse, .pse_dtype = pse_dtype,
+                     .pse_maxq = pse_maxq, .pse_maxkv = pse_maxkv, .sink = sink,
+                     .k_scale = k_scale, .k_offset = k_offset, .v_scale = v_scale,
+                     .v_offset = v_offset, .kv_layout = kv_layout, .k_mode = k_mode,
+                     .v_mode = v_mode, .k_tok_stride = k_tok_stride, .v_tok_stride = v_tok_stride,
+                     .band = band, .pre_tokens = pre_tokens, .next_tokens = next_tokens};
     int64_t token = 0;
     for (int bb = 0; bb < b; ++bb) token += seq_len[bb];
     token += i;

@@ -12,7 +12,7 @@ attention, and a missing libfia.so raises at import.
 from __future__ import annotations
 
 import ctypes
-from typing import Optional, Sequence
+from typing import Optional, Sequence, Tuple
 
 import torch
 
@@ -52,6 +52,8 @@ class FiaOp:
     """One planned call (phase 1 done); ``run()`` enqueues phase 2.
 
     Arguments follow ``fia_get_workspace_size``: query ``[nTokens, H, D]``,
+    ``band=(preTokens, nextTokens)``: band mask (sliding window with
+    nextTokens = 0) instead of mask_type, which must then be FIA_MASK_NONE.
     int8 caches take k_scale/k_offset/v_scale/v_offset per (KV head, channel)
     ``[kvHeadNum, D]``, or per (sequence, token) ``[batch, S]`` with
     ``k_antiquant_mode`` / ``v_antiquant_mode`` = 1.
@@ -68,7 +70,8 @@ class FiaOp:
                  mask_type: int = FIA_MASK_NONE, slopes=None, pse=None, sink=None, k_scale=None,
                  k_offset=None, v_scale=None, v_offset=None, out=None, lse=None,
                  want_lse: bool = True, kv_layout: int = FIA_KV_BNBSH,
-                 k_antiquant_mode: int = 0, v_antiquant_mode: int = 0):
+                 k_antiquant_mode: int = 0, v_antiquant_mode: int = 0,
+                 band: Optional[Tuple[int, int]] = None):
         dev = query.device
         self.out = out if out is not None else torch.empty_like(query)
         if lse is None and want_lse:
@@ -83,7 +86,8 @@ class FiaOp:
         self._ext = fia_ext(_ptr(self._d["pse"]), _ptr(self._d["sink"]), _ptr(self._d["ks"]),
                             _ptr(self._d["ko"]), _ptr(self._d["vs"]), _ptr(self._d["vo"]),
                             _ptr(self._d["lse"]), int(kv_layout), int(k_antiquant_mode),
-                            int(v_antiquant_mode))
+                            int(v_antiquant_mode), _lib.FIA_SPARSE_BAND if band else 0,
+                            int(band[0]) if band else 0, int(band[1]) if band else 0)
         b = len(seq_len)
         self._sl = (ctypes.c_int32 * max(b, 1))(*[int(x) for x in seq_len])
         self._kl = (ctypes.c_int32 * max(b, 1))(*[int(x) for x in kv_seq_len])
@@ -170,12 +174,12 @@ def fused_infer_attention(query, key, value, block_tables, seq_len, kv_seq_len, 
                           kv_head_num, qk_scale, mask_type=FIA_MASK_NONE, slopes=None, pse=None,
                           sink=None, k_scale=None, k_offset=None, v_scale=None, v_offset=None,
                           want_lse=True, kv_layout=FIA_KV_BNBSH, k_antiquant_mode=0,
-                          v_antiquant_mode=0):
+                          v_antiquant_mode=0, band=None):
     """One-shot call: plan, run on the current stream, return (out, lse)."""
     op = FiaOp(query, key, value, block_tables, seq_len, kv_seq_len, head_num, kv_head_num,
                qk_scale, mask_type, slopes, pse, sink, k_scale, k_offset, v_scale, v_offset,
                want_lse=want_lse, kv_layout=kv_layout, k_antiquant_mode=k_antiquant_mode,
-               v_antiquant_mode=v_antiquant_mode)
+               v_antiquant_mode=v_antiquant_mode, band=band)
     out, lse = op.run()
     op._keep.append(op.workspace)
     return out, lse

@@ -25,6 +25,7 @@ FIA_F16, FIA_BF16, FIA_F32, FIA_I8, FIA_I32 = 0, 1, 2, 3, 4
 FIA_MASK_NONE, FIA_MASK_ALIBI, FIA_MASK_CAUSAL = 0, 3, 9
 FIA_KV_BNBSH, FIA_KV_BNNBSD = 0, 1
 FIA_ANTIQUANT_PER_CHANNEL, FIA_ANTIQUANT_PER_TOKEN = 0, 1
+FIA_SPARSE_NONE, FIA_SPARSE_BAND = 0, 4
 
 
 class fia_tensor(ctypes.Structure):
@@ -37,7 +38,9 @@ class fia_ext(ctypes.Structure):
                 ("kScale", ctypes.POINTER(fia_tensor)), ("kOffset", ctypes.POINTER(fia_tensor)),
                 ("vScale", ctypes.POINTER(fia_tensor)), ("vOffset", ctypes.POINTER(fia_tensor)),
                 ("lse", ctypes.POINTER(fia_tensor)), ("kvLayout", ctypes.c_int32),
-                ("kAntiquantMode", ctypes.c_int32), ("vAntiquantMode", ctypes.c_int32)]
+                ("kAntiquantMode", ctypes.c_int32), ("vAntiquantMode", ctypes.c_int32),
+                ("sparseMode", ctypes.c_int32), ("preTokens", ctypes.c_int64),
+                ("nextTokens", ctypes.c_int64)]
 
 
 class fia_plan_info(ctypes.Structure):

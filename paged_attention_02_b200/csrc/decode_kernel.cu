@@ -198,7 +198,9 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
         // Interior tile without bias: every key of the 16 is visible to every
         // row (rows past R only carry zeros and are never written out).
         const bool simple = !alibi && !a.c.pse && (tw + 16 <= u.t_end) &&
-                            (!causal || tw + 15 <= si.kvlen - si.qlen);
+                            (!causal || tw + 15 <= si.kvlen - si.qlen) &&
+                            (!a.c.band || (tw >= si.kvlen - 1 - a.c.pre &&
+                                           tw + 15 <= si.kvlen - si.qlen + a.c.next));
         if (simple) {
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
@@ -224,8 +226,10 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
                     }
                     if (pse_a && in) x = fmaf(to_f32<T>(pse_a[t]), kLog2e, x);
                     if (pse_b && in) y = fmaf(to_f32<T>(pse_b[t]), kLog2e, y);
-                    const bool ka = in && va && !(causal && t > qpos_a);
-                    const bool kb = in && vb && !(causal && t > qpos_b);
+                    const bool ka = in && va && !(causal && t > qpos_a) &&
+                                    !(a.c.band && (t < qpos_a - a.c.pre || t > qpos_a + a.c.next));
+                    const bool kb = in && vb && !(causal && t > qpos_b) &&
+                                    !(a.c.band && (t < qpos_b - a.c.pre || t > qpos_b + a.c.next));
                     sv[nt][e] = ka ? x : -INFINITY;
                     sv[nt][2 + e] = kb ? y : -INFINITY;
                     mx_a = fmaxf(mx_a, sv[nt][e]);
@@ -610,7 +614,9 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
         // accumulator element q of column tile nt: key tw + r + 8 (q >> 1),
         // row 8nt + 2c + (q & 1)
         const bool simple = !alibi && !a.c.pse && (tw + 16 <= u.t_end) &&
-                            (!causal || tw + 15 <= si.kvlen - si.qlen);
+                            (!causal || tw + 15 <= si.kvlen - si.qlen) &&
+                            (!a.c.band || (tw >= si.kvlen - 1 - a.c.pre &&
+                                           tw + 15 <= si.kvlen - si.qlen + a.c.next));
         float sv[NT][4];
         float mx[NT][2];
         // per-token K of this thread's keys tw + r and tw + r + 8 (keys past
@@ -639,7 +645,9 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
                     const bool in = t < u.t_end;
                     if (alibi) x = fmaf(slope[nt][e], (float)(t - qpos[nt][e]), x);
                     if (pse_row[nt][e] && in) x = fmaf(to_f32<T>(pse_row[nt][e][t]), kLog2e, x);
-                    const bool keep = in && vrow[nt][e] && !(causal && t > qpos[nt][e]);
+                    const bool keep = in && vrow[nt][e] && !(causal && t > qpos[nt][e]) &&
+                                      !(a.c.band && (t < qpos[nt][e] - a.c.pre ||
+                                                     t > qpos[nt][e] + a.c.next));
                     x = keep ? x : -INFINITY;
                 }
                 sv[nt][q] = x;

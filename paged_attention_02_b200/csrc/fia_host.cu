@@ -148,6 +148,17 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
     if (!std::isfinite(qkScale)) return FIA_ERR_PARAM;
     if (maskType != FIA_MASK_NONE && maskType != FIA_MASK_ALIBI && maskType != FIA_MASK_CAUSAL)
         return FIA_ERR_PARAM;
+    // band mask (sparseMode 4): replaces maskType; the band must not be empty
+    const int32_t sparse = ext ? ext->sparseMode : (int32_t)FIA_SPARSE_NONE;
+    if (sparse != FIA_SPARSE_NONE && sparse != FIA_SPARSE_BAND) return FIA_ERR_PARAM;
+    const bool band = (sparse == FIA_SPARSE_BAND);
+    // limits past +-2^40 cut nothing (lengths < 2^31); clamping first keeps
+    // the sum below from overflowing
+    const int64_t kLim = int64_t(1) << 40;
+    int64_t pre_tok = band ? std::max(-kLim, std::min(ext->preTokens, kLim)) : 0;
+    int64_t next_tok = band ? std::max(-kLim, std::min(ext->nextTokens, kLim)) : 0;
+    if (band && (maskType != FIA_MASK_NONE || pre_tok + next_tok < 0)) return FIA_ERR_PARAM;
+
 
     // ---- dtypes ----
     if (query->dtype != FIA_F16 && query->dtype != FIA_BF16) return FIA_ERR_DTYPE;
@@ -281,6 +292,7 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
     if (D != 64 && D != 128) return FIA_ERR_UNSUPPORTED;
     if (bs < 16 || bs > 256 || bs % 16 != 0) return FIA_ERR_UNSUPPORTED;
     if (nb * bs >= (int64_t(1) << 31) || n_tokens >= (int64_t(1) << 31)) return FIA_ERR_UNSUPPORTED;
+    if (band && max_kv >= (int64_t(1) << 30)) return FIA_ERR_UNSUPPORTED;
     const bool decode = (max_q * g <= kDecodeRows);
     if (kv_int8 && (!decode || D != 128)) return FIA_ERR_UNSUPPORTED;
 
@@ -338,6 +350,11 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
     c.D = (int32_t)D;
     c.bs = (int32_t)bs;
     c.kv_layout = kv_layout;
+    c.band = band ? 1 : 0;
+    // beyond +-(max kvSeqLen + 1) a band limit cuts nothing; clamped there the
+    // kernels' int32 position arithmetic cannot overflow (kvSeqLen < 2^30)
+    c.pre = (int32_t)std::max<int64_t>(-(max_kv + 1), std::min<int64_t>(pre_tok, max_kv + 1));
+    c.next = (int32_t)std::max<int64_t>(-(max_kv + 1), std::min<int64_t>(next_tok, max_kv + 1));
     c.mask_type = maskType;
     c.scale_log2 = qkScale * 1.4426950408889634f;
     if (kv_int8) {
@@ -414,8 +431,26 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
         o->max_rows = (int32_t)(max_q * g);
         const bool causal = (maskType != FIA_MASK_NONE);
         (void)causal;
+        // keys a sequence's rows can see: all of [0, kvSeqLen), or under a band
+        // [minQpos - pre, maxQpos + next] with the start rounded down to a
+        // 64-key tile (TMA boxes stay block-aligned)
+        auto key_range = [&](int b, int64_t *lo, int64_t *hi) {
+            const int64_t kl = kvSeqLen[b], ql = seqLen[b];
+            *lo = 0;
+            *hi = kl;
+            if (band) {
+                *lo = std::max<int64_t>(0, kl - ql - pre_tok);
+                *hi = std::min<int64_t>(kl, kl + next_tok);
+                if (*hi <= *lo) *hi = *lo = 0;
+                *lo = (*lo / kDecodeTile) * kDecodeTile;
+            }
+        };
         int64_t total = 0;
-        for (int b = 0; b < batch; ++b) total += (int64_t)kvSeqLen[b] * kvHeadNum;
+        for (int b = 0; b < batch; ++b) {
+            int64_t lo, hi;
+            key_range(b, &lo, &hi);
+            total += (hi - lo) * kvHeadNum;
+        }
         const int64_t target_units = (int64_t)nsm * 2 * 4;
         int64_t split = (total + target_units - 1) / std::max<int64_t>(target_units, 1);
         split = std::max<int64_t>(2 * kDecodeTile, align_up(std::max<int64_t>(split, 1), kDecodeTile));
@@ -425,16 +460,17 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
         int32_t slot = 0;
         for (int b = 0; b < batch; ++b) {
             if (seqLen[b] == 0) continue;
-            const int64_t kl = kvSeqLen[b];
-            const int ns = (int)std::max<int64_t>(1, (kl + split - 1) / split);
+            int64_t lo, hi;
+            key_range(b, &lo, &hi);
+            const int ns = (int)std::max<int64_t>(1, (hi - lo + split - 1) / split);
             for (int kvh = 0; kvh < kvHeadNum; ++kvh) {
                 citems.push_back({slot, ns, b, kvh});
                 for (int s = 0; s < ns; ++s) {
                     DecodeUnit u{};
                     u.b = b;
                     u.kvh = kvh;
-                    u.t_begin = (int32_t)std::min<int64_t>(kl, s * split);
-                    u.t_end = (int32_t)std::min<int64_t>(kl, (s + 1) * split);
+                    u.t_begin = (int32_t)std::min<int64_t>(hi, lo + s * split);
+                    u.t_end = (int32_t)std::min<int64_t>(hi, lo + (s + 1) * split);
                     u.slot = slot + s;
                     units.push_back(u);
                 }
@@ -466,13 +502,21 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
         const bool causal = (maskType != FIA_MASK_NONE);
         // Pairs of 128-token tiles that read the same KV head: two heads of a
         // GQA group (same tile), else two consecutive tiles of one head.  Tile
-        // 0 of a pair needs no more key tiles than tile 1.
+        // 0 of a pair needs no more key tiles than tile 1.  Under a band mask
+        // a tile's key tiles start past 0 too, so g = 1 tiles stay unpaired
+        // (both tiles of a pair then always share one key-tile range).
+        // (The kernel derives the same ranges from the same rule.)
         auto ntiles = [&](int b, int q0) {
-            const int ql = seqLen[b], kl = kvSeqLen[b];
-            const int rows = std::min(kPrefillBM, ql - q0);
-            int kv_end = causal ? std::min(kl, kl - ql + q0 + rows) : kl;
-            kv_end = std::max(kv_end, 0);
-            return (kv_end + kPrefillBN - 1) / kPrefillBN;
+            const int64_t ql = seqLen[b], kl = kvSeqLen[b];
+            const int64_t rows = std::min<int64_t>(kPrefillBM, ql - q0);
+            const int64_t qmin = kl - ql + q0, qmax = qmin + rows - 1;
+            int64_t lo = 0, hi = causal ? std::min(kl, qmax + 1) : kl;
+            if (band) {
+                lo = std::max<int64_t>(0, qmin - pre_tok);
+                hi = std::min<int64_t>(kl, qmax + next_tok + 1);
+            }
+            if (hi <= lo) return 0;
+            return (int)((hi + kPrefillBN - 1) / kPrefillBN - lo / kPrefillBN);
         };
         struct Cand {
             PrefillItem it;
@@ -503,9 +547,10 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
             } else {
                 for (int h = 0; h < headNum; ++h) {
                     int qt = 0;
-                    for (; qt + 1 < nqt; qt += 2)
-                        add(b, h, qt * kPrefillBM, h, (qt + 1) * kPrefillBM, h);
-                    if (qt < nqt) add(b, h, 0, -1, qt * kPrefillBM, h);
+                    if (!band)
+                        for (; qt + 1 < nqt; qt += 2)
+                            add(b, h, qt * kPrefillBM, h, (qt + 1) * kPrefillBM, h);
+                    for (; qt < nqt; ++qt) add(b, h, 0, -1, qt * kPrefillBM, h);
                 }
             }
         }

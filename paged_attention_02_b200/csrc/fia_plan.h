@@ -58,6 +58,8 @@ struct CommonArgs {
     int32_t pse_vec;        // pse rows 16-byte aligned (vector loads allowed)
     int32_t pse_tma;        // prefill: pse boxes fetched by TMA (tensor map tp)
     int32_t kv_layout;      // 0: [blocks, bs, KVH, D]; 1: [blocks, KVH, bs, D]
+    int32_t band;           // band mask: keys qpos - pre .. qpos + next
+    int32_t pre, next;      // band limits (clamped to +-2^30)
     float scale_log2;       // qkScale * log2(e)
 };
 

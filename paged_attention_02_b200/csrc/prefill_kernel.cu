@@ -91,8 +91,10 @@ struct PairGeom {
     int b, kvh, cu_q, qlen, kvlen;
     SubGeom t[2];
     int nA, nB;   // key tiles of tile 0 (0 if absent) and tile 1; nA <= nB
+    int j0;       // first key tile (past 0 only under a band mask; both tiles share it)
 };
 
+template <bool BAND>
 __device__ __forceinline__ PairGeom pair_geom(const PrefillArgs &a, const PrefillItem *items,
                                               const SeqInfo *seqs, int idx) {
     const PrefillItem it = items[idx];
@@ -100,6 +102,7 @@ __device__ __forceinline__ PairGeom pair_geom(const PrefillArgs &a, const Prefil
     const bool causal = (a.c.mask_type == 9 || a.c.mask_type == 3);
     PairGeom g;
     g.b = it.b; g.kvh = it.kvh; g.cu_q = si.cu_q; g.qlen = si.qlen; g.kvlen = si.kvlen;
+    g.j0 = 0;
 #pragma unroll
     for (int x = 0; x < 2; ++x) {
         SubGeom &s = g.t[x];
@@ -107,9 +110,15 @@ __device__ __forceinline__ PairGeom pair_geom(const PrefillArgs &a, const Prefil
         s.q0 = it.q0[x];
         s.h = it.h[x];
         s.rows = s.valid ? min(kPrefillBM, si.qlen - it.q0[x]) : 0;
-        int kv_end = causal ? min(si.kvlen, si.kvlen - si.qlen + it.q0[x] + s.rows) : si.kvlen;
-        kv_end = max(kv_end, 0);
-        s.n = s.valid ? (kv_end + kPrefillBN - 1) / kPrefillBN : 0;
+        // keys the tile's rows can see: [lo, hi) (same rule as the host plan)
+        const int qmin = si.kvlen - si.qlen + it.q0[x], qmax = qmin + s.rows - 1;
+        int lo = 0, hi = causal ? min(si.kvlen, qmax + 1) : si.kvlen;
+        if constexpr (BAND) {
+            lo = max(0, qmin - a.c.pre);
+            hi = min(si.kvlen, qmax + a.c.next + 1);
+        }
+        s.n = (s.valid && hi > lo) ? (hi + kPrefillBN - 1) / kPrefillBN - lo / kPrefillBN : 0;
+        if (BAND && s.valid && hi > lo) g.j0 = lo / kPrefillBN;
     }
     g.nA = g.t[0].n;
     g.nB = g.t[1].n;
@@ -127,7 +136,7 @@ __device__ __forceinline__ PairGeom pair_geom(const PrefillArgs &a, const Prefil
         }                                                                                 \
     } while (0)
 
-template <typename T, int D, int MODE, int PB>
+template <typename T, int D, int MODE, int PB, bool BAND>
 __global__ void __launch_bounds__(576, 1)
 fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tq,
                    const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
@@ -215,7 +224,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             uint32_t q_it = 0, kv_it = 0;
             const int br = a.c.box_rows;
             for (idx = it_begin; idx < it_end; ++idx) {
-                const PairGeom gm = pair_geom(a, items, seqs, idx);
+                const PairGeom gm = pair_geom<BAND>(a, items, seqs, idx);
                 if (gm.nB == 0) continue;
                 FIA_WAIT(q_empty, (q_it & 1) ^ 1, 10);
                 mbar_arrive_expect_tx(q_full, (gm.t[0].valid ? 2 : 1) * Cfg::kTileBytes);
@@ -230,7 +239,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 const int32_t *bt_row = a.c.bt + (int64_t)gm.b * a.c.bt_stride;
                 for (int j = 0; j < gm.nB; ++j, ++kv_it) {
                     dbg_j = j;
-                    const int t0 = j * kPrefillBN;
+                    const int t0 = (gm.j0 + j) * kPrefillBN;
                     const int t1 = min(t0 + kPrefillBN, gm.kvlen);
                     const int nbox = (t1 - t0 + br - 1) / br;
                     const uint32_t bytes = (uint32_t)(nbox * br * 128 * Cfg::kHalves);
@@ -300,7 +309,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         static_assert(kPrefillBN / 16 == 8, "PV issue assumes 8 key steps per tile");
         static_assert(NKQ == 4 || NKQ == 8, "QK issue assumes D = 64 or 128");
         for (idx = it_begin; idx < it_end; ++idx) {
-            const PairGeom gm = pair_geom(a, items, seqs, idx);
+            const PairGeom gm = pair_geom<BAND>(a, items, seqs, idx);
             if (gm.nB == 0) continue;
             dbg_j = -1;
             // descriptors are rebuilt before each wait rather than kept live:
@@ -337,7 +346,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 vmajor(v_lo + vs * kTileStep, vd);
                 kmajor(k_lo + ksn * kTileStep, kd);
                 FIA_WAIT(&v_full[vs], (kvi / VS) & 1, 24);
-                const int valid = gm.kvlen - j * kPrefillBN;
+                const int valid = gm.kvlen - (gm.j0 + j) * kPrefillBN;
                 if (valid < kPrefillBN) {
                     // rows past kvSeqLen: P is 0 there, but the slots may hold
                     // anything (NaN * 0 = NaN in the MMA): the bulk-copy engine
@@ -454,24 +463,30 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         uint8_t *pslot = smem + Cfg::kOffPse + sw * 4096;
         uint64_t *pbar = &pse_full[sw];
         // lane 0 fetches this warp's two pse boxes (16 rows x 64 keys each) of
-        // key tile jt
+        // the item's key tile jt (counted from its first key tile j0)
         auto pse_fetch = [&](const PairGeom &g2, const SubGeom &s2, int jt) {
             if (lane == 0) {
                 mbar_arrive_expect_tx(pbar, 4096);
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh)
-                    tma_load_3d(pslot + hh * 2048, &tp, pbar, jt * kPrefillBN + 64 * hh,
+                    tma_load_3d(pslot + hh * 2048, &tp, pbar, (g2.j0 + jt) * kPrefillBN + 64 * hh,
                                 s2.q0 + 32 * quad + 16 * sub, g2.b * a.c.H + s2.h);
             }
         };
 
         for (idx = it_begin; idx < it_end; ++idx) {
-            const PairGeom gm = pair_geom(a, items, seqs, idx);
+            const PairGeom gm = pair_geom<BAND>(a, items, seqs, idx);
             const SubGeom sg = gm.t[X];
             if (!sg.valid) continue;
             const int i = sg.q0 + row;
             const bool valid = i < gm.qlen;
             const int qpos = gm.kvlen - gm.qlen + i;
+            // under a band mask the keys this row may see are [klo, khi)
+            int klo = 0, khi = gm.kvlen;
+            if constexpr (BAND) {
+                klo = max(0, qpos - a.c.pre);
+                khi = min(khi, qpos + a.c.next + 1);
+            }
             const int64_t orow = ((int64_t)(gm.cu_q + i) * a.c.H + sg.h);
             if (sg.n == 0) {
                 if (valid) {
@@ -494,7 +509,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             if (pse_tma) pse_fetch(gm, sg, 0);
             for (int j = 0; j < sg.n; ++j) {
                 dbg_j = j;
-                const int tb = j * kPrefillBN + 64 * half;     // first key of this lane
+                const int tb = (gm.j0 + j) * kPrefillBN + 64 * half;   // first key of this lane
                 FIA_WAIT(&s_full[X], s_it & 1, 30);
                 ++s_it;
                 __syncwarp();          // tcgen05.ld/st below are warp-collective (.aligned)
@@ -507,7 +522,8 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 for (int cc = 0; cc < 2; ++cc) reg_fence32(sr[cc]);
 
                 // ---- scores (log2 units unless folded), bias, masks ----
-                const bool edge = (tb + 64 > gm.kvlen) || (causal && tb + 63 > qpos);
+                const bool edge = BAND ? (tb < klo) || (tb + 64 > khi)
+                                       : (tb + 64 > gm.kvlen) || (causal && tb + 63 > qpos);
                 if constexpr (MODE == kModeAlibi) {
                     // bias slope * (t - qpos) in log2 units, two keys at a time:
                     // the key offset pair is carried as exact floats (integers
@@ -592,7 +608,8 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
 #pragma unroll
                         for (int x = 0; x < 32; ++x) {
                             const int t = tb + cc * 32 + x;
-                            const bool keep = (t < gm.kvlen) && !(causal && t > qpos);
+                            const bool keep = BAND ? (t >= klo) && (t < khi)
+                                                   : (t < gm.kvlen) && !(causal && t > qpos);
                             if (!keep) sr[cc][x] = __float_as_uint(-INFINITY);
                         }
                 }
@@ -700,7 +717,10 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 M = fmaxf(mu, s2);
                 lt = l * ex2(mu - M) + ex2(s2 - M);
             }
-            const float oscale = ex2(mu - M) / lt;
+            // a row with no visible key (possible under a band mask): out 0,
+            // lse +inf, with or without a sink
+            const bool no_key = BAND && (m == -INFINITY);
+            const float oscale = no_key ? 0.f : ex2(mu - M) / lt;
 #pragma unroll
             for (int cc = 0; cc < DH / 32; ++cc) {
                 uint32_t orr[32];
@@ -720,7 +740,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 }
                 __syncwarp();
             }
-            if (valid && a.c.lse && half == 0) a.c.lse[orow] = (M + log2f(lt)) * kLn2;
+            if (valid && a.c.lse && half == 0) a.c.lse[orow] = no_key ? INFINITY : (M + log2f(lt)) * kLn2;
             tc_fence_before();
             __syncwarp();
         }
@@ -735,21 +755,21 @@ done:
     }
 }
 
-template <typename T, int D, int MODE>
+template <typename T, int D, int MODE, bool BAND>
 static cudaError_t launch_prefill_t(const PrefillArgs &a, const CUtensorMap &tq,
                                     const CUtensorMap &tk, const CUtensorMap &tv,
                                     const CUtensorMap &tp, int grid,
                                     const uint8_t *inline_plan, cudaStream_t s) {
     const int smem = PrefillCfg<D, MODE>::kSmem;
     if (inline_plan) {
-        auto kern = fia_prefill_kernel<T, D, MODE, kInlinePlanBytes>;
+        auto kern = fia_prefill_kernel<T, D, MODE, kInlinePlanBytes, BAND>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         // inline_plan points at a full PlanBytes<kInlinePlanBytes> kept by the op
         kern<<<grid, PrefillCfg<D, MODE>::kThreads, smem, s>>>(
             a, tq, tk, tv, tp, *reinterpret_cast<const PlanBytes<kInlinePlanBytes> *>(inline_plan));
     } else {
-        auto kern = fia_prefill_kernel<T, D, MODE, 16>;
+        auto kern = fia_prefill_kernel<T, D, MODE, 16, BAND>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         PlanBytes<16> pl{};
@@ -763,9 +783,16 @@ static cudaError_t launch_prefill_mode(const PrefillArgs &a, const CUtensorMap &
                                        const CUtensorMap &tk, const CUtensorMap &tv,
                                        const CUtensorMap &tp, int grid, const uint8_t *ip,
                                        cudaStream_t s) {
-    if (a.c.pse) return launch_prefill_t<T, D, kModePse>(a, tq, tk, tv, tp, grid, ip, s);
-    if (a.c.mask_type == 3) return launch_prefill_t<T, D, kModeAlibi>(a, tq, tk, tv, tp, grid, ip, s);
-    return launch_prefill_t<T, D, kModePlain>(a, tq, tk, tv, tp, grid, ip, s);
+    // a band mask excludes maskType (no causal, no ALiBi): its own instances
+    // keep the band's range checks out of the other kernels
+    if (a.c.band) {
+        if (a.c.mask_type != 0) return cudaErrorInvalidValue;
+        if (a.c.pse) return launch_prefill_t<T, D, kModePse, true>(a, tq, tk, tv, tp, grid, ip, s);
+        return launch_prefill_t<T, D, kModePlain, true>(a, tq, tk, tv, tp, grid, ip, s);
+    }
+    if (a.c.pse) return launch_prefill_t<T, D, kModePse, false>(a, tq, tk, tv, tp, grid, ip, s);
+    if (a.c.mask_type == 3) return launch_prefill_t<T, D, kModeAlibi, false>(a, tq, tk, tv, tp, grid, ip, s);
+    return launch_prefill_t<T, D, kModePlain, false>(a, tq, tk, tv, tp, grid, ip, s);
 }
 
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tq, const CUtensorMap &tk,

@@ -20,7 +20,8 @@ def run_gpu(p, device="cuda", **overrides):
               v_offset=d(p.v_offset), want_lse=p.want_lse,
               kv_layout=int(getattr(p, "kv_layout", 0)),
               k_antiquant_mode=int(getattr(p, "k_antiquant_mode", 0)),
-              v_antiquant_mode=int(getattr(p, "v_antiquant_mode", 0)))
+              v_antiquant_mode=int(getattr(p, "v_antiquant_mode", 0)),
+              band=getattr(p, "band", None))
     kw.update(overrides)
     op = fia.FiaOp(d(p.query), d(p.key_cache), d(p.value_cache), d(p.block_tables),
                    [int(x) for x in p.seq_len], [int(x) for x in p.kv_seq_len], p.head_num,

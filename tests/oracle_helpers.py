@@ -108,6 +108,11 @@ def dense_sdpa(p: Problem) -> np.ndarray:
         if p.mask_type in (3, 9):
             allowed = torch.ones(ql, kl, dtype=torch.bool).tril(diagonal=kl - ql)
             bias = bias.masked_fill(~allowed, float("-inf"))
+        if getattr(p, "band", None) is not None:
+            pre, nxt = p.band
+            rel = torch.arange(kl)[None, :] - (torch.arange(ql)[:, None] + (kl - ql))   # t - qpos
+            inside = (rel >= -pre) & (rel <= nxt)
+            bias = bias.masked_fill(~inside, float("-inf"))
         if p.mask_type == 3:
             rel = (torch.arange(kl)[None, :] - (torch.arange(ql)[:, None] + (kl - ql))).double()
             bias = bias + p.slopes.double()[:, None, None] * rel[None]

@@ -61,7 +61,8 @@ def _call(**kw):
     d = {k: tensor_desc(v) for k, v in t.items()}
     P = lambda x: ctypes.pointer(x) if x is not None else None
     ext = fia_ext(P(d["pse"]), P(d["sink"]), P(d["ks"]), None, P(d["vs"]), None, P(d["lse"]),
-                  int(args.get("layout", 0)), int(args.get("kmode", 0)), int(args.get("vmode", 0)))
+                  int(args.get("layout", 0)), int(args.get("kmode", 0)), int(args.get("vmode", 0)),
+                  int(args.get("sparse", 0)), int(args.get("pre", 0)), int(args.get("next", 0)))
     n = max(len(args["seq"]), 1)
     sl = (ctypes.c_int32 * n)(*args["seq"])
     kl = (ctypes.c_int32 * n)(*args["kv"])
@@ -176,3 +177,16 @@ def test_phase1_per_token_antiquant_rules():
                  vmode=1) == L.FIA_ERR_DTYPE
     # a mode on a bf16 cache is a parameter error
     assert _call(kmode=1) == L.FIA_ERR_PARAM
+
+
+def test_phase1_band_rules():
+    """Band mask (V3 sparseMode 4): replaces maskType (which must be
+    FIA_MASK_NONE) and needs preTokens + nextTokens >= 0."""
+    from paged_attention_02_b200 import _lib as L
+    ok = (L.FIA_ERR_CUDA, L.FIA_OK)
+    assert _call(mask=0, sparse=4, pre=100, next=0) in ok
+    assert _call(mask=0, sparse=4, pre=-5, next=5) in ok
+    assert _call(mask=0, sparse=4, pre=2 ** 62, next=2 ** 62) in ok        # huge limits clamp
+    assert _call(mask=9, sparse=4, pre=100, next=0) == L.FIA_ERR_PARAM      # with causal
+    assert _call(mask=0, sparse=4, pre=3, next=-4) == L.FIA_ERR_PARAM       # empty band
+    assert _call(mask=0, sparse=3, pre=3, next=0) == L.FIA_ERR_PARAM        # other sparse modes

@@ -309,3 +309,37 @@ def test_int8_per_token_antiquant(name):
     _, out, lse = run_gpu(p)
     ref_out, ref_lse = oracle.attention(p)
     compare(out, lse, ref_out, ref_lse, name)
+
+
+# Band mask (V3 sparseMode 4 with preTokens / nextTokens; sliding window is
+# nextTokens = 0): prefill skips the key tiles outside the band, decode reads
+# only the band's keys; rows whose band holds no key give out 0, lse +inf.
+BAND_CASES = {
+    "prefill_gqa_window200": dict(seq_len=[300, 130], kv_seq_len=[700, 130], head_num=8,
+                                  kv_head_num=2, head_size=128, block_size=64, band=(200, 0)),
+    "prefill_mha_band_f16": dict(seq_len=[400], kv_seq_len=[512], head_num=4, kv_head_num=4,
+                                 head_size=128, block_size=32, dtype="f16", band=(150, 20)),
+    "prefill_empty_rows_sink": dict(seq_len=[200, 50], kv_seq_len=[260, 50], head_num=4,
+                                    kv_head_num=2, head_size=64, block_size=16, sink=True,
+                                    band=(-3, 10)),
+    "prefill_pse_window": dict(seq_len=[140], kv_seq_len=[400], head_num=4, kv_head_num=2,
+                               head_size=128, block_size=128, pse=True, band=(100, 0)),
+    "decode_window256": dict(seq_len=[1] * 3, kv_seq_len=[4000, 100, 1300], head_num=16,
+                             kv_head_num=4, head_size=128, block_size=128, band=(255, 0)),
+    "decode_mtp_band_d64": dict(seq_len=[3, 2], kv_seq_len=[500, 64], head_num=8, kv_head_num=2,
+                                head_size=64, block_size=16, band=(77, 1)),
+    "decode_int8_window": dict(seq_len=[1, 2], kv_seq_len=[3000, 777], head_num=16,
+                               kv_head_num=2, head_size=128, block_size=64, kv_dtype="i8",
+                               sink=True, band=(500, 0)),
+    "decode_band_excludes_all": dict(seq_len=[1, 1], kv_seq_len=[300, 40], head_num=8,
+                                     kv_head_num=2, head_size=128, block_size=16, band=(-50, 60)),
+}
+
+
+@pytest.mark.parametrize("name", sorted(BAND_CASES))
+def test_band_mask(name):
+    p = W.make_problem(name=name, seed=zlib.crc32(name.encode()) % 10000, spare_blocks=2,
+                       **BAND_CASES[name])
+    _, out, lse = run_gpu(p)
+    ref_out, ref_lse = oracle.attention(p)
+    compare(out, lse, ref_out, ref_lse, name)

@@ -344,3 +344,69 @@ def test_oracle_per_token_uses_each_tokens_own_scale():
     rows_seq1 = slice(int(p.seq_len[0]), int(p.seq_len[0] + p.seq_len[1]))
     assert not np.allclose(out4[rows_seq1], out[rows_seq1])
     assert np.array_equal(out4[:int(p.seq_len[0])], out[:int(p.seq_len[0])])
+
+
+def _band_problem(band, mask=W.MASK_NONE, **kw):
+    cfg = dict(seq_len=[40, 1, 7, 3], kv_seq_len=[100, 90, 7, 60], head_num=4, kv_head_num=2,
+               head_size=64, block_size=16)
+    cfg.update(kw)
+    return W.make_problem(seed=23, mask_type=mask, band=band, **cfg)
+
+
+def test_oracle_band_special_cases():
+    """Band mask (V3 sparseMode 4, preTokens / nextTokens): with preTokens
+    past every key and nextTokens = 0 it is the causal mask; with both past
+    every key it is no mask (bitwise)."""
+    big = 10 ** 6
+    causal = oracle.attention(_band_problem(None, mask=W.MASK_CAUSAL))
+    band_causal = oracle.attention(_band_problem((big, 0)))
+    assert all(np.array_equal(x, y) for x, y in zip(causal, band_causal))
+    full = oracle.attention(_band_problem(None))
+    band_full = oracle.attention(_band_problem((big, big)))
+    assert all(np.array_equal(x, y) for x, y in zip(full, band_full))
+
+
+def test_oracle_band_single_key():
+    """preTokens = nextTokens = 0 leaves each row exactly one key, its own
+    position qpos: out is that key's value row (softmax of one score is 1) and
+    lse is the scaled score itself."""
+    p = _band_problem((0, 0), want_lse=True)
+    out, lse = oracle.attention(p)
+    g = p.head_num // p.kv_head_num
+    bs = p.block_size
+    cu = p.cu_seq()
+    q = p.query.double()
+    for b in range(p.batch):
+        kl, ql = int(p.kv_seq_len[b]), int(p.seq_len[b])
+        for i in range(ql):
+            qpos = kl - ql + i
+            blk = int(p.block_tables[b, qpos // bs])
+            for h in range(p.head_num):
+                kvh = h // g
+                k = p.key_cache[blk, qpos % bs, kvh].double()
+                v = p.value_cache[blk, qpos % bs, kvh].double().numpy()
+                r = cu[b] + i
+                assert np.array_equal(out[r, h], v)
+                score = p.qk_scale * float(q[r, h] @ k)
+                assert abs(lse[r, h] - score) <= 1e-12 * max(1.0, abs(score))
+
+
+@pytest.mark.parametrize("band", [(20, 3), (0, 0), (5, -2), (-3, 40)])
+def test_oracle_band_against_sdpa(band):
+    """Against torch SDPA with the band written out as an additive mask
+    (t - qpos in [-preTokens, nextTokens]); rows whose band holds no key give
+    out 0 and lse +inf (the empty-row rule)."""
+    p = _band_problem(band, sink=True)
+    out, lse = oracle.attention(p)
+    ref = dense_sdpa(p)
+    empty = np.isinf(lse)
+    cu = p.cu_seq()
+    # which rows must be empty: band interval clipped to [0, kvSeqLen) is void
+    for b in range(p.batch):
+        kl, ql = int(p.kv_seq_len[b]), int(p.seq_len[b])
+        for i in range(ql):
+            qpos = kl - ql + i
+            lo, hi = max(0, qpos - band[0]), min(kl - 1, qpos + band[1])
+            assert bool(empty[cu[b] + i].all()) == (hi < lo)
+    assert np.all(out[empty] == 0)
+    assert np.abs(out[~empty] - ref[~empty]).max() < 1e-9

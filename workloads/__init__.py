@@ -23,7 +23,7 @@ from __future__ import annotations
 
 import dataclasses
 import math
-from typing import List, Optional, Sequence
+from typing import List, Optional, Sequence, Tuple
 
 import numpy as np
 import torch
@@ -61,6 +61,7 @@ class Problem:
     kv_layout: int = 0                        # 0 BnBsH, 1 BnNBsD
     k_antiquant_mode: int = 0                 # int8: 0 per-channel [KVH, D], 1 per-token [B, S]
     v_antiquant_mode: int = 0
+    band: Optional[Tuple[int, int]] = None    # (preTokens, nextTokens): band mask
 
     @property
     def batch(self) -> int:
@@ -121,6 +122,7 @@ def make_problem(
     kv_layout: int = 0,
     k_antiquant: str = "channel",
     v_antiquant: str = "channel",
+    band: Optional[Tuple[int, int]] = None,
 ) -> Problem:
     """Draw a seeded problem.
 
@@ -223,6 +225,7 @@ def make_problem(
         k_scale=ks, k_offset=ko, v_scale=vs, v_offset=vo, want_lse=want_lse,
         k_antiquant_mode=km if kv_dtype == "i8" else 0,
         v_antiquant_mode=vm if kv_dtype == "i8" else 0,
+        band=tuple(band) if band is not None else None,
     )
     return to_bnnbsd(p) if kv_layout == 1 else p
 
