@@ -56,7 +56,13 @@ def unmasked_pairs(p) -> int:
     tot = 0
     for b in range(p.batch):
         ql, kl = int(p.seq_len[b]), int(p.kv_seq_len[b])
-        if p.mask_type in (W.MASK_CAUSAL, W.MASK_ALIBI):
+        if p.band is not None:
+            # band: keys qpos - pre .. qpos + next, clipped to [0, kvSeqLen)
+            qpos = np.arange(kl - ql, kl, dtype=np.int64)
+            lo = np.maximum(0, qpos - p.band[0])
+            hi = np.minimum(kl - 1, qpos + p.band[1])
+            tot += int(np.maximum(0, hi - lo + 1).sum())
+        elif p.mask_type in (W.MASK_CAUSAL, W.MASK_ALIBI):
             pre = kl - ql
             tot += ql * pre + ql * (ql + 1) // 2
         else:
@@ -69,9 +75,17 @@ def flops(p) -> float:
 
 
 def kv_bytes(p) -> int:
-    """K+V bytes a decode pass must read once per KV head."""
+    """K+V bytes a decode pass must read once per KV head, plus the per-token
+    dequantisation scales / offsets (fp32, one per cached token) once."""
     es = 1 if p.kv_is_int8 else 2
-    return int(sum(int(k) for k in p.kv_seq_len)) * p.kv_head_num * p.head_size * es * 2
+    tokens = int(sum(int(k) for k in p.kv_seq_len))
+    per_token = 0
+    if p.kv_is_int8:
+        for mode, arrs in ((p.k_antiquant_mode, (p.k_scale, p.k_offset)),
+                           (p.v_antiquant_mode, (p.v_scale, p.v_offset))):
+            if mode == 1:
+                per_token += tokens * 4 * sum(a is not None for a in arrs)
+    return tokens * p.kv_head_num * p.head_size * es * 2 + per_token
 
 
 def io_bytes(p) -> int:
@@ -402,7 +416,10 @@ def main():
                          ("alibi_prefill_pse", lambda: W.alibi_prefill(True)),
                          ("tiny_decode", W.tiny_decode),
                          ("decode_large_batch_bnnbsd", W.decode_large_batch_bnnbsd),
-                         ("prefill_prefix_bnnbsd", W.prefill_prefix_bnnbsd)):
+                         ("prefill_prefix_bnnbsd", W.prefill_prefix_bnnbsd),
+                         ("mtp_decode", W.mtp_decode),
+                         ("int8_per_token_decode", W.int8_per_token_decode),
+                         ("sliding_window_prefill", W.sliding_window_prefill)):
             q = fn()
             td = to_dev(q, dev)
             o2 = make_op(q, td)

@@ -238,6 +238,31 @@ def test_config_int8_long_decode_full():
     _full_size(p, 256, 4)
 
 
+def test_config_bnnbsd_full():
+    """The two BnNBsD bench workloads at full size."""
+    op, _, _ = _full_size(W.decode_large_batch_bnnbsd(), 256, 5)
+    assert op.plan_info()["path"] == 1
+    op, _, _ = _full_size(W.prefill_prefix_bnnbsd(), 256, 6)
+    assert op.plan_info()["path"] == 2
+
+
+def test_config_mtp_decode_full():
+    p = W.mtp_decode()
+    op, _, _ = _full_size(p, 512, 7)
+    assert op.plan_info()["path"] == 1
+
+
+def test_config_int8_per_token_decode_full():
+    _full_size(W.int8_per_token_decode(), 256, 8)
+
+
+def test_config_sliding_window_prefill_full():
+    p = W.sliding_window_prefill()
+    op, _, lse = _full_size(p, 384, 9)
+    assert op.plan_info()["path"] == 2
+    assert np.all(np.isfinite(lse))          # every row sees at least itself
+
+
 # BnNBsD cache layout [numBlocks, kvHeadNum, blockSize, headSize] (V3 paged
 # attention constraints: BnBsH or BnNBsD, the latter recommended): the kernels
 # read each (block, KV head) run as one TMA box.  Checked against the oracle on

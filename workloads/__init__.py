@@ -306,6 +306,36 @@ def prefill_prefix_bnnbsd() -> Problem:
     return dataclasses.replace(to_bnnbsd(prefill_prefix()), name="prefill_prefix_bnnbsd")
 
 
+def mtp_decode() -> Problem:
+    """Multi-token (speculative) decode: 4 new tokens per sequence, causal
+    among themselves, on the decode_large_batch sequences (B=64, kvSeqLen ~
+    U[1024, 8192] including the 4 new tokens, H=32, KVH=8 so 16 rows per KV
+    head, D=128, bs=128, bf16)."""
+    rng = np.random.Generator(np.random.PCG64(3))
+    kv = rng.integers(1024, 8193, 64).astype(np.int32)
+    return make_problem(name="mtp_decode_causal", seed=6, seq_len=[4] * 64, kv_seq_len=kv,
+                        head_num=32, kv_head_num=8, head_size=128, block_size=128,
+                        dtype="bf16", mask_type=MASK_CAUSAL)
+
+
+def int8_per_token_decode() -> Problem:
+    """int8_long_decode with per-token dequantisation: K and V scale / offset
+    of shape [B, S] fp32 (one pair per cached token, shared by the KV heads)."""
+    return make_problem(name="int8_long_decode_per_token", seed=7, seq_len=[1] * 16,
+                        kv_seq_len=[32768] * 16, head_num=64, kv_head_num=8, head_size=128,
+                        block_size=128, dtype="bf16", kv_dtype="i8", mask_type=MASK_NONE,
+                        sink=True, k_antiquant="token", v_antiquant="token")
+
+
+def sliding_window_prefill() -> Problem:
+    """Sliding-window prefill (band mask, preTokens=1023, nextTokens=0: each
+    token sees itself and the 1023 before it): B=2, seqLen=kvSeqLen=4096,
+    H=32, KVH=8, D=128, bs=128, bf16."""
+    return make_problem(name="sliding_window_prefill", seed=8, seq_len=[4096, 4096],
+                        kv_seq_len=[4096, 4096], head_num=32, kv_head_num=8, head_size=128,
+                        block_size=128, dtype="bf16", mask_type=MASK_NONE, band=(1023, 0))
+
+
 NAMED = {
     "tiny_decode": tiny_decode,
     "prefill_prefix": prefill_prefix,
@@ -315,6 +345,9 @@ NAMED = {
     "int8_long_decode": int8_long_decode,
     "decode_large_batch_bnnbsd": decode_large_batch_bnnbsd,
     "prefill_prefix_bnnbsd": prefill_prefix_bnnbsd,
+    "mtp_decode": mtp_decode,
+    "int8_per_token_decode": int8_per_token_decode,
+    "sliding_window_prefill": sliding_window_prefill,
 }
 
 
