@@ -387,7 +387,11 @@ struct DecodeI8Cfg {
     static constexpr int kMergeBytes = 4 * kDecodeRows * D * 4 + 4 * kDecodeRows * 8;
     static constexpr int kDataBytes =
         (kStages * kStageBytes > kMergeBytes) ? kStages * kStageBytes : kMergeBytes;
-    static constexpr int kSmem = 1024 /*align slack*/ + kDataBytes + 2 * kStages * 8 + 16;
+    // per-token dequantisation parameters, per warp: [2 buffers][4 arrays:
+    // K scale, K offset, V scale, V offset][16 keys] fp32, after the barriers
+    static constexpr int kOffTok = kDataBytes + 2 * kStages * 8 + 16;
+    static constexpr int kTokBytes = 4 * 2 * 4 * 16 * 4;
+    static constexpr int kSmem = 1024 /*align slack*/ + kOffTok + kTokBytes;
 };
 
 int decode_smem_bytes(int D, bool kv_int8) {
@@ -564,6 +568,25 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
     const float *kor = (ktok && a.k_offset) ? a.k_offset + (int64_t)u.b * a.k_tok_stride : nullptr;
     const float *vsr = vtok ? a.v_scale + (int64_t)u.b * a.v_tok_stride : nullptr;
     const float *vor = (vtok && a.v_offset) ? a.v_offset + (int64_t)u.b * a.v_tok_stride : nullptr;
+    // This warp's 16 keys of key tile jt: their per-token parameters are
+    // copied into shared-memory buffer jt & 1 one tile ahead (lane L copies
+    // array L >> 4 and array 2 + (L >> 4) for key L & 15), so their latency
+    // hides behind the previous tile.  Keys past the unit's end and absent
+    // offsets read as 0 (the key loop then needs no bounds tests: a zero V
+    // scale keeps 0 * garbage out of P).  One commit group per call.
+    float *tokbuf = reinterpret_cast<float *>(smem + Cfg::kOffTok) + warp * 128;
+    auto tok_fetch = [&](int jt) {
+        const int t = u.t_begin + jt * kDecodeTile + warp * 16 + (lane & 15);
+        const float *s0 = (lane < 16) ? ksr : kor;
+        const float *s1 = (lane < 16) ? vsr : vor;
+        float *dst = tokbuf + (jt & 1) * 64;
+        if (s0 && t < u.t_end) cp_async4(smem_u32(dst + lane), s0 + t);
+        else dst[lane] = 0.f;
+        if (s1 && t < u.t_end) cp_async4(smem_u32(dst + 32 + lane), s1 + t);
+        else dst[32 + lane] = 0.f;
+        cp_async_commit();
+    };
+    if constexpr (KTOK || VTOK) tok_fetch(0);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
         voff[nt][0] = voff[nt][1] = 0.f;
@@ -580,7 +603,15 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
     for (int j = 0; j < n_tiles; ++j) {
         const int s = j % STAGES;
         if (!mbar_wait(&full[s], (j / STAGES) & 1, abort_flag, a.c.err, 1)) { ok = false; break; }
-        __syncwarp();      // movmatrix / mma.sync below are warp-collective (.aligned)
+        const float *tok = tokbuf + (j & 1) * 64;
+        if constexpr (KTOK || VTOK) {
+            // buffer (j + 1) & 1 was last read in tile j - 1, before a __syncwarp
+            if (j + 1 < n_tiles) tok_fetch(j + 1);
+            else cp_async_commit();
+            cp_async_wait<1>();            // this tile's group has landed
+        }
+        __syncwarp();      // movmatrix / mma.sync below are warp-collective (.aligned);
+                           // also makes every lane's parameter copies visible
         const uint32_t kst = smem_u32(smem + s * Cfg::kStageBytes);
         const uint32_t vst = kst + Cfg::kTileBytes;
         const int tw = u.t_begin + j * kDecodeTile + warp * 16;   // first key of this warp
@@ -625,11 +656,8 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
         if constexpr (KTOK) {
 #pragma unroll
             for (int hk = 0; hk < 2; ++hk) {
-                const int t = tw + r + 8 * hk;
-                if (t < u.t_end) {
-                    kf[hk] = ksr[t] * a.c.scale_log2;
-                    kof[hk] = kor ? kor[t] : 0.f;
-                }
+                kf[hk] = tok[r + 8 * hk] * a.c.scale_log2;
+                kof[hk] = tok[16 + r + 8 * hk];
             }
         }
 #pragma unroll
@@ -686,9 +714,8 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
         if constexpr (VTOK) {
 #pragma unroll
             for (int hk = 0; hk < 2; ++hk) {
-                const int t = tw + r + 8 * hk;
-                vf[hk] = (t < u.t_end) ? vsr[t] : 0.f;
-                vof[hk] = (vor && t < u.t_end) ? vor[t] : 0.f;
+                vf[hk] = tok[32 + r + 8 * hk];
+                vof[hk] = tok[48 + r + 8 * hk];
             }
         }
         __syncwarp();      // movmatrix and mma.sync below are .aligned
@@ -786,6 +813,7 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
         __syncwarp();
     }
     (void)ok;
+    if constexpr (KTOK || VTOK) cp_async_wait<0>();   // no copy outlives the loop
 
     // ---- merge the 4 warps' (m, l, O) and write this unit's partial ----
 #pragma unroll
