@@ -168,7 +168,11 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
         const int s = j % STAGES;
-        if (!mbar_wait(&full[s], (j / STAGES) & 1, abort_flag, a.c.err, 1)) { ok = false; break; }
+        // every lane waits; the warp leaves together if any lane gave up
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (j / STAGES) & 1, abort_flag, a.c.err, 1))) {
+            ok = false;
+            break;
+        }
         __syncwarp();      // ldmatrix / mma.sync below are warp-collective (.aligned)
         const uint32_t kst = smem_u32(smem + s * Cfg::kStageBytes);
         const uint32_t vst = kst + Cfg::kTileBytes;
@@ -308,11 +312,15 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
 
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
+        bool stop = false;
         if (tid == 0 && j + STAGES < n_tiles) {
-            if (!mbar_wait(&empty[s], (j / STAGES) & 1, abort_flag, a.c.err, 2)) { ok = false; break; }
-            issue(j + STAGES);
+            if (mbar_wait(&empty[s], (j / STAGES) & 1, abort_flag, a.c.err, 2)) issue(j + STAGES);
+            else stop = true;
         }
         __syncwarp();
+        // a failed wait ends the key loop for the whole warp at once (lane 0
+        // alone leaving would strand its siblings at a warp barrier)
+        if (__any_sync(0xffffffffu, stop)) { ok = false; break; }
     }
     (void)ok;
 
@@ -602,7 +610,11 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
         const int s = j % STAGES;
-        if (!mbar_wait(&full[s], (j / STAGES) & 1, abort_flag, a.c.err, 1)) { ok = false; break; }
+        // every lane waits; the warp leaves together if any lane gave up
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (j / STAGES) & 1, abort_flag, a.c.err, 1))) {
+            ok = false;
+            break;
+        }
         const float *tok = tokbuf + (j & 1) * 64;
         if constexpr (KTOK || VTOK) {
             // buffer (j + 1) & 1 was last read in tile j - 1, before a __syncwarp
@@ -806,11 +818,15 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
 
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
+        bool stop = false;
         if (tid == 0 && j + STAGES < n_tiles) {
-            if (!mbar_wait(&empty[s], (j / STAGES) & 1, abort_flag, a.c.err, 2)) { ok = false; break; }
-            issue(j + STAGES);
+            if (mbar_wait(&empty[s], (j / STAGES) & 1, abort_flag, a.c.err, 2)) issue(j + STAGES);
+            else stop = true;
         }
         __syncwarp();
+        // a failed wait ends the key loop for the whole warp at once (lane 0
+        // alone leaving would strand its siblings at a warp barrier)
+        if (__any_sync(0xffffffffu, stop)) { ok = false; break; }
     }
     (void)ok;
     if constexpr (KTOK || VTOK) cp_async_wait<0>();   // no copy outlives the loop
