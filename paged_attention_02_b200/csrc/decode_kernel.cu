@@ -942,7 +942,7 @@ static cudaError_t launch_decode_t(const DecodeArgs &a, const CUtensorMap &tk,
                                    const CUtensorMap &tv, int grid, cudaStream_t s) {
     auto kern = fia_decode_kernel<T, D>;
     const int smem = DecodeCfg<D>::kSmem;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = ensure_smem_attr<fia_decode_kernel<T, D>>(smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, 128, smem, s>>>(a, tk, tv);
     return cudaGetLastError();
@@ -953,7 +953,7 @@ static cudaError_t launch_decode_i8_m(const DecodeArgs &a, const CUtensorMap &tk
                                       const CUtensorMap &tv, int grid, cudaStream_t s) {
     auto kern = fia_decode_i8_kernel<T, NT, KTOK, VTOK>;
     const int smem = DecodeI8Cfg::kSmem;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = ensure_smem_attr<fia_decode_i8_kernel<T, NT, KTOK, VTOK>>(smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, 128, smem, s>>>(a, tk, tv);
     return cudaGetLastError();

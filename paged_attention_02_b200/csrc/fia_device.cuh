@@ -8,6 +8,7 @@
 // the final barrier and release TMEM.
 #pragma once
 
+#include <atomic>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -486,6 +487,26 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t r;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
     return r;
+}
+
+// ---------------------------------------------------------------------------
+// Host-side launch helper.
+// ---------------------------------------------------------------------------
+// Dynamic shared-memory opt-in for kernel KERN, set once per device: it is a
+// per-context setting, and setting it on every run costs host time on the
+// launch path (and is best kept out of a stream capture).  One instance of
+// the flag word per kernel (KERN is a template argument).
+template <auto KERN>
+static cudaError_t ensure_smem_attr(int smem) {
+    static std::atomic<uint64_t> done{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(KERN, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+    return e;
 }
 
 // ---------------------------------------------------------------------------

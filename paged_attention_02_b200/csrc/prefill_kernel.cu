@@ -763,14 +763,14 @@ static cudaError_t launch_prefill_t(const PrefillArgs &a, const CUtensorMap &tq,
     const int smem = PrefillCfg<D, MODE>::kSmem;
     if (inline_plan) {
         auto kern = fia_prefill_kernel<T, D, MODE, kInlinePlanBytes, BAND>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaError_t e = ensure_smem_attr<fia_prefill_kernel<T, D, MODE, kInlinePlanBytes, BAND>>(smem);
         if (e != cudaSuccess) return e;
         // inline_plan points at a full PlanBytes<kInlinePlanBytes> kept by the op
         kern<<<grid, PrefillCfg<D, MODE>::kThreads, smem, s>>>(
             a, tq, tk, tv, tp, *reinterpret_cast<const PlanBytes<kInlinePlanBytes> *>(inline_plan));
     } else {
         auto kern = fia_prefill_kernel<T, D, MODE, 16, BAND>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaError_t e = ensure_smem_attr<fia_prefill_kernel<T, D, MODE, 16, BAND>>(smem);
         if (e != cudaSuccess) return e;
         PlanBytes<16> pl{};
         kern<<<grid, PrefillCfg<D, MODE>::kThreads, smem, s>>>(a, tq, tk, tv, tp, pl);

@@ -361,6 +361,35 @@ BAND_CASES = {
 }
 
 
+@pytest.mark.parametrize("band", [(255, 0), (0, 0), (-70, 200), (10 ** 6, 10 ** 6), (5, -3)])
+def test_band_decode_plan_covers_only_the_band(band):
+    """Phase 1 under a band mask splits only the keys the band can reach: per
+    sequence [kvSeqLen - seqLen - pre, kvSeqLen + next) clipped to the
+    sequence, its start rounded down to a 64-key tile (empty when the band
+    misses every key, which still gets one unit for the empty-row output)."""
+    import paged_attention_02_b200 as fia
+    kv = [4000, 100, 1300, 64, 1]
+    p = W.make_problem(seed=77, seq_len=[1, 2, 1, 3, 1], kv_seq_len=kv, head_num=16,
+                       kv_head_num=4, head_size=128, block_size=64, band=band)
+    d = lambda t: None if t is None else t.cuda().contiguous()
+    op = fia.FiaOp(d(p.query), d(p.key_cache), d(p.value_cache), d(p.block_tables),
+                   [int(x) for x in p.seq_len], kv, p.head_num, p.kv_head_num, p.qk_scale,
+                   band=band)
+    info = op.plan_info()
+    assert info["path"] == 1
+    split = info["split_tokens"]
+    assert split > 0 and split % 64 == 0
+    units = 0
+    for ql, kl in zip(p.seq_len, kv):
+        lo = max(0, kl - int(ql) - band[0])
+        hi = min(kl, kl + band[1])
+        if hi <= lo:
+            lo = hi = 0
+        lo = lo // 64 * 64
+        units += max(1, -(-(hi - lo) // split)) * p.kv_head_num
+    assert info["work_items"] == units
+
+
 @pytest.mark.parametrize("name", sorted(BAND_CASES))
 def test_band_mask(name):
     p = W.make_problem(name=name, seed=zlib.crc32(name.encode()) % 10000, spare_blocks=2,
@@ -368,3 +397,53 @@ def test_band_mask(name):
     _, out, lse = run_gpu(p)
     ref_out, ref_lse = oracle.attention(p)
     compare(out, lse, ref_out, ref_lse, name)
+
+
+# ---------------------------------------------------------------------------
+# CUDA graphs: fia_run (plan upload + kernels) captured once, replayed.
+# ---------------------------------------------------------------------------
+GRAPH_CASES = {
+    "decode": dict(seq_len=[1] * 3, kv_seq_len=[700, 33, 2000], head_num=16, kv_head_num=4,
+                   head_size=128, block_size=64),
+    "decode_int8_sink": dict(seq_len=[1, 1], kv_seq_len=[1500, 90], head_num=16, kv_head_num=2,
+                             head_size=128, block_size=128, kv_dtype="i8", sink=True),
+    "prefill_causal": dict(seq_len=[200, 64], kv_seq_len=[300, 64], head_num=8, kv_head_num=2,
+                           head_size=128, block_size=64, mask_type=W.MASK_CAUSAL),
+}
+
+
+@pytest.mark.parametrize("name", sorted(GRAPH_CASES))
+def test_cuda_graph_capture_and_replay(name):
+    """A captured fia_run replays to the eager result bitwise and reads its
+    inputs at replay time (new query values in place give the eager result on
+    the new values)."""
+    import paged_attention_02_b200 as fia
+    p = W.make_problem(name=name, seed=zlib.crc32(name.encode()) % 10000, **GRAPH_CASES[name])
+    d = lambda t: None if t is None else t.cuda().contiguous()
+    q = d(p.query)
+    op = fia.FiaOp(q, d(p.key_cache), d(p.value_cache), d(p.block_tables),
+                   [int(x) for x in p.seq_len], [int(x) for x in p.kv_seq_len], p.head_num,
+                   p.kv_head_num, p.qk_scale, mask_type=p.mask_type, sink=d(p.sink),
+                   k_scale=d(p.k_scale), k_offset=d(p.k_offset), v_scale=d(p.v_scale),
+                   v_offset=d(p.v_offset), want_lse=True)
+    out, lse = op.run()
+    torch.cuda.synchronize()
+    ref_o, ref_l = out.clone(), lse.clone()
+    out.zero_()
+    lse.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        op.run()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref_o) and torch.equal(lse, ref_l)
+    q.copy_((q.float() * 0.5 + 0.25).to(q.dtype))
+    g.replay()
+    torch.cuda.synchronize()
+    got_o, got_l = out.clone(), lse.clone()
+    assert not torch.equal(got_o, ref_o)
+    op.run()
+    torch.cuda.synchronize()
+    assert torch.equal(out, got_o) and torch.equal(lse, got_l)
+    assert op.error_word() == 0
+    del g
