@@ -58,7 +58,6 @@ struct DecodeCfg {
 };
 
 struct DecodeI8Cfg;
-int decode_smem_bytes(int D, bool kv_int8);
 
 template <typename T, int D>
 __global__ void __launch_bounds__(128, 2)
@@ -401,13 +400,6 @@ struct DecodeI8Cfg {
     static constexpr int kTokBytes = 4 * 2 * 4 * 16 * 4;
     static constexpr int kSmem = 1024 /*align slack*/ + kOffTok + kTokBytes;
 };
-
-int decode_smem_bytes(int D, bool kv_int8) {
-    if (kv_int8) return D == 128 ? DecodeI8Cfg::kSmem : -1;
-    if (D == 64) return DecodeCfg<64>::kSmem;
-    if (D == 128) return DecodeCfg<128>::kSmem;
-    return -1;
-}
 
 template <typename T, int NT, bool KTOK, bool VTOK>
 __global__ void __launch_bounds__(128, 4)

@@ -125,7 +125,5 @@ cudaError_t launch_combine(const CombineArgs &a, int q_dtype, bool kv_int8, int 
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tq, const CUtensorMap &tk,
                            const CUtensorMap &tv, const CUtensorMap &tp, int q_dtype, int grid,
                            const uint8_t *inline_plan, cudaStream_t s);
-int decode_smem_bytes(int D, bool kv_int8);
-int prefill_smem_bytes(int D);
 
 }  // namespace fia

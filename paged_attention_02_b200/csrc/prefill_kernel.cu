@@ -77,12 +77,6 @@ struct PrefillCfg {
     static constexpr int kThreads = 576;   // producer, UMMA, 2 x 8 softmax warps
 };
 
-int prefill_smem_bytes(int D) {
-    if (D == 64) return PrefillCfg<64, kModePse>::kSmem;
-    if (D == 128) return PrefillCfg<128, kModePse>::kSmem;
-    return -1;
-}
-
 struct SubGeom {
     bool valid;
     int q0, h, rows, n;
