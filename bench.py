@@ -220,35 +220,64 @@ def time_op(op, steps, warmup, flush):
 
 def time_e2e(p, steps, warmup, dev):
     """Same metric through the public API with HOST inputs: every step copies
-    the inputs host->device (pinned), runs, and copies out+lse back."""
+    all of its inputs host->device (pinned), runs, and copies out + lse back.
+    Two device buffer sets (each with its own op) and three streams let step
+    i's upload, step i-1's run and step i-2's download overlap, as a serving
+    loop would; events order the reuse of each set."""
     host = {k: (v.pin_memory() if v is not None else None) for k, v in
             dict(query=p.query, key=p.key_cache, value=p.value_cache,
                  block_tables=p.block_tables, slopes=p.slopes, pse=p.pse, sink=p.sink,
                  k_scale=p.k_scale, k_offset=p.k_offset, v_scale=p.v_scale,
                  v_offset=p.v_offset).items()}
-    devt = {k: (torch.empty_like(v, device=dev) if v is not None else None) for k, v in host.items()}
-    op = make_op(p, devt)
-    out_h = torch.empty_like(p.query).pin_memory()
-    lse_h = torch.empty((p.n_tokens, p.head_num), dtype=torch.float32).pin_memory()
+    sets = []
+    for _ in range(2):
+        devt = {k: (torch.empty_like(v, device=dev) if v is not None else None)
+                for k, v in host.items()}
+        sets.append(dict(devt=devt, op=make_op(p, devt),
+                         out_h=torch.empty_like(p.query).pin_memory(),
+                         lse_h=torch.empty((p.n_tokens, p.head_num),
+                                           dtype=torch.float32).pin_memory()))
     h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
-    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * 4
+    d2h = sets[0]["out_h"].numel() * sets[0]["out_h"].element_size() + sets[0]["lse_h"].numel() * 4
+    s_in, s_run, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    ev = {n: [torch.cuda.Event() for _ in range(2)] for n in ("in", "run", "out")}
+    for lst in ev.values():
+        for e in lst:
+            e.record(torch.cuda.current_stream(dev))
 
-    def step():
-        for k, v in host.items():
-            if v is not None:
-                devt[k].copy_(v, non_blocking=True)
-        out, lse = op.run()
-        out_h.copy_(out, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
+    def step(i):
+        k = i % 2
+        st = sets[k]
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev["run"][k])          # set k's last run has read its inputs
+            for name, v in host.items():
+                if v is not None:
+                    st["devt"][name].copy_(v, non_blocking=True)
+            ev["in"][k].record(s_in)
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(ev["in"][k])
+            s_run.wait_event(ev["out"][k])         # set k's last result has been read back
+            out, lse = st["op"].run(s_run)
+            ev["run"][k].record(s_run)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev["run"][k])
+            st["out_h"].copy_(out, non_blocking=True)
+            st["lse_h"].copy_(lse, non_blocking=True)
+            ev["out"][k].record(s_out)
 
-    for _ in range(warmup):
-        step()
+    for i in range(warmup):
+        step(i)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(steps):
-        step()
-    b.record()
+    cur = torch.cuda.current_stream(dev)
+    a.record(cur)
+    for s in (s_in, s_run, s_out):
+        s.wait_event(a)
+    for i in range(steps):
+        step(i)
+    for s in (s_in, s_run, s_out):
+        cur.wait_stream(s)
+    b.record(cur)
     torch.cuda.synchronize()
     return a.elapsed_time(b) / steps, h2d, d2h
 
