@@ -124,7 +124,7 @@ const char *fia_status_string(fia_status s) {
     case FIA_ERR_PARAM: return "a scalar parameter is out of range";
     case FIA_ERR_DTYPE: return "unsupported or mismatched dtype";
     case FIA_ERR_SHAPE: return "inconsistent tensor shapes";
-    case FIA_ERR_UNSUPPORTED: return "configuration not supported by this build";
+    case FIA_ERR_UNSUPPORTED: return "configuration not supported by this library";
     case FIA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case FIA_ERR_CUDA: return "a CUDA call failed";
     }
