@@ -66,9 +66,18 @@ def test_matches_torch_sdpa(case):
     np.testing.assert_allclose(out, ref, rtol=1e-10, atol=1e-10)
 
 
-def test_row_subset_matches_full():
+@pytest.mark.parametrize("kw", [
+    dict(mask_type=W.MASK_CAUSAL),
+    dict(band=(3, 1), sink=True),
+    dict(kv_dtype="i8", k_antiquant="token", v_antiquant="channel", sink=True),
+    dict(mask_type=W.MASK_CAUSAL, pse=True),
+    dict(kv_layout=1, mask_type=W.MASK_ALIBI, alibi_slopes=True),
+])
+def test_row_subset_matches_full(kw):
+    """The sampled-rows mode (used by the full-size GPU tests) gives exactly
+    the rows of the full computation, for every feature it is sampled with."""
     p = W.make_problem(seed=7, seq_len=[3, 5], kv_seq_len=[10, 5], head_num=4, kv_head_num=2,
-                       head_size=8, block_size=4, mask_type=W.MASK_CAUSAL)
+                       head_size=8, block_size=4, **kw)
     out, lse = oracle.attention(p)
     rows = [(0, 1), (7, 3), (4, 0)]
     so, sl = oracle.attention(p, rows=rows)
