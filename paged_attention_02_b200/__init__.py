@@ -21,7 +21,8 @@ from ._lib import (FIA_KV_BNBSH, FIA_KV_BNNBSD, FIA_MASK_ALIBI, FIA_MASK_CAUSAL,
                    FiaError, fia_ext, fia_plan_info, fia_tensor)
 
 __all__ = ["FiaOp", "fused_infer_attention", "FIA_MASK_NONE", "FIA_MASK_ALIBI",
-           "FIA_MASK_CAUSAL", "FIA_KV_BNBSH", "FIA_KV_BNNBSD", "FiaError", "tensor_desc"]
+           "FIA_MASK_CAUSAL", "FIA_KV_BNBSH", "FIA_KV_BNNBSD", "FiaError", "tensor_desc",
+           "validate_block_tables"]
 
 _DT = {torch.float16: _lib.FIA_F16, torch.bfloat16: _lib.FIA_BF16, torch.float32: _lib.FIA_F32,
        torch.int8: _lib.FIA_I8, torch.int32: _lib.FIA_I32}
@@ -48,6 +49,30 @@ def _ptr(d: Optional[fia_tensor]):
     return ctypes.pointer(d) if d is not None else None
 
 
+def validate_block_tables(block_tables, kv_seq_len: Sequence[int], block_size: int,
+                          num_blocks: int) -> None:
+    """Debug check of a block table, on the host (the kernels, like the
+    operator they implement, do not validate block ids).  Every entry a
+    sequence reads -- entries j < ceil(kvSeqLen / blockSize) of its row --
+    must name a block in [0, numBlocks); entries past that are never read and
+    may hold anything.  Copies the table to the host; raises ValueError naming
+    the first bad entry."""
+    bt = block_tables.detach().to("cpu")
+    if bt.dim() != 2 or bt.shape[0] < len(kv_seq_len):
+        raise ValueError("block table must be [batch, maxBlockNum]")
+    for b, kl in enumerate(kv_seq_len):
+        need = (int(kl) + block_size - 1) // block_size
+        if need > bt.shape[1]:
+            raise ValueError("sequence %d needs %d blocks, the table row has %d"
+                             % (b, need, bt.shape[1]))
+        row = bt[b, :need]
+        bad = ((row < 0) | (row >= num_blocks)).nonzero()
+        if bad.numel():
+            j = int(bad[0, 0])
+            raise ValueError("block_tables[%d][%d] = %d is outside [0, %d)"
+                             % (b, j, int(row[j]), num_blocks))
+
+
 class FiaOp:
     """One planned call (phase 1 done); ``run()`` enqueues phase 2.
 
@@ -62,7 +87,8 @@ class FiaOp:
     ``[batch, maxBlockNum]`` int32 (all on the same CUDA device), host
     sequence lengths.  ``out`` / ``lse`` are allocated when not given
     (``want_lse=False`` skips lse).  Tensors are referenced, not copied: keep
-    them unchanged while runs are in flight.
+    them unchanged while runs are in flight.  ``check_block_tables=True``
+    runs ``validate_block_tables`` on the table first (a host copy: debugging only).
     """
 
     def __init__(self, query, key, value, block_tables, seq_len: Sequence[int],
@@ -71,8 +97,12 @@ class FiaOp:
                  k_offset=None, v_scale=None, v_offset=None, out=None, lse=None,
                  want_lse: bool = True, kv_layout: int = FIA_KV_BNBSH,
                  k_antiquant_mode: int = 0, v_antiquant_mode: int = 0,
-                 band: Optional[Tuple[int, int]] = None):
+                 band: Optional[Tuple[int, int]] = None, check_block_tables: bool = False):
         dev = query.device
+        if check_block_tables:
+            bnnbsd = int(kv_layout) == FIA_KV_BNNBSD
+            validate_block_tables(block_tables, kv_seq_len,
+                                  int(key.shape[2] if bnnbsd else key.shape[1]), int(key.shape[0]))
         self.out = out if out is not None else torch.empty_like(query)
         if lse is None and want_lse:
             lse = torch.empty((query.shape[0], head_num), dtype=torch.float32, device=dev)

@@ -17,6 +17,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -30,6 +31,17 @@
 #include "../../include/fia.h"
 #include "fia_device.cuh"
 #include "fia_plan.h"
+
+namespace {
+// NVTX range over one API call (a no-op unless a profiler is attached), so a
+// timeline shows planning and each run's launches by name.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
+}  // namespace
 
 using namespace fia;
 
@@ -137,6 +149,7 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
                                   const fia_tensor *slopes, int32_t maskType, int32_t headNum,
                                   int32_t kvHeadNum, float qkScale, const fia_ext *ext,
                                   fia_tensor *attnOut, uint64_t *workspaceSize, fia_op **op) {
+    NvtxRange range("fia_get_workspace_size");
     if (!workspaceSize || !op) return FIA_ERR_NULLPTR;
     *workspaceSize = 0;
     *op = nullptr;
@@ -614,6 +627,7 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
 fia_status fia_run(void *workspace, uint64_t workspaceSize, fia_op *op, void *stream_ptr) {
     if (!op) return FIA_ERR_NULLPTR;
     if (op->path == 0) return FIA_OK;
+    NvtxRange range(op->path == 1 ? "fia_run decode" : "fia_run prefill");
     if (!workspace || workspaceSize < op->ws_size ||
         (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return FIA_ERR_WORKSPACE;
