@@ -204,12 +204,13 @@ def fused_infer_attention(query, key, value, block_tables, seq_len, kv_seq_len, 
                           kv_head_num, qk_scale, mask_type=FIA_MASK_NONE, slopes=None, pse=None,
                           sink=None, k_scale=None, k_offset=None, v_scale=None, v_offset=None,
                           want_lse=True, kv_layout=FIA_KV_BNBSH, k_antiquant_mode=0,
-                          v_antiquant_mode=0, band=None):
+                          v_antiquant_mode=0, band=None, check_block_tables=False):
     """One-shot call: plan, run on the current stream, return (out, lse)."""
     op = FiaOp(query, key, value, block_tables, seq_len, kv_seq_len, head_num, kv_head_num,
                qk_scale, mask_type, slopes, pse, sink, k_scale, k_offset, v_scale, v_offset,
                want_lse=want_lse, kv_layout=kv_layout, k_antiquant_mode=k_antiquant_mode,
-               v_antiquant_mode=v_antiquant_mode, band=band)
+               v_antiquant_mode=v_antiquant_mode, band=band,
+               check_block_tables=check_block_tables)
     out, lse = op.run()
     op._keep.append(op.workspace)
     return out, lse
