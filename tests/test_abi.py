@@ -63,9 +63,12 @@ def _call(**kw):
     ext = fia_ext(P(d["pse"]), P(d["sink"]), P(d["ks"]), None, P(d["vs"]), None, P(d["lse"]),
                   int(args.get("layout", 0)), int(args.get("kmode", 0)), int(args.get("vmode", 0)),
                   int(args.get("sparse", 0)), int(args.get("pre", 0)), int(args.get("next", 0)))
-    n = max(len(args["seq"]), 1)
-    sl = (ctypes.c_int32 * n)(*args["seq"])
-    kl = (ctypes.c_int32 * n)(*args["kv"])
+    if args["seq"] is None:                       # NULL host length arrays
+        sl = kl = None
+    else:
+        n = max(len(args["seq"]), 1)
+        sl = (ctypes.c_int32 * n)(*args["seq"])
+        kl = (ctypes.c_int32 * n)(*args["kv"])
     ws = ctypes.c_uint64(123)
     op = ctypes.c_void_p()
     st = _lib.fia_get_workspace_size(P(d["q"]), P(d["k"]), P(d["v"]), P(d["bt"]), sl, kl,
@@ -96,6 +99,52 @@ def test_phase1_rejects_bad_inputs():
     assert _call(pse=torch.zeros(2, 4, 2, 16, dtype=torch.bfloat16)) == L.FIA_ERR_SHAPE
     assert _call(scale=float("nan")) == L.FIA_ERR_PARAM
     assert _call(batch=-1) == L.FIA_ERR_PARAM
+
+
+def test_phase1_rejects_more_bad_inputs():
+    """The remaining phase-1 rejection rules (each case breaks exactly one)."""
+    from paged_attention_02_b200 import _lib as L
+    bf = lambda *sh: torch.zeros(*sh, dtype=torch.bfloat16)
+    ok = (L.FIA_ERR_CUDA, L.FIA_OK)               # valid: no GPU here, phase 1 stops at encoding
+    # null pointers
+    assert L.fia_get_workspace_size(None, None, None, None, None, None, 0, None, 0, 0, 0, 0.0,
+                                    None, None, None, None) == L.FIA_ERR_NULLPTR
+    assert _call(q=None) == L.FIA_ERR_NULLPTR
+    assert _call(bt=None) == L.FIA_ERR_NULLPTR
+    assert _call(out=None) == L.FIA_ERR_NULLPTR
+    assert _call(seq=None) == L.FIA_ERR_NULLPTR                                   # batch 2, no lengths
+    # head counts
+    assert _call(H=0) == L.FIA_ERR_PARAM
+    assert _call(KVH=0) == L.FIA_ERR_PARAM
+    assert _call(H=2048, KVH=2, q=bf(3, 2048, 128), out=bf(3, 2048, 128)) == L.FIA_ERR_PARAM
+    # query / output shapes; the 2-D query form [nTokens, H * D] is accepted
+    assert _call(q=bf(3, 4, 128, 1), out=bf(3, 4, 128, 1)) == L.FIA_ERR_SHAPE
+    assert _call(q=bf(3, 5, 128), out=bf(3, 5, 128)) == L.FIA_ERR_SHAPE
+    assert _call(q=bf(3, 512), out=bf(3, 512)) in ok
+    assert _call(q=bf(3, 510), out=bf(3, 510)) == L.FIA_ERR_SHAPE
+    assert _call(out=bf(3, 4, 64)) == L.FIA_ERR_SHAPE
+    # cache shapes: the 3-D BnBsH form [numBlocks, blockSize, kvHeadNum * D] is accepted
+    assert _call(k=bf(8, 16, 256), v=bf(8, 16, 256)) in ok
+    assert _call(k=bf(8, 16, 250), v=bf(8, 16, 250)) == L.FIA_ERR_SHAPE
+    assert _call(k=bf(8, 4096), v=bf(8, 4096)) == L.FIA_ERR_SHAPE                  # 2-D cache
+    assert _call(v=bf(8, 16, 256)) == L.FIA_ERR_SHAPE                             # k 4-D, v 3-D
+    # block table
+    assert _call(bt=torch.zeros(8, dtype=torch.int32)) == L.FIA_ERR_SHAPE
+    assert _call(bt=torch.zeros(3, 4, dtype=torch.int32)) == L.FIA_ERR_SHAPE     # 3 rows, batch 2
+    # lengths
+    assert _call(seq=[-1, 4]) == L.FIA_ERR_PARAM
+    assert _call(kv=[-1, 33]) == L.FIA_ERR_PARAM
+    # pse
+    assert _call(pse=torch.zeros(2, 4, 2, 40, dtype=torch.float16)) == L.FIA_ERR_DTYPE
+    assert _call(pse=bf(2, 4, 2, 40)) in ok
+    assert _call(pse=bf(2, 4, 1, 40)) == L.FIA_ERR_SHAPE                          # maxQ is 2
+    assert _call(mask=3, slopes=torch.zeros(4), pse=bf(2, 4, 2, 40)) == L.FIA_ERR_PARAM
+    # sink / lse / slopes dtypes and shapes
+    assert _call(sink=torch.zeros(4, dtype=torch.float16)) == L.FIA_ERR_DTYPE
+    assert _call(sink=torch.zeros(4)) in ok
+    assert _call(mask=3, slopes=torch.zeros(3)) == L.FIA_ERR_SHAPE
+    assert _call(lse=torch.zeros(3, 5)) == L.FIA_ERR_SHAPE
+    assert _call(lse=torch.zeros(3, 4)) in ok
 
 
 def test_phase1_int8_rules():
