@@ -447,3 +447,30 @@ def test_cuda_graph_capture_and_replay(name):
     assert torch.equal(out, got_o) and torch.equal(lse, got_l)
     assert op.error_word() == 0
     del g
+
+
+@pytest.mark.parametrize("kind", ["decode", "prefill"])
+def test_flat_query_and_cache_forms_are_bitwise_equal(kind):
+    """The 2-D query form [nTokens, H * D] and the 3-D cache form
+    [numBlocks, blockSize, kvHeadNum * D] (same memory) give the same result
+    as the 4-D forms, bit for bit."""
+    import paged_attention_02_b200 as fia
+    cfg = dict(decode=dict(seq_len=[1, 2], kv_seq_len=[300, 77], mask_type=W.MASK_CAUSAL),
+               prefill=dict(seq_len=[150, 40], kv_seq_len=[400, 40],
+                            mask_type=W.MASK_CAUSAL))[kind]
+    p = W.make_problem(seed=91, head_num=8, kv_head_num=2, head_size=128, block_size=32, **cfg)
+    _, ref, ref_lse = run_gpu(p)
+    q = p.query.cuda().contiguous()
+    k = p.key_cache.cuda().contiguous()
+    v = p.value_cache.cuda().contiguous()
+    n, h, d = q.shape
+    nb, bs, kvh, _ = k.shape
+    op = fia.FiaOp(q.view(n, h * d), k.view(nb, bs, kvh * d), v.view(nb, bs, kvh * d),
+                   p.block_tables.cuda().contiguous(), [int(x) for x in p.seq_len],
+                   [int(x) for x in p.kv_seq_len], p.head_num, p.kv_head_num, p.qk_scale,
+                   mask_type=p.mask_type)
+    out, lse = op.run()
+    torch.cuda.synchronize()
+    assert op.error_word() == 0
+    assert np.array_equal(out.view(n, h, d).float().double().cpu().numpy(), ref)
+    assert np.array_equal(lse.double().cpu().numpy(), ref_lse)
