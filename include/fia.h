@@ -33,9 +33,13 @@
  *    needs a CUDA device (it returns FIA_ERR_CUDA without one).
  *  - fia_run is asynchronous on `stream`, allocates nothing and does not
  *    synchronise.  It may be called any number of times on the same op.
- *  - Block ids in blockTables are not validated on the device (the pages say
- *    the same: "the validity of block IDs is not verified").  Entries past
- *    ceil(kvSeqLen[b] / blockSize) are never read.
+ *  - Block ids in blockTables are not validated on the device; the V3 page's
+ *    paged-attention constraints leave that check to the caller as well.
+ *    Entries past ceil(kvSeqLen[b] / blockSize) are never read.
+ *  - An op belongs to the device that was current when phase 1 ran (its
+ *    pointers and TMA descriptors refer to that device's memory).  Every call
+ *    that launches work checks that the same device is current and returns
+ *    FIA_ERR_PARAM otherwise.
  *  - Errors are returned as fia_status; nothing is printed and nothing aborts.
  */
 #ifndef FIA_H
@@ -152,8 +156,8 @@ typedef struct {
 typedef struct fia_op fia_op;
 
 /*
- * Phase 1 (ATB AtbSelfAttentionPrefixEncoderGetWorkspaceSize; aclnn
- * ...GetWorkspaceSize "implements input parameter verification").
+ * Phase 1 (ATB AtbSelfAttentionPrefixEncoderGetWorkspaceSize; the aclnn
+ * ...GetWorkspaceSize call, the phase in which the V4/V3 pages check the inputs).
  *
  *  query        [nTokens, headNum, headSize] or [nTokens, headNum*headSize], f16|bf16.
  *               The new tokens of all sequences, concatenated in batch order.
@@ -174,7 +178,7 @@ typedef struct fia_op fia_op;
  *  headNum      > 0;  kvHeadNum > 0 and headNum % kvHeadNum == 0; query head h
  *               reads KV head h / (headNum / kvHeadNum).
  *  qkScale      multiplies Q K^T before the bias is added (PrefixEncoder
- *               "post-multiplied by Q*K^T").
+ *               parameter table, qkScale row: the scale applies to the product).
  *  ext          optional extensions (see fia_ext), may be NULL.
  *  attnOut      [nTokens, headNum, headSize] (or 2-D), the query's dtype.
  *  workspaceSize  out: bytes of device workspace fia_run needs (0 if none).
@@ -198,8 +202,9 @@ FIA_API fia_status fia_get_workspace_size(const fia_tensor *query, const fia_ten
  *                 (may be NULL only when workspaceSize was 0).  Its contents
  *                 are scratch: fia_run overwrites them.
  *  stream         a cudaStream_t (0 = legacy default stream), passed as void*.
- * Returns FIA_ERR_WORKSPACE for a NULL/misaligned/too-small workspace and
- * FIA_ERR_CUDA when a copy or launch fails (the op stays usable).
+ * Returns FIA_ERR_WORKSPACE for a NULL/misaligned/too-small workspace,
+ * FIA_ERR_PARAM when the current device is not the op's, and FIA_ERR_CUDA when
+ * a copy or launch fails (the op stays usable).
  */
 FIA_API fia_status fia_run(void *workspace, uint64_t workspaceSize, fia_op *op, void *stream);
 
@@ -241,6 +246,23 @@ typedef struct {
 FIA_API fia_status fia_op_get_plan_info(const fia_op *op, fia_plan_info *info);
 
 /*
+ * Failure detection (V3 long-sequence restriction: an over-long run ends in a
+ * device time-out error; here every internal wait of the kernels is bounded
+ * instead).  Each wait on an on-chip barrier gives up after a time limit
+ * (default 2 s); the kernel then sets the error word (error_word_offset above;
+ * bits 8.. name the wait site, bit 0 = time-out), records up to 31 trail
+ * entries after it, lets every role of the CTA leave, waits for its copies and
+ * MMAs still in flight, releases its resources and returns.  The run's output
+ * is then undefined, and the device stays usable.
+ *   wait_limit_ns  new limit for this op's runs (0 restores the default).
+ *   stall          test hook, 0 or 1: with 1, one role of every CTA first waits
+ *                  on a barrier that nothing signals, so that the time-out path
+ *                  runs and its report can be checked.  Never set it in service.
+ * FIA_ERR_NULLPTR for a NULL op, FIA_ERR_PARAM for another stall value.
+ */
+FIA_API fia_status fia_op_set_wait_limit(fia_op *op, uint64_t wait_limit_ns, int32_t stall);
+
+/*
  * Decode without a caller workspace (no counterpart in the pages: the aclnn and
  * ATB interfaces always take a caller-allocated workspace).
  *
@@ -258,16 +280,31 @@ FIA_API fia_status fia_op_get_plan_info(const fia_op *op, fia_plan_info *info);
  *  - An op whose workspaceSize exceeds it gets FIA_ERR_WORKSPACE; a prefill op
  *    gets FIA_ERR_UNSUPPORTED; a no-op op returns FIA_OK.  Nothing is launched
  *    in those cases.
- *  - Call it with the op's device current.  The first call on a device looks up
- *    the array's device address (cudaGetSymbolAddress); make that first call
- *    before any stream capture.  A failed lookup returns FIA_ERR_CUDA.
+ *  - Call it with the op's device current (FIA_ERR_PARAM otherwise).  The first
+ *    call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *    A failed lookup returns FIA_ERR_CUDA.
  *  - All calls on a device share the one array, which keeps the last call's
  *    contents.  Calls that overlap on the GPU (two streams, or two host threads
  *    without ordering) race on it: serialise them.
  *  - Asynchronous on `stream` (a cudaStream_t passed as void*), like fia_run.
+ *    Timing events set with fia_op_set_timing_events are recorded around its
+ *    kernels as for fia_run.
+ *  - The kernels' error word (see fia_op_set_wait_limit) lives in the array:
+ *    read it with fia_decode_static_error_word.
  */
 #define FIA_STATIC_WORKSPACE_BYTES (32u * 1024u * 1024u)
 FIA_API fia_status fia_decode_run_static(fia_op *op, void *stream);
+
+/*
+ * The error word of the last fia_decode_run_static call of this op's shape on
+ * the op's device (0 = every internal wait completed).  Copies 4 bytes out of
+ * the library's array with cudaMemcpyFromSymbol, which waits for the device
+ * to finish its queued work.  *word is 0 for a no-op op.  FIA_ERR_UNSUPPORTED
+ * for a prefill op, FIA_ERR_PARAM when another device is current,
+ * FIA_ERR_CUDA when the copy fails.
+ */
+FIA_API fia_status fia_decode_static_error_word(const fia_op *op, uint32_t *word);
 
 #ifdef __cplusplus
 }

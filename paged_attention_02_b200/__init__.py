@@ -174,6 +174,14 @@ class FiaOp:
                             bar=(r[7] << 32) | r[6]))
         return out
 
+    def set_wait_limit(self, wait_limit_ns: int = 0, stall: bool = False):
+        """Bound every internal wait of this op's kernels by ``wait_limit_ns``
+        (0: the 2 s default).  ``stall=True`` is a test hook that makes the
+        kernels time out on purpose (see fia_op_set_wait_limit in fia.h)."""
+        st = _lib.fia_op_set_wait_limit(self._op, int(wait_limit_ns), 1 if stall else 0)
+        if st != _lib.FIA_OK:
+            raise FiaError(st, "fia_op_set_wait_limit")
+
     def set_timing_events(self, start: Optional[torch.cuda.Event], stop: Optional[torch.cuda.Event]):
         """Have run() record ``start``/``stop`` around its kernels only."""
         if start is None:

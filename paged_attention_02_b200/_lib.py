@@ -80,6 +80,10 @@ def _load():
     lib.fia_op_get_plan_info.restype = ctypes.c_int
     lib.fia_decode_run_static.argtypes = [P, P]
     lib.fia_decode_run_static.restype = ctypes.c_int
+    lib.fia_decode_static_error_word.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
+    lib.fia_decode_static_error_word.restype = ctypes.c_int
+    lib.fia_op_set_wait_limit.argtypes = [P, ctypes.c_uint64, ctypes.c_int32]
+    lib.fia_op_set_wait_limit.restype = ctypes.c_int
     return lib
 
 
@@ -115,6 +119,10 @@ def fia_op_get_plan_info(op, info) -> int:
     return _lib.fia_op_get_plan_info(op, info)
 
 
+def fia_op_set_wait_limit(op, wait_limit_ns, stall) -> int:
+    return _lib.fia_op_set_wait_limit(op, wait_limit_ns, stall)
+
+
 FIA_STATIC_WORKSPACE_BYTES = 32 * 1024 * 1024
 
 
@@ -122,3 +130,9 @@ def fia_decode_run_static(op, stream) -> int:
     """Decode-path run with the library's fixed scratch array (no workspace
     argument, no allocation); see include/fia.h."""
     return _lib.fia_decode_run_static(op, stream)
+
+
+def fia_decode_static_error_word(op, word) -> int:
+    """Error word of the last fia_decode_run_static call on the op's device
+    (a synchronous 4-byte copy)."""
+    return _lib.fia_decode_static_error_word(op, word)

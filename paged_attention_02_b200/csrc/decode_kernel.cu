@@ -53,7 +53,9 @@ struct DecodeCfg {
     static constexpr int kMergeBytes = 4 * kDecodeRows * D * 4 + 4 * kDecodeRows * 8;
     static constexpr int kDataBytes =
         (kStages * kStageBytes > kMergeBytes) ? kStages * kStageBytes : kMergeBytes;
-    static constexpr int kSmem = 1024 /*align slack*/ + kDataBytes + 2 * kStages * 8 + 16;
+    // full[S], empty[S], one barrier nothing signals (test hook), abort flag
+    static constexpr int kBarBytes = ((2 * kStages + 1) * 8 + 4 + 15) & ~15;
+    static constexpr int kSmem = 1024 /*align slack*/ + kDataBytes + kBarBytes;
     static_assert(kRowBytes % 128 == 0, "row must be a whole number of 128-byte groups");
 };
 
@@ -73,7 +75,8 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
                                                 ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + Cfg::kDataBytes);
     uint64_t *empty = full + STAGES;
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + STAGES);
+    uint64_t *never = empty + STAGES;       // test hook: nothing arrives on it
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(never + 1);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -92,6 +95,7 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 4);
         }
+        mbar_init(never, 1);
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tk);
@@ -121,8 +125,21 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
             }
         }
     };
+    int n_issued = 0;      // tiles requested (thread 0)
     if (tid == 0) {
         for (int j = 0; j < STAGES && j < n_tiles; ++j) issue(j);
+        n_issued = min(STAGES, n_tiles);
+    }
+    // Test hook: every warp first waits on a barrier nothing signals; the
+    // bounded wait gives up, and the CTA takes the error exit below with its
+    // first tiles' copies still in flight.
+    int n_run = n_tiles;
+    if (a.c.stall) {
+        const bool got = mbar_wait(never, 0, abort_flag, a.c.err, 3, a.c.wait_ns);
+        if (!__all_sync(0xffffffffu, got)) {
+            if (lane == 0) fail_trail(a.c.err, 3, (uint32_t)u.b, (uint32_t)u.kvh, 0u, never);
+            n_run = 0;
+        }
     }
 
     // ---- per-row constants and the Q operand (rows ra = r, rb = r + 8) ----
@@ -165,10 +182,11 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
     for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
 
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
+    for (int j = 0; j < n_run; ++j) {
         const int s = j % STAGES;
         // every lane waits; the warp leaves together if any lane gave up
-        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (j / STAGES) & 1, abort_flag, a.c.err, 1))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (j / STAGES) & 1, abort_flag, a.c.err, 1,
+                                               a.c.wait_ns))) {
             ok = false;
             break;
         }
@@ -313,8 +331,12 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
         if (lane == 0) mbar_arrive(&empty[s]);
         bool stop = false;
         if (tid == 0 && j + STAGES < n_tiles) {
-            if (mbar_wait(&empty[s], (j / STAGES) & 1, abort_flag, a.c.err, 2)) issue(j + STAGES);
-            else stop = true;
+            if (mbar_wait(&empty[s], (j / STAGES) & 1, abort_flag, a.c.err, 2, a.c.wait_ns)) {
+                issue(j + STAGES);
+                ++n_issued;
+            } else {
+                stop = true;
+            }
         }
         __syncwarp();
         // a failed wait ends the key loop for the whole warp at once (lane 0
@@ -330,6 +352,16 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
         l_b += __shfl_xor_sync(0xffffffffu, l_b, x);
     }
     __syncthreads();   // every warp is done with the stage buffers
+    // Error exit (the flag is final here: no wait follows): the copies of the
+    // last STAGES requested tiles may still be in flight; wait for them before
+    // the buffers are reused below and before the CTA ends.  Earlier tiles'
+    // copies completed before their stage was requested again.
+    if (*abort_flag) {
+        if (tid == 0)
+            for (int j = max(0, n_issued - STAGES); j < n_issued; ++j)
+                mbar_wait_drain(&full[j % STAGES], (j / STAGES) & 1);
+        __syncthreads();
+    }
     float *ow = reinterpret_cast<float *>(smem);                          // [4][16][D]
     float2 *mlw = reinterpret_cast<float2 *>(smem + 4 * kDecodeRows * D * 4);  // [4][16]
     float *oww = ow + warp * kDecodeRows * D;
@@ -394,9 +426,11 @@ struct DecodeI8Cfg {
     static constexpr int kMergeBytes = 4 * kDecodeRows * D * 4 + 4 * kDecodeRows * 8;
     static constexpr int kDataBytes =
         (kStages * kStageBytes > kMergeBytes) ? kStages * kStageBytes : kMergeBytes;
+    // full[S], empty[S], one barrier nothing signals (test hook), abort flag
+    static constexpr int kBarBytes = ((2 * kStages + 1) * 8 + 4 + 15) & ~15;
     // per-token dequantisation parameters, per warp: [2 buffers][4 arrays:
     // K scale, K offset, V scale, V offset][16 keys] fp32, after the barriers
-    static constexpr int kOffTok = kDataBytes + 2 * kStages * 8 + 16;
+    static constexpr int kOffTok = kDataBytes + kBarBytes;
     static constexpr int kTokBytes = 4 * 2 * 4 * 16 * 4;
     static constexpr int kSmem = 1024 /*align slack*/ + kOffTok + kTokBytes;
 };
@@ -418,7 +452,8 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
                                                 ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + Cfg::kDataBytes);
     uint64_t *empty = full + STAGES;
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + STAGES);
+    uint64_t *never = empty + STAGES;       // test hook: nothing arrives on it
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(never + 1);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -437,6 +472,7 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 4);
         }
+        mbar_init(never, 1);
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tk);
@@ -462,8 +498,21 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
             tma_load_3d(vst + bi * br * 128, &tv, &full[s], 0, y, z);
         }
     };
+    int n_issued = 0;      // tiles requested (thread 0)
     if (tid == 0) {
         for (int j = 0; j < STAGES && j < n_tiles; ++j) issue(j);
+        n_issued = min(STAGES, n_tiles);
+    }
+    // Test hook: every warp first waits on a barrier nothing signals; the
+    // bounded wait gives up, and the CTA takes the error exit below with its
+    // first tiles' copies still in flight.
+    int n_run = n_tiles;
+    if (a.c.stall) {
+        const bool got = mbar_wait(never, 0, abort_flag, a.c.err, 3, a.c.wait_ns);
+        if (!__all_sync(0xffffffffu, got)) {
+            if (lane == 0) fail_trail(a.c.err, 3, (uint32_t)u.b, (uint32_t)u.kvh, 0u, never);
+            n_run = 0;
+        }
     }
 
     // ---- Q'^T fragments: this thread holds query row nb = 8nt + r ----
@@ -600,10 +649,11 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
     const uint32_t ones4[4] = {ones, ones, ones, ones};
 
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
+    for (int j = 0; j < n_run; ++j) {
         const int s = j % STAGES;
         // every lane waits; the warp leaves together if any lane gave up
-        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (j / STAGES) & 1, abort_flag, a.c.err, 1))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (j / STAGES) & 1, abort_flag, a.c.err, 1,
+                                               a.c.wait_ns))) {
             ok = false;
             break;
         }
@@ -812,8 +862,12 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
         if (lane == 0) mbar_arrive(&empty[s]);
         bool stop = false;
         if (tid == 0 && j + STAGES < n_tiles) {
-            if (mbar_wait(&empty[s], (j / STAGES) & 1, abort_flag, a.c.err, 2)) issue(j + STAGES);
-            else stop = true;
+            if (mbar_wait(&empty[s], (j / STAGES) & 1, abort_flag, a.c.err, 2, a.c.wait_ns)) {
+                issue(j + STAGES);
+                ++n_issued;
+            } else {
+                stop = true;
+            }
         }
         __syncwarp();
         // a failed wait ends the key loop for the whole warp at once (lane 0
@@ -836,6 +890,16 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
             }
         }
     __syncthreads();   // every warp is done with the stage buffers
+    // Error exit (the flag is final here: no wait follows): the copies of the
+    // last STAGES requested tiles may still be in flight; wait for them before
+    // the buffers are reused below and before the CTA ends.  Earlier tiles'
+    // copies completed before their stage was requested again.
+    if (*abort_flag) {
+        if (tid == 0)
+            for (int j = max(0, n_issued - STAGES); j < n_issued; ++j)
+                mbar_wait_drain(&full[j % STAGES], (j / STAGES) & 1);
+        __syncthreads();
+    }
     float *ow = reinterpret_cast<float *>(smem);                               // [4][16][D]
     float2 *mlw = reinterpret_cast<float2 *>(smem + 4 * kDecodeRows * D * 4);  // [4][16]
     float *oww = ow + warp * kDecodeRows * D;

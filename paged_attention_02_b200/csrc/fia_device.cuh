@@ -22,7 +22,10 @@ enum : uint32_t {
     kErrWaitTimeout = 1,
 };
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per wait
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per wait (the default limit)
+// After a role has given up, each copy or MMA still in flight is waited for
+// (up to this long) before the CTA releases its shared memory and TMEM.
+constexpr uint64_t kDrainLimitNs = 100000000ull;   // 100 ms
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
@@ -79,21 +82,33 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
 
 // Waits for the phase of `bar` with parity `parity` to complete.  Returns
 // false (after recording the error and raising `abort`) when the wait runs
-// past kWaitLimitNs, or when another role has already raised `abort`.
+// past `limit_ns`, or when another role has already raised `abort`.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          uint32_t *err, uint32_t where) {
+                                          uint32_t *err, uint32_t where, uint64_t limit_ns) {
     if (mbar_test_wait(bar, parity)) return true;
     uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 63u) == 63u) {
             if (*abort) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 *abort = 1;
                 if (err) atomicCAS(err, 0u, (where << 8) | kErrWaitTimeout);
                 return false;
             }
         }
+    }
+}
+
+// Error exit only: waits (up to kDrainLimitNs, ignoring `abort`) for the
+// phase of `bar` with parity `parity`, i.e. for the copies or MMAs that will
+// complete it, so that none of them still writes into shared memory or TMEM
+// after the CTA has released them.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 63u && globaltimer_ns() - t0 > kDrainLimitNs) return false;
     }
 }
 

@@ -47,6 +47,7 @@ using namespace fia;
 
 struct fia_op {
     int32_t path = 0;          // 0 no-op, 1 decode, 2 prefill
+    int32_t device = -1;       // the device current at phase 1 (runs must use it)
     int32_t q_dtype = 0;       // 0 f16, 1 bf16
     bool kv_int8 = false;
     CUtensorMap tq{}, tk{}, tv{}, tp{};
@@ -80,6 +81,18 @@ int64_t numel(const fia_tensor *t) {
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// FIA_OK when the current device is the one the op was planned on (its TMA
+// descriptors and pointers belong to that device), FIA_ERR_PARAM when another
+// device is current, FIA_ERR_CUDA when the query fails.
+fia_status check_device(const fia_op *op) {
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) {
+        cudaGetLastError();
+        return FIA_ERR_CUDA;
+    }
+    return cur == op->device ? FIA_OK : FIA_ERR_PARAM;
+}
 
 int gcd_int(int a, int b) { return b == 0 ? a : gcd_int(b, a % b); }
 
@@ -370,6 +383,9 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
     c.next = (int32_t)std::max<int64_t>(-(max_kv + 1), std::min<int64_t>(next_tok, max_kv + 1));
     c.mask_type = maskType;
     c.scale_log2 = qkScale * 1.4426950408889634f;
+    c.wait_ns = kWaitLimitNs;
+    c.stall = 0;
+    o->device = dev;
     if (kv_int8) {
         o->k_mode = k_mode;
         o->v_mode = v_mode;
@@ -631,6 +647,8 @@ fia_status fia_run(void *workspace, uint64_t workspaceSize, fia_op *op, void *st
     if (!workspace || workspaceSize < op->ws_size ||
         (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return FIA_ERR_WORKSPACE;
+    const fia_status dst = check_device(op);
+    if (dst != FIA_OK) return dst;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_ptr);
     uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
     if (!op->inline_plan &&
@@ -718,11 +736,11 @@ fia_status fia_decode_run_static(fia_op *op, void *stream_ptr) {
     if (op->path == 0) return FIA_OK;
     if (op->path != 1) return FIA_ERR_UNSUPPORTED;
     if (op->ws_size > FIA_STATIC_WORKSPACE_BYTES) return FIA_ERR_WORKSPACE;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxStaticDevices) {
-        cudaGetLastError();
-        return FIA_ERR_CUDA;
-    }
+    NvtxRange range("fia_decode_run_static");
+    const fia_status dst = check_device(op);
+    if (dst != FIA_OK) return dst;
+    const int dev = op->device;
+    if (dev < 0 || dev >= kMaxStaticDevices) return FIA_ERR_UNSUPPORTED;
     uint8_t *ws = nullptr;
     {
         std::lock_guard<std::mutex> lock(g_static_mu);
@@ -761,6 +779,10 @@ fia_status fia_decode_run_static(fia_op *op, void *stream_ptr) {
     d.v_mode = op->v_mode;
     d.n_units = op->grid;
     d.max_rows = op->max_rows;
+    if (op->ev_start && cudaEventRecord(op->ev_start, s) != cudaSuccess) {
+        cudaGetLastError();
+        return FIA_ERR_CUDA;
+    }
     cudaError_t e = cudaSuccess;
     if (op->grid > 0) e = launch_decode(d, op->tk, op->tv, op->q_dtype, op->kv_int8, op->grid, s);
     if (e == cudaSuccess && op->grid2 > 0) {
@@ -779,6 +801,25 @@ fia_status fia_decode_run_static(fia_op *op, void *stream_ptr) {
         cudaGetLastError();
         return FIA_ERR_CUDA;
     }
+    if (op->ev_stop && cudaEventRecord(op->ev_stop, s) != cudaSuccess) {
+        cudaGetLastError();
+        return FIA_ERR_CUDA;
+    }
+    return FIA_OK;
+}
+
+fia_status fia_decode_static_error_word(const fia_op *op, uint32_t *word) {
+    if (!op || !word) return FIA_ERR_NULLPTR;
+    *word = 0;
+    if (op->path == 0) return FIA_OK;
+    if (op->path != 1) return FIA_ERR_UNSUPPORTED;
+    const fia_status dst = check_device(op);
+    if (dst != FIA_OK) return dst;
+    if (cudaMemcpyFromSymbol(word, g_fia_static_ws, sizeof(uint32_t), op->off_err,
+                             cudaMemcpyDeviceToHost) != cudaSuccess) {
+        cudaGetLastError();
+        return FIA_ERR_CUDA;
+    }
     return FIA_OK;
 }
 
@@ -794,6 +835,14 @@ fia_status fia_op_set_timing_events(fia_op *op, void *start, void *stop) {
     if ((start == nullptr) != (stop == nullptr)) return FIA_ERR_PARAM;
     op->ev_start = reinterpret_cast<cudaEvent_t>(start);
     op->ev_stop = reinterpret_cast<cudaEvent_t>(stop);
+    return FIA_OK;
+}
+
+fia_status fia_op_set_wait_limit(fia_op *op, uint64_t wait_limit_ns, int32_t stall) {
+    if (!op) return FIA_ERR_NULLPTR;
+    if (stall != 0 && stall != 1) return FIA_ERR_PARAM;
+    op->common.wait_ns = wait_limit_ns ? wait_limit_ns : kWaitLimitNs;
+    op->common.stall = stall;
     return FIA_OK;
 }
 

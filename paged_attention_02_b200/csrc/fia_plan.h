@@ -61,6 +61,11 @@ struct CommonArgs {
     int32_t band;           // band mask: keys qpos - pre .. qpos + next
     int32_t pre, next;      // band limits (clamped to +-2^30)
     float scale_log2;       // qkScale * log2(e)
+    // Failure detection: every bounded wait gives up after wait_ns.  With
+    // stall set (a test hook), one role first waits on a barrier that nothing
+    // signals, so the time-out exit runs and reports through the error word.
+    uint64_t wait_ns;
+    int32_t stall;
 };
 
 // TMA coordinates (y, z) of cache row `off` of block `blk`, KV head kvh, in

@@ -66,8 +66,9 @@ struct PrefillCfg {
     static constexpr int kPseBytes = (MODE == kModePse) ? 16 * 4096 : 0;
     static constexpr int kOffBar = kOffPse + kPseBytes;
     // q_full, q_empty, k_full/k_empty[KS], v_full/v_empty[VS],
-    // s_full[2], p_full[2], pv_done[2], o_full[2], pse_full[16], vz_full
-    static constexpr int kNumBar = 2 + 2 * kKStages + 2 * kVStages + 8 + 16 + 1;
+    // s_full[2], p_full[2], pv_done[2], o_full[2], pse_full[16], vz_full,
+    // mma_drain (error exit), never (test hook: nothing arrives on it)
+    static constexpr int kNumBar = 2 + 2 * kKStages + 2 * kVStages + 8 + 16 + 1 + 2;
     static constexpr int kUsed = kOffBar + kNumBar * 8 + 16;
     // Keep one CTA per SM (each CTA holds all 512 TMEM columns).
     static constexpr int kSmem = 1024 + (kUsed > 118 * 1024 ? kUsed : 118 * 1024);
@@ -119,13 +120,29 @@ __device__ __forceinline__ PairGeom pair_geom(const PrefillArgs &a, const Prefil
     return g;
 }
 
-// Bounded wait; on failure lane 0 leaves a trail record (item, tile, parity).
+// Bounded wait of a single-lane role (TMA producer, MMA issuer); on failure
+// the lane leaves a trail record (item, tile, parity) and goes to the exit.
 #define FIA_WAIT(bar, parity, where)                                                      \
     do {                                                                                  \
         const uint32_t _par = (parity);                                                   \
-        if (!mbar_wait((bar), _par, abort_flag, a.c.err, (where))) {                      \
+        if (!mbar_wait((bar), _par, abort_flag, a.c.err, (where), a.c.wait_ns)) {         \
+            fail_trail(a.c.err, (where), (uint32_t)idx, (uint32_t)dbg_j, _par, (bar));    \
+            goto done;                                                                    \
+        }                                                                                 \
+    } while (0)
+
+// Bounded wait of a whole softmax warp: every lane polls, and the warp leaves
+// together when any lane gave up, so no lane reaches the warp-collective
+// (.sync.aligned) tcgen05 loads and stores or the shuffles that follow without
+// its siblings; pending TMEM stores are waited for before leaving.
+#define FIA_WAIT_W(bar, parity, where)                                                    \
+    do {                                                                                  \
+        const uint32_t _par = (parity);                                                   \
+        const bool _ok = mbar_wait((bar), _par, abort_flag, a.c.err, (where), a.c.wait_ns); \
+        if (!__all_sync(0xffffffffu, _ok)) {                                              \
             if (lane == 0) fail_trail(a.c.err, (where), (uint32_t)idx, (uint32_t)dbg_j,   \
                                       _par, (bar));                                       \
+            tmem_st_wait();                                                               \
             goto done;                                                                    \
         }                                                                                 \
     } while (0)
@@ -157,6 +174,8 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     uint64_t *o_full = pv_done + 2;         // [2]  last PV_X of the pair done
     uint64_t *pse_full = o_full + 2;        // [16] per softmax warp (pse mode)
     uint64_t *vz_full = pse_full + 16;      // zero rows copied over a ragged V tile
+    uint64_t *mma_drain = vz_full + 1;      // error exit: every MMA issued so far is done
+    uint64_t *never = mma_drain + 1;        // test hook: nothing arrives on it
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + Cfg::kNumBar);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -183,6 +202,8 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         }
         for (int x = 0; x < 16; ++x) mbar_init(&pse_full[x], 1);
         mbar_init(vz_full, 1);
+        mbar_init(mma_drain, 1);
+        mbar_init(never, 1);
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tq);
@@ -200,6 +221,9 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     const uint32_t tmem = *tmem_slot;
     int dbg_j = -1;     // tile index recorded in failure trails
     int idx = -1;
+    // Copies each role has requested and (for the error exit) seen complete:
+    // producer Q / K / V tiles, issuer zero-row copies, softmax pse boxes.
+    uint32_t req_q = 0, req_k = 0, req_v = 0, req_vz = 0, seen_vz = 0, req_ps = 0, seen_ps = 0;
 
     // the plan: inline kernel parameter, or the workspace copy
     const uint8_t *plan = (PB >= kInlinePlanBytes) ? pl.b : a.plan;
@@ -215,12 +239,11 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            uint32_t q_it = 0, kv_it = 0;
             const int br = a.c.box_rows;
             for (idx = it_begin; idx < it_end; ++idx) {
                 const PairGeom gm = pair_geom<BAND>(a, items, seqs, idx);
                 if (gm.nB == 0) continue;
-                FIA_WAIT(q_empty, (q_it & 1) ^ 1, 10);
+                FIA_WAIT(q_empty, (req_q & 1) ^ 1, 10);
                 mbar_arrive_expect_tx(q_full, (gm.t[0].valid ? 2 : 1) * Cfg::kTileBytes);
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
@@ -229,16 +252,16 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                         tma_load_3d(smem + Cfg::kOffQ + x * Cfg::kTileBytes + hv * Cfg::kGroupBytes,
                                     &tq, q_full, hv * 64, gm.t[x].h, gm.cu_q + gm.t[x].q0);
                 }
-                ++q_it;
+                ++req_q;
                 const int32_t *bt_row = a.c.bt + (int64_t)gm.b * a.c.bt_stride;
-                for (int j = 0; j < gm.nB; ++j, ++kv_it) {
+                for (int j = 0; j < gm.nB; ++j) {
                     dbg_j = j;
                     const int t0 = (gm.j0 + j) * kPrefillBN;
                     const int t1 = min(t0 + kPrefillBN, gm.kvlen);
                     const int nbox = (t1 - t0 + br - 1) / br;
                     const uint32_t bytes = (uint32_t)(nbox * br * 128 * Cfg::kHalves);
-                    const int ks = kv_it % KS, vs = kv_it % VS;
-                    FIA_WAIT(&k_empty[ks], ((kv_it / KS) & 1) ^ 1, 11);
+                    const int ks = req_k % KS, vs = req_v % VS;
+                    FIA_WAIT(&k_empty[ks], ((req_k / KS) & 1) ^ 1, 11);
                     uint8_t *kd = smem + Cfg::kOffK + ks * Cfg::kTileBytes;
                     mbar_arrive_expect_tx(&k_full[ks], bytes);
                     for (int bi = 0; bi < nbox; ++bi) {
@@ -249,7 +272,8 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                             tma_load_3d(kd + hv * Cfg::kGroupBytes + bi * br * 128, &tk, &k_full[ks],
                                         hv * 64, y, z);
                     }
-                    FIA_WAIT(&v_empty[vs], ((kv_it / VS) & 1) ^ 1, 12);
+                    ++req_k;
+                    FIA_WAIT(&v_empty[vs], ((req_v / VS) & 1) ^ 1, 12);
                     uint8_t *vd = smem + Cfg::kOffV + vs * Cfg::kTileBytes;
                     mbar_arrive_expect_tx(&v_full[vs], bytes);
                     for (int bi = 0; bi < nbox; ++bi) {
@@ -260,6 +284,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                             tma_load_3d(vd + hv * Cfg::kGroupBytes + bi * br * 128, &tv, &v_full[vs],
                                         hv * 64, y, z);
                     }
+                    ++req_v;
                 }
             }
         }
@@ -272,7 +297,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         // asm statement with descriptors prepared before the wait that
         // precedes it.
         if (lane != 0) goto done;
-        uint32_t q_it = 0, kv_it = 0, p_it[2] = {0, 0}, vz_it = 0;
+        uint32_t q_it = 0, kv_it = 0, p_it[2] = {0, 0};
         constexpr int NKQ = D / 16;                     // K-steps of QK^T
         constexpr uint32_t kHi = umma_desc_hi_sw128(1024);
         constexpr uint32_t kTileStep = Cfg::kTileBytes >> 4;
@@ -351,8 +376,9 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                     for (int hv = 0; hv < Cfg::kHalves; ++hv)
                         bulk_load(vdst + hv * Cfg::kGroupBytes + valid * 128, g_zero_rows, nbytes,
                                   vz_full);
-                    FIA_WAIT(vz_full, vz_it & 1, 27);
-                    ++vz_it;
+                    ++req_vz;
+                    FIA_WAIT(vz_full, seen_vz & 1, 27);
+                    ++seen_vz;
                 }
                 if constexpr (KS >= 2) {
                     // Every wait comes before a block, so each tile's PV(j) and
@@ -451,7 +477,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         // plain mode with a positive scale: mask raw scores and fold the scale
         // into the exponent (one FFMA per element)
         const bool fold = (MODE == kModePlain) && (sl2 > 0.f);
-        uint32_t s_it = 0, p_it = 0, o_it = 0, ps_it = 0;
+        uint32_t s_it = 0, p_it = 0, o_it = 0;
         T *outp = reinterpret_cast<T *>(a.c.out);
         const bool pse_tma = (MODE == kModePse) && a.c.pse_tma;
         uint8_t *pslot = smem + Cfg::kOffPse + sw * 4096;
@@ -460,6 +486,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         // the item's key tile jt (counted from its first key tile j0)
         auto pse_fetch = [&](const PairGeom &g2, const SubGeom &s2, int jt) {
             if (lane == 0) {
+                ++req_ps;
                 mbar_arrive_expect_tx(pbar, 4096);
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh)
@@ -468,6 +495,9 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             }
         };
 
+        // test hook: wait on a barrier nothing signals, so the bounded wait
+        // gives up and the whole CTA takes the error exit
+        if (a.c.stall) FIA_WAIT_W(never, 0, 35);
         for (idx = it_begin; idx < it_end; ++idx) {
             const PairGeom gm = pair_geom<BAND>(a, items, seqs, idx);
             const SubGeom sg = gm.t[X];
@@ -504,7 +534,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             for (int j = 0; j < sg.n; ++j) {
                 dbg_j = j;
                 const int tb = (gm.j0 + j) * kPrefillBN + 64 * half;   // first key of this lane
-                FIA_WAIT(&s_full[X], s_it & 1, 30);
+                FIA_WAIT_W(&s_full[X], s_it & 1, 30);
                 ++s_it;
                 __syncwarp();          // tcgen05.ld/st below are warp-collective (.aligned)
                 tc_fence_after();
@@ -541,8 +571,8 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                         }
                 } else if (MODE == kModePse && pse_tma) {
                     // this lane's row of pse box `half` for tile j (128-byte swizzle)
-                    FIA_WAIT(pbar, ps_it & 1, 34);
-                    ++ps_it;
+                    FIA_WAIT_W(pbar, seen_ps & 1, 34);
+                    ++seen_ps;
                     const int r16 = lane & 15;
                     const uint32_t prow = smem_u32(pslot) + half * 2048 + r16 * 128;
 #pragma unroll
@@ -674,7 +704,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 // after all eight warps have signalled this P.)
                 if (__any_sync(0xffffffffu, need)) {
                     if (j > 0) {
-                        FIA_WAIT(&pv_done[X], (p_it - 1) & 1, 31);
+                        FIA_WAIT_W(&pv_done[X], (p_it - 1) & 1, 31);
                         __syncwarp();
                         tc_fence_after();
                     }
@@ -700,7 +730,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             // ---- epilogue: O / l (+ sink), lse; each lane writes D/2 columns ----
             dbg_j = sg.n;
             l += __shfl_xor_sync(0xffffffffu, l, 16);
-            FIA_WAIT(&o_full[X], o_it & 1, 32);
+            FIA_WAIT_W(&o_full[X], o_it & 1, 32);
             ++o_it;
             __syncwarp();
             tc_fence_after();
@@ -742,6 +772,28 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
 done:
     tc_fence_before();
     __syncthreads();
+    // Error exit: every role has left its loop, so the flag is final here.
+    // Wait for what may still be in flight -- the producer's latest copy into
+    // each ring stage (earlier ones completed before their stage was requested
+    // again), the issuer's MMAs and zero-row copy, a softmax warp's prefetched
+    // pse boxes -- before shared memory and TMEM are released.
+    if (*abort_flag) {
+        if (warp == 0 && lane == 0) {
+            if (req_q > 0) mbar_wait_drain(q_full, (req_q - 1) & 1);
+            for (uint32_t i = (req_k > KS ? req_k - KS : 0u); i < req_k; ++i)
+                mbar_wait_drain(&k_full[i % KS], (i / KS) & 1);
+            for (uint32_t i = (req_v > VS ? req_v - VS : 0u); i < req_v; ++i)
+                mbar_wait_drain(&v_full[i % VS], (i / VS) & 1);
+        } else if (warp == 1 && lane == 0) {
+            umma_commit(mma_drain);
+            mbar_wait_drain(mma_drain, 0);
+            if (req_vz > seen_vz) mbar_wait_drain(vz_full, seen_vz & 1);
+        } else if (warp >= 2 && lane == 0 && req_ps > seen_ps) {
+            mbar_wait_drain(&pse_full[warp - 2], seen_ps & 1);
+        }
+        tc_fence_before();
+        __syncthreads();
+    }
     if (warp == 1) {
         __syncwarp();          // lanes 1-31 left the issuer role early; dealloc is .aligned
         tc_fence_after();

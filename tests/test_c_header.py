@@ -26,6 +26,9 @@ int main(void) {
     if (fia_op_get_plan_info(NULL, &info) != FIA_ERR_NULLPTR) return 3;
     if (fia_decode_run_static(NULL, NULL) != FIA_ERR_NULLPTR) return 4;
     if (strlen(fia_status_string(FIA_ERR_SHAPE)) == 0) return 5;
+    uint32_t word = 7;
+    if (fia_decode_static_error_word(NULL, &word) != FIA_ERR_NULLPTR) return 6;
+    if (fia_op_set_wait_limit(NULL, 0, 0) != FIA_ERR_NULLPTR) return 7;
     printf("%s\n", fia_status_string(FIA_OK));
     return 0;
 }
