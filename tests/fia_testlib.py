@@ -51,6 +51,47 @@ def compare(out, lse, ref_out, ref_lse, what=""):
     return mx, mean
 
 
+def lse_err(lse, ref_lse):
+    """max |err| of the finite lse entries (0 when there are none)."""
+    fin = ~np.isinf(ref_lse)
+    return float(np.abs(lse[fin] - ref_lse[fin]).max()) if fin.any() else 0.0
+
+
+def compare_full(p, out, lse):
+    """Every element of problem p's output against the oracle; prints and
+    returns (max|err|, mean|err|, lse |err|)."""
+    import oracle
+    ref_out, ref_lse = oracle.attention(p)
+    mx, mean = compare(out, lse, ref_out, ref_lse, p.name)
+    le = lse_err(lse, ref_lse) if lse is not None else 0.0
+    print("%-28s %9d rows  max|err| %.3e  mean|err| %.3e  lse|err| %.3e"
+          % (p.name, out.shape[0] * out.shape[1], mx, mean, le))
+    return mx, mean, le
+
+
+def head_slice(p, kvh, h0, n):
+    """Sub-problem of p with the n query heads kvh * g + h0 .. + n - 1 (all
+    reading KV head kvh) and that KV head alone: same tokens, block table and
+    cache rows, so its result must equal those heads' rows of p's result.
+    Only inputs are sliced; nothing is computed."""
+    import dataclasses
+    g = p.head_num // p.kv_head_num
+    assert 0 <= h0 and h0 + n <= g
+    hs = slice(kvh * g + h0, kvh * g + h0 + n)
+    kv_ax = 1 if p.kv_layout == 1 else 2
+    cut = lambda t: t.narrow(kv_ax, kvh, 1).contiguous()
+    per_ch = lambda t, mode: (None if t is None else
+                              (t[kvh:kvh + 1].contiguous() if mode == 0 else t))
+    return dataclasses.replace(
+        p, name=p.name + "_kvh%d_h%d" % (kvh, h0), query=p.query[:, hs].contiguous(),
+        key_cache=cut(p.key_cache), value_cache=cut(p.value_cache), head_num=n, kv_head_num=1,
+        slopes=None if p.slopes is None else p.slopes[hs].contiguous(),
+        pse=None if p.pse is None else p.pse[:, hs].contiguous(),
+        sink=None if p.sink is None else p.sink[hs].contiguous(),
+        k_scale=per_ch(p.k_scale, p.k_antiquant_mode), k_offset=per_ch(p.k_offset, p.k_antiquant_mode),
+        v_scale=per_ch(p.v_scale, p.v_antiquant_mode), v_offset=per_ch(p.v_offset, p.v_antiquant_mode))
+
+
 def sample_rows(p, n, seed):
     """Seeded sample of (token, head) rows, always including the first and
     last token of every sequence."""

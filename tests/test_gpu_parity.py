@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import workloads as W
-from fia_testlib import compare, run_gpu, sample_rows
+from fia_testlib import compare, compare_full, head_slice, run_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -46,6 +46,22 @@ DECODE_CASES = {
     "int8_mtp_causal": dict(seq_len=[2, 3], kv_seq_len=[50, 700], head_num=8, kv_head_num=2,
                             head_size=128, block_size=64, kv_dtype="i8",
                             mask_type=W.MASK_CAUSAL),
+    # block sizes that are not powers of two, and the largest accepted (256):
+    # TMA boxes of gcd(blockSize, 64) rows
+    "bs48_gqa4_bf16": dict(seq_len=[1, 1, 1], kv_seq_len=[100, 481, 48], head_num=16,
+                           kv_head_num=4, head_size=128, block_size=48),
+    "bs80_mtp_causal_f16": dict(seq_len=[2, 1], kv_seq_len=[333, 80], head_num=8, kv_head_num=2,
+                                head_size=128, block_size=80, dtype="f16",
+                                mask_type=W.MASK_CAUSAL),
+    "bs256_gqa8_sink": dict(seq_len=[1, 1], kv_seq_len=[700, 2000], head_num=32, kv_head_num=4,
+                            head_size=128, block_size=256, sink=True),
+    "bs80_d64": dict(seq_len=[1, 1], kv_seq_len=[161, 79], head_num=4, kv_head_num=2,
+                     head_size=64, block_size=80),
+    "int8_bs48": dict(seq_len=[1, 1], kv_seq_len=[500, 47], head_num=16, kv_head_num=2,
+                      head_size=128, block_size=48, kv_dtype="i8", sink=True),
+    "int8_bs256_per_token": dict(seq_len=[1, 1], kv_seq_len=[1000, 300], head_num=16,
+                                 kv_head_num=2, head_size=128, block_size=256, kv_dtype="i8",
+                                 k_antiquant="token", v_antiquant="token"),
 }
 
 PREFILL_CASES = {
@@ -85,6 +101,21 @@ PREFILL_CASES = {
     "d64_pairs_causal_sink": dict(seq_len=[256, 100], kv_seq_len=[300, 400], head_num=8,
                                   kv_head_num=2, head_size=64, block_size=64,
                                   mask_type=W.MASK_CAUSAL, sink=True),
+    # block sizes that are not powers of two, and 256: TMA boxes of
+    # gcd(blockSize, 128) rows, block runs that straddle key tiles
+    "bs48_causal_prefix": dict(seq_len=[140, 60], kv_seq_len=[400, 60], head_num=8,
+                               kv_head_num=2, head_size=128, block_size=48,
+                               mask_type=W.MASK_CAUSAL),
+    "bs80_nomask_d64_f16": dict(seq_len=[130, 50], kv_seq_len=[250, 81], head_num=4,
+                                kv_head_num=2, head_size=64, block_size=80, dtype="f16"),
+    "bs256_causal_prefix_sink": dict(seq_len=[200, 129], kv_seq_len=[900, 129], head_num=8,
+                                     kv_head_num=2, head_size=128, block_size=256,
+                                     mask_type=W.MASK_CAUSAL, sink=True),
+    "bs256_alibi_f16": dict(seq_len=[300], kv_seq_len=[300], head_num=4, kv_head_num=4,
+                            head_size=128, block_size=256, dtype="f16",
+                            mask_type=W.MASK_ALIBI, alibi_slopes=True),
+    "bs48_pse_causal": dict(seq_len=[150], kv_seq_len=[200], head_num=4, kv_head_num=2,
+                            head_size=128, block_size=48, mask_type=W.MASK_CAUSAL, pse=True),
 }
 
 
@@ -202,65 +233,156 @@ def test_empty_kv_rows_and_empty_query():
 
 
 # ---------------------------------------------------------------------------
-# The five named workloads at full size: sampled rows against the oracle.
+# The five named workloads (and the f-row workloads) at full size, in the
+# launch configuration the benchmark times: every output element and every
+# lse against the oracle.
 # ---------------------------------------------------------------------------
-def _full_size(p, n_rows, seed):
+def _full_size(p):
     op, out, lse = run_gpu(p)
-    rows = sample_rows(p, n_rows, seed)
-    ref_o, ref_l = oracle.attention(p, rows=rows)
-    got_o = np.stack([out[t, h] for t, h in rows])
-    got_l = np.array([lse[t, h] for t, h in rows])
-    compare(got_o, got_l, ref_o, ref_l, p.name)
+    compare_full(p, out, lse)
     return op, out, lse
 
 
 def test_config_prefill_prefix_full():
-    _full_size(W.prefill_prefix(), 384, 1)
+    op, _, _ = _full_size(W.prefill_prefix())
+    assert op.plan_info()["path"] == 2
 
 
 def test_config_decode_large_batch_full():
-    p = W.decode_large_batch()
-    op, out, lse = _full_size(p, 512, 2)
+    op, _, _ = _full_size(W.decode_large_batch())
+    assert op.plan_info()["path"] == 1
+
+
+def test_config_tiny_decode_full():
+    op, _, _ = _full_size(W.tiny_decode())
     assert op.plan_info()["path"] == 1
 
 
 def test_config_alibi_prefill_and_pse_agree():
     a = W.alibi_prefill(False)
-    _, oa, la = _full_size(a, 256, 3)
+    _, oa, la = _full_size(a)
     b = W.alibi_prefill(True)
-    _, ob, lb = _full_size(b, 256, 3)
+    _, ob, lb = _full_size(b)
     # same bias in two forms: slope generated in registers vs fp16 pse tensor
     assert float(np.abs(oa - ob).max()) <= 2e-2
 
 
 def test_config_int8_long_decode_full():
-    p = W.int8_long_decode()
-    _full_size(p, 256, 4)
+    op, _, _ = _full_size(W.int8_long_decode())
+    assert op.plan_info()["path"] == 1
 
 
 def test_config_bnnbsd_full():
     """The two BnNBsD bench workloads at full size."""
-    op, _, _ = _full_size(W.decode_large_batch_bnnbsd(), 256, 5)
+    op, _, _ = _full_size(W.decode_large_batch_bnnbsd())
     assert op.plan_info()["path"] == 1
-    op, _, _ = _full_size(W.prefill_prefix_bnnbsd(), 256, 6)
+    op, _, _ = _full_size(W.prefill_prefix_bnnbsd())
     assert op.plan_info()["path"] == 2
 
 
 def test_config_mtp_decode_full():
-    p = W.mtp_decode()
-    op, _, _ = _full_size(p, 512, 7)
+    op, _, _ = _full_size(W.mtp_decode())
     assert op.plan_info()["path"] == 1
 
 
 def test_config_int8_per_token_decode_full():
-    _full_size(W.int8_per_token_decode(), 256, 8)
+    _full_size(W.int8_per_token_decode())
 
 
 def test_config_sliding_window_prefill_full():
     p = W.sliding_window_prefill()
-    op, _, lse = _full_size(p, 384, 9)
+    op, _, lse = _full_size(p)
     assert op.plan_info()["path"] == 2
     assert np.all(np.isfinite(lse))          # every row sees at least itself
+
+
+# ---------------------------------------------------------------------------
+# Consistency pins (one operator for Q_S = 1 and Q_S > 1 -- V3 / V4 Formula;
+# deterministic by default -- V3 / V4 determinism statement).
+# ---------------------------------------------------------------------------
+# Each problem takes the prefill (tcgen05) kernel: seqLen * g > 16 rows per KV
+# head.  Its heads, cut into groups small enough for the decode (split-KV)
+# kernels, must give the same rows.
+KERNEL_AGREE_CASES = {
+    "decode_shape_g32_bf16": dict(seq_len=[1, 1, 1], kv_seq_len=[300, 1000, 77], head_num=32,
+                                  kv_head_num=1, head_size=128, block_size=64),
+    "mtp_causal_g8_q3": dict(seq_len=[2, 3], kv_seq_len=[200, 650], head_num=16, kv_head_num=2,
+                             head_size=128, block_size=32, mask_type=W.MASK_CAUSAL),
+    "alibi_sink_g32_f16": dict(seq_len=[1, 2], kv_seq_len=[513, 90], head_num=64, kv_head_num=2,
+                               head_size=128, block_size=128, dtype="f16",
+                               mask_type=W.MASK_ALIBI, alibi_slopes=True, sink=True),
+    "band_d64_g16_q2": dict(seq_len=[2, 1], kv_seq_len=[400, 160], head_num=32, kv_head_num=2,
+                            head_size=64, block_size=16, band=(100, 0)),
+}
+
+
+@pytest.mark.parametrize("name", sorted(KERNEL_AGREE_CASES))
+def test_decode_and_prefill_kernels_agree(name):
+    p = W.make_problem(name=name, seed=zlib.crc32(name.encode()) % 10000, **KERNEL_AGREE_CASES[name])
+    op, out, lse = run_gpu(p)
+    assert op.plan_info()["path"] == 2
+    compare_full(p, out, lse)
+    g = p.head_num // p.kv_head_num
+    qmax = int(max(p.seq_len))
+    # heads per decode-sized group: the largest divisor of g with n * qmax <= 16
+    n = max(d for d in range(1, g + 1) if g % d == 0 and d * qmax <= 16)
+    for kvh in range(p.kv_head_num):
+        for h0 in range(0, g, n):
+            q = head_slice(p, kvh, h0, n)
+            qop, qout, qlse = run_gpu(q)
+            assert qop.plan_info()["path"] == 1
+            hs = slice(kvh * g + h0, kvh * g + h0 + n)
+            compare(qout, qlse, out[:, hs], lse[:, hs], q.name + " vs prefill kernel")
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "i8"])
+def test_split_count_does_not_change_result(kv_dtype):
+    """One sequence planned alone (many short splits) and inside a large batch
+    (few long splits): the same rows up to rounding, and both match the
+    oracle."""
+    big = W.make_problem(name="split_batch_" + kv_dtype, seed=61,
+                         seq_len=[1] * 24, kv_seq_len=[8000] + [6000] * 23, head_num=32,
+                         kv_head_num=8, head_size=128, block_size=128, kv_dtype=kv_dtype,
+                         sink=True)
+    alone = dataclasses.replace(big, name="split_alone_" + kv_dtype, query=big.query[:1].clone(),
+                                block_tables=big.block_tables[:1].clone(),
+                                seq_len=big.seq_len[:1].copy(), kv_seq_len=big.kv_seq_len[:1].copy())
+    op_b, out_b, lse_b = run_gpu(big)
+    op_a, out_a, lse_a = run_gpu(alone)
+    sa, sb = op_a.plan_info()["split_tokens"], op_b.plan_info()["split_tokens"]
+    assert sa < sb and 8000 // sa > 2 * (8000 // sb), (sa, sb)
+    compare_full(alone, out_a, lse_a)
+    compare(out_a, lse_a, out_b[:1], lse_b[:1], "split %d vs %d" % (sa, sb))
+
+
+DETERMINISM_CASES = {
+    "int8_decode_sink": dict(seq_len=[1] * 3, kv_seq_len=[3000, 70, 1500], head_num=16,
+                             kv_head_num=2, head_size=128, block_size=128, kv_dtype="i8",
+                             sink=True),
+    "int8_per_token_mtp": dict(seq_len=[2, 1], kv_seq_len=[900, 2500], head_num=16,
+                               kv_head_num=2, head_size=128, block_size=64, kv_dtype="i8",
+                               k_antiquant="token", v_antiquant="token",
+                               mask_type=W.MASK_CAUSAL),
+    "band_prefill": dict(seq_len=[300, 130], kv_seq_len=[700, 130], head_num=8, kv_head_num=2,
+                         head_size=128, block_size=64, band=(200, 0)),
+    "band_decode": dict(seq_len=[1, 1], kv_seq_len=[4000, 1300], head_num=16, kv_head_num=4,
+                        head_size=128, block_size=128, band=(255, 0)),
+    "alibi_prefill_f16": dict(seq_len=[200, 64], kv_seq_len=[200, 300], head_num=4,
+                              kv_head_num=4, head_size=128, block_size=64,
+                              mask_type=W.MASK_ALIBI, alibi_slopes=True, dtype="f16"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(DETERMINISM_CASES))
+def test_run_to_run_determinism_more_kernels(name):
+    p = W.make_problem(name=name, seed=zlib.crc32(name.encode()) % 10000, **DETERMINISM_CASES[name])
+    op, out, lse = run_gpu(p)
+    for _ in range(3):
+        o2, l2 = op.run()
+        torch.cuda.synchronize()
+        assert np.array_equal(o2.float().double().cpu().numpy(), out)
+        assert np.array_equal(l2.double().cpu().numpy(), lse)
+    assert op.error_word() == 0
 
 
 # BnNBsD cache layout [numBlocks, kvHeadNum, blockSize, headSize] (V3 paged
@@ -290,6 +412,13 @@ BNNBSD_CASES = {
                                      pse=True),
     "prefill_nomask_d64_bs16": dict(seq_len=[129, 40], kv_seq_len=[129, 90], head_num=4,
                                     kv_head_num=1, head_size=64, block_size=16),
+    "decode_bs48_gqa": dict(seq_len=[1, 1], kv_seq_len=[500, 47], head_num=16, kv_head_num=2,
+                            head_size=128, block_size=48),
+    "prefill_bs256_causal": dict(seq_len=[200, 60], kv_seq_len=[600, 60], head_num=8,
+                                 kv_head_num=2, head_size=128, block_size=256,
+                                 mask_type=W.MASK_CAUSAL),
+    "decode_int8_bs80": dict(seq_len=[1, 2], kv_seq_len=[321, 700], head_num=16, kv_head_num=2,
+                             head_size=128, block_size=80, kv_dtype="i8"),
 }
 
 
