@@ -25,6 +25,10 @@ pytestmark = pytest.mark.gpu
 LIMIT_NS = 1_000_000          # 1 ms
 SITE_DECODE_STALL = 3         # decode kernels: the hook's wait
 SITE_PREFILL_STALL = 35       # prefill softmax warps: the hook's wait
+# Prefill wait sites: producer 10-12, issuer 20-27, softmax warps 30-35.  With
+# the softmax warps stalled, the issuer's wait for their P can run out first;
+# either is a time-out of a wait that nothing completed.
+PREFILL_SITES = set(range(10, 13)) | set(range(20, 28)) | set(range(30, 36))
 
 CASES = {
     "decode_bf16": (dict(seq_len=[1, 1, 1], kv_seq_len=[900, 70, 3000], head_num=16,
@@ -56,9 +60,10 @@ def test_bounded_wait_times_out_and_reports(name):
     op.run()
     torch.cuda.synchronize()          # the run returns: no hang, no fault
     ew = op.error_word()
-    assert ew & 0xff == 1 and (ew >> 8) == site, hex(ew)
+    sites = {site} if path == 1 else PREFILL_SITES
+    assert ew & 0xff == 1 and (ew >> 8) in sites, hex(ew)
     trail = op.error_trail()
-    assert trail and any(r["where"] == site for r in trail), trail
+    assert trail and all(r["where"] in sites for r in trail), trail
     assert all(r["block"] < op.plan_info()["grid"] for r in trail)
     # default limit again: the same op, the same device, the oracle's result
     op.set_wait_limit(0, stall=False)
