@@ -23,7 +23,7 @@ REPO = os.path.dirname(PKG_DIR)
 CSRC = os.path.join(PKG_DIR, "csrc")
 LIB_PATH = os.path.join(PKG_DIR, "libfia.so")
 SOURCES = ["fia_host.cu", "decode_kernel.cu", "prefill_kernel.cu"]
-HEADERS = ["fia_device.cuh", "fia_plan.h"]
+HEADERS = ["fia_device.cuh", "fia_plan.h", "prefill_common.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -269,6 +269,62 @@ __device__ __forceinline__ void umma_ts_x8(uint32_t d_tmem, const uint32_t (&a)[
                  : "memory");
 }
 
+// One tile's PV(j) and QK^T(j + 1) from a single asm statement, each
+// descriptor derived inside it from its base: a thread issues a tcgen05.mma
+// about every 63 cycles (measured on B200, for any N), about as long as a
+// 128x128x16 step runs, so the adds issue while the thread waits for its next
+// MMA slot instead of lengthening the issue path.
+//   PV: O[o_col] (+)= P V, P at TMEM column p_col + 8k, V descriptor
+//       v0 + 128k (16-key steps of 2048 bytes), 8 steps, accumulating from
+//       the first step unless acc == 0;
+//   QK: S[s_col] = Q K^T, Q and K descriptors q0 / k0 + 2k within a 64-column
+//       group and + 1024 for the second group (128-row tiles), 8 steps;
+//   then one commit on `bar`.
+__device__ __forceinline__ void umma_pv_qk(uint32_t o_col, uint32_t p_col, uint64_t v0,
+                                           uint32_t idesc_pv, uint32_t acc, uint32_t s_col,
+                                           uint64_t q0, uint64_t k0, uint32_t idesc_qk,
+                                           uint64_t *bar) {
+    asm volatile(
+        "{\n\t.reg .pred p, t, z;\n\t.reg .b64 v, q, k;\n\t.reg .b32 pa;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.b32 t, %4, %4;\n\t"
+        "setp.ne.b32 z, %4, %4;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+        "add.s32 pa, %1, 8;\n\tadd.s64 v, %2, 128;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [pa], v, %3, t;\n\t"
+        "add.s32 pa, %1, 16;\n\tadd.s64 v, %2, 256;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [pa], v, %3, t;\n\t"
+        "add.s32 pa, %1, 24;\n\tadd.s64 v, %2, 384;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [pa], v, %3, t;\n\t"
+        "add.s32 pa, %1, 32;\n\tadd.s64 v, %2, 512;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [pa], v, %3, t;\n\t"
+        "add.s32 pa, %1, 40;\n\tadd.s64 v, %2, 640;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [pa], v, %3, t;\n\t"
+        "add.s32 pa, %1, 48;\n\tadd.s64 v, %2, 768;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [pa], v, %3, t;\n\t"
+        "add.s32 pa, %1, 56;\n\tadd.s64 v, %2, 896;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [pa], v, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%5], %6, %7, %8, z;\n\t"
+        "add.s64 q, %6, 2;\n\tadd.s64 k, %7, 2;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%5], q, k, %8, t;\n\t"
+        "add.s64 q, %6, 4;\n\tadd.s64 k, %7, 4;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%5], q, k, %8, t;\n\t"
+        "add.s64 q, %6, 6;\n\tadd.s64 k, %7, 6;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%5], q, k, %8, t;\n\t"
+        "add.s64 q, %6, 1024;\n\tadd.s64 k, %7, 1024;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%5], q, k, %8, t;\n\t"
+        "add.s64 q, %6, 1026;\n\tadd.s64 k, %7, 1026;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%5], q, k, %8, t;\n\t"
+        "add.s64 q, %6, 1028;\n\tadd.s64 k, %7, 1028;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%5], q, k, %8, t;\n\t"
+        "add.s64 q, %6, 1030;\n\tadd.s64 k, %7, 1030;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%5], q, k, %8, t;\n\t"
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%9];\n\t}"
+        ::"r"(o_col), "r"(p_col), "l"(v0), "r"(idesc_pv), "r"(acc), "r"(s_col), "l"(q0), "l"(k0),
+          "r"(idesc_qk), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // Arrive (once) on `bar` when every tcgen05 op this thread issued so far is done.
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"

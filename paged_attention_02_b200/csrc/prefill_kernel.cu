@@ -40,10 +40,9 @@
 
 #include "fia_device.cuh"
 #include "fia_plan.h"
+#include "prefill_common.cuh"
 
 namespace fia {
-
-enum { kModePlain = 0, kModeAlibi = 1, kModePse = 2 };
 
 // 128 rows x 128 bytes of zeros (static storage starts zeroed): copied by the
 // bulk-copy engine over the V rows past kvSeqLen of a ragged last key tile.
@@ -66,9 +65,9 @@ struct PrefillCfg {
     static constexpr int kPseBytes = (MODE == kModePse) ? 16 * 4096 : 0;
     static constexpr int kOffBar = kOffPse + kPseBytes;
     // q_full, q_empty, k_full/k_empty[KS], v_full/v_empty[VS],
-    // s_full[2], p_full[2], pv_done[2], o_full[2], pse_full[16], vz_full,
+    // s_full[2], p_full[2], o_full[2], pse_full[16], vz_full,
     // mma_drain (error exit), never (test hook: nothing arrives on it)
-    static constexpr int kNumBar = 2 + 2 * kKStages + 2 * kVStages + 8 + 16 + 1 + 2;
+    static constexpr int kNumBar = 2 + 2 * kKStages + 2 * kVStages + 6 + 16 + 1 + 2;
     static constexpr int kUsed = kOffBar + kNumBar * 8 + 16;
     // Keep one CTA per SM (each CTA holds all 512 TMEM columns).
     static constexpr int kSmem = 1024 + (kUsed > 118 * 1024 ? kUsed : 118 * 1024);
@@ -77,48 +76,6 @@ struct PrefillCfg {
     static constexpr uint32_t col_o(int x) { return 256u + (uint32_t)x * D; }
     static constexpr int kThreads = 576;   // producer, UMMA, 2 x 8 softmax warps
 };
-
-struct SubGeom {
-    bool valid;
-    int q0, h, rows, n;
-};
-struct PairGeom {
-    int b, kvh, cu_q, qlen, kvlen;
-    SubGeom t[2];
-    int nA, nB;   // key tiles of tile 0 (0 if absent) and tile 1; nA <= nB
-    int j0;       // first key tile (past 0 only under a band mask; both tiles share it)
-};
-
-template <bool BAND>
-__device__ __forceinline__ PairGeom pair_geom(const PrefillArgs &a, const PrefillItem *items,
-                                              const SeqInfo *seqs, int idx) {
-    const PrefillItem it = items[idx];
-    const SeqInfo si = seqs[it.b];
-    const bool causal = (a.c.mask_type == 9 || a.c.mask_type == 3);
-    PairGeom g;
-    g.b = it.b; g.kvh = it.kvh; g.cu_q = si.cu_q; g.qlen = si.qlen; g.kvlen = si.kvlen;
-    g.j0 = 0;
-#pragma unroll
-    for (int x = 0; x < 2; ++x) {
-        SubGeom &s = g.t[x];
-        s.valid = it.h[x] >= 0;
-        s.q0 = it.q0[x];
-        s.h = it.h[x];
-        s.rows = s.valid ? min(kPrefillBM, si.qlen - it.q0[x]) : 0;
-        // keys the tile's rows can see: [lo, hi) (same rule as the host plan)
-        const int qmin = si.kvlen - si.qlen + it.q0[x], qmax = qmin + s.rows - 1;
-        int lo = 0, hi = causal ? min(si.kvlen, qmax + 1) : si.kvlen;
-        if constexpr (BAND) {
-            lo = max(0, qmin - a.c.pre);
-            hi = min(si.kvlen, qmax + a.c.next + 1);
-        }
-        s.n = (s.valid && hi > lo) ? (hi + kPrefillBN - 1) / kPrefillBN - lo / kPrefillBN : 0;
-        if (BAND && s.valid && hi > lo) g.j0 = lo / kPrefillBN;
-    }
-    g.nA = g.t[0].n;
-    g.nB = g.t[1].n;
-    return g;
-}
 
 // Bounded wait of a single-lane role (TMA producer, MMA issuer); on failure
 // the lane leaves a trail record (item, tile, parity) and goes to the exit.
@@ -170,8 +127,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     uint64_t *v_empty = v_full + VS;        // [VS]
     uint64_t *s_full = v_empty + VS;        // [2]  QK_X done
     uint64_t *p_full = s_full + 2;          // [2]  P_X written (4 warps)
-    uint64_t *pv_done = p_full + 2;         // [2]  PV_X done
-    uint64_t *o_full = pv_done + 2;         // [2]  last PV_X of the pair done
+    uint64_t *o_full = p_full + 2;          // [2]  last PV_X of the pair done
     uint64_t *pse_full = o_full + 2;        // [16] per softmax warp (pse mode)
     uint64_t *vz_full = pse_full + 16;      // zero rows copied over a ragged V tile
     uint64_t *mma_drain = vz_full + 1;      // error exit: every MMA issued so far is done
@@ -197,7 +153,6 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         for (int x = 0; x < 2; ++x) {
             mbar_init(&s_full[x], 1);
             mbar_init(&p_full[x], 8);
-            mbar_init(&pv_done[x], 1);
             mbar_init(&o_full[x], 1);
         }
         for (int x = 0; x < 16; ++x) mbar_init(&pse_full[x], 1);
@@ -304,6 +259,9 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         const uint32_t q_lo = umma_desc_lo(sm_q, 16);
         const uint32_t k_lo = umma_desc_lo(sm_k0, 16);
         const uint32_t v_lo = umma_desc_lo(sm_v0, Cfg::kGroupBytes);
+        // first-step Q descriptors of the two tiles (the fused blocks derive the rest)
+        const uint64_t q0d = ((uint64_t)kHi << 32) | q_lo;
+        const uint64_t q1d = ((uint64_t)kHi << 32) | (q_lo + kTileStep);
         // K-major 128-row operand (a Q or K tile): 16 columns per K-step
         auto kmajor = [&](uint32_t lo, uint64_t (&d)[NKQ]) {
 #pragma unroll
@@ -382,36 +340,55 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 }
                 if constexpr (KS >= 2) {
                     // Every wait comes before a block, so each tile's PV(j) and
-                    // QK(j+1) go out back to back with only commits between
-                    // them.  K(j+1) was requested a whole key tile earlier:
-                    // waiting for it up front almost never waits.
+                    // QK(j+1) go out back to back.  K(j+1) was requested a whole
+                    // key tile earlier: waiting for it up front almost never waits.
+                    // QK_X(j+1) is issued after PV_X(j), so its S-ready commit also
+                    // tells the softmax warps that PV_X(j) is done with O.
                     if (more) FIA_WAIT(&k_full[ksn], (kn / KS) & 1, 22);
                     if (j < gm.nA) {
-                        ptmem(0, pa);
-                        kmajor(q_lo, qd);
                         FIA_WAIT(&p_full[0], p_it[0] & 1, 23);
                         ++p_it[0];
                         tc_fence_after();
-                        umma_ts_x8(tmem + Cfg::col_o(0), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
-                        umma_commit(&pv_done[0]);
-                        if (j + 1 < gm.nA) {
-                            qk(0, qd, kd);
-                            umma_commit(&s_full[0]);
+                        if constexpr (NKQ == 8) {
+                            if (j + 1 < gm.nA) {
+                                umma_pv_qk(tmem + Cfg::col_o(0), tmem + Cfg::col_s(0), vd[0],
+                                           IDESC_PV, j > 0 ? 1u : 0u, tmem + Cfg::col_s(0), q0d,
+                                           kd[0], IDESC_QK, &s_full[0]);
+                            } else {
+                                ptmem(0, pa);
+                                umma_ts_x8(tmem + Cfg::col_o(0), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
+                                umma_commit(&o_full[0]);
+                            }
                         } else {
-                            umma_commit(&o_full[0]);
+                            ptmem(0, pa);
+                            kmajor(q_lo, qd);
+                            umma_ts_x8(tmem + Cfg::col_o(0), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
+                            if (j + 1 < gm.nA) {
+                                qk(0, qd, kd);
+                                umma_commit(&s_full[0]);
+                            } else {
+                                umma_commit(&o_full[0]);
+                            }
                         }
                     }
-                    ptmem(1, pa);
-                    kmajor(q_lo + kTileStep, qd);
                     FIA_WAIT(&p_full[1], p_it[1] & 1, 25);
                     ++p_it[1];
                     tc_fence_after();
-                    umma_ts_x8(tmem + Cfg::col_o(1), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
-                    umma_commit(&pv_done[1]);
+                    if (NKQ == 8 && more) {
+                        umma_pv_qk(tmem + Cfg::col_o(1), tmem + Cfg::col_s(1), vd[0], IDESC_PV,
+                                   j > 0 ? 1u : 0u, tmem + Cfg::col_s(1), q1d, kd[0], IDESC_QK,
+                                   &s_full[1]);
+                    } else {
+                        ptmem(1, pa);
+                        kmajor(q_lo + kTileStep, qd);
+                        umma_ts_x8(tmem + Cfg::col_o(1), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
+                        if (more) {
+                            qk(1, qd, kd);
+                            umma_commit(&s_full[1]);
+                        }
+                    }
                     umma_commit(&v_empty[vs]);
                     if (more) {
-                        qk(1, qd, kd);
-                        umma_commit(&s_full[1]);
                         umma_commit(&k_empty[ksn]);
                         if (j + 1 == gm.nB - 1) umma_commit(q_empty);
                     } else {
@@ -427,7 +404,6 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                         ++p_it[0];
                         tc_fence_after();
                         umma_ts_x8(tmem + Cfg::col_o(0), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
-                        umma_commit(&pv_done[0]);
                         if (j == gm.nA - 1) umma_commit(&o_full[0]);
                         if (j + 1 < gm.nA) {
                             FIA_WAIT(&k_full[ksn], (kn / KS) & 1, 22);
@@ -442,7 +418,6 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                     ++p_it[1];
                     tc_fence_after();
                     umma_ts_x8(tmem + Cfg::col_o(1), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
-                    umma_commit(&pv_done[1]);
                     umma_commit(&v_empty[vs]);
                     if (j == gm.nB - 1) umma_commit(&o_full[1]);
                     if (more) {
@@ -702,12 +677,9 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 // of this tile must be done with O first.  (The softmax warps
                 // cannot drift apart: S for the next key tile is only produced
                 // after all eight warps have signalled this P.)
+                // (S of tile j was written by QK(j), which the issuer put after
+                // PV(j - 1): that PV is done with O.)
                 if (__any_sync(0xffffffffu, need)) {
-                    if (j > 0) {
-                        FIA_WAIT_W(&pv_done[X], (p_it - 1) & 1, 31);
-                        __syncwarp();
-                        tc_fence_after();
-                    }
 #pragma unroll
                     for (int cc = 0; cc < DH / 32; ++cc) {
                         uint32_t orr[32];
