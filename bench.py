@@ -447,6 +447,8 @@ def main():
                          ("mtp_decode", W.mtp_decode),
                          ("int8_per_token_decode", W.int8_per_token_decode),
                          ("sliding_window_prefill", W.sliding_window_prefill),
+                         ("int8_prefix_prefill", W.int8_prefix_prefill),
+                         ("int8_mtp_decode", W.int8_mtp_decode),
                          ("c1_tiny_decode", W.tiny_decode),
                          ("c4a_alibi_prefill", lambda: W.alibi_prefill(False)),
                          ("c4b_alibi_prefill_pse", lambda: W.alibi_prefill(True)),
@@ -458,7 +460,10 @@ def main():
             r2, k2 = time_op(o2, max(5, args.steps // 2), 3, flush)
             m2, km2 = statistics.mean(r2), statistics.mean(k2)
             ent = {"kernel_ms": round(km2, 5), "ms_per_call": round(m2, 5)}
-            if o2.plan_info()["path"] == 1:
+            # decode shapes are bound by the cache read, whichever kernel runs
+            # them (multi-token int8 decode with 24 rows per KV head takes the
+            # tensor-core kernel)
+            if o2.plan_info()["path"] == 1 or name.endswith("_decode"):
                 byts = kv_bytes(q) + io_bytes(q)
                 gbs = byts / (km2 * 1e-3) / 1e9
                 ent.update({"value": round(gbs, 1), "unit": "GB/s", "bound": "hbm",

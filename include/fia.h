@@ -184,9 +184,12 @@ typedef struct fia_op fia_op;
  *  workspaceSize  out: bytes of device workspace fia_run needs (0 if none).
  *  op           out: the planned operation; free with fia_op_destroy.
  *
- * Supported build limits: headSize in {64, 128}; blockSize a multiple of 16,
- * 16 <= blockSize <= 256; headNum <= 1024.  Everything else the pages allow
- * returns FIA_ERR_UNSUPPORTED.
+ * Supported build limits: headSize in {64, 128} (128 with an int8 cache);
+ * blockSize a multiple of 16, 16 <= blockSize <= 256; headNum <= 1024.
+ * Everything else the pages allow returns FIA_ERR_UNSUPPORTED.  With an int8
+ * cache and more than 16 query rows per KV head (seqLen * headNum / kvHeadNum)
+ * the tensor-core path dequantises each K/V tile into the query dtype before
+ * the products, so a dequantised value must lie in that dtype's range.
  * nTokens == 0 returns FIA_OK with workspaceSize 0 and an op whose run is a no-op.
  */
 FIA_API fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key,

@@ -480,6 +480,12 @@ __device__ __forceinline__ uint2 lds64(uint32_t addr) {
     asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
     return v;
 }
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                       uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
+}
 // Transpose of an 8x8 16-bit matrix held in the usual fragment layout
 // (thread t: row t/4, columns 2(t%4), 2(t%4)+1).
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {

@@ -320,7 +320,8 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
     if (nb * bs >= (int64_t(1) << 31) || n_tokens >= (int64_t(1) << 31)) return FIA_ERR_UNSUPPORTED;
     if (band && max_kv >= (int64_t(1) << 30)) return FIA_ERR_UNSUPPORTED;
     const bool decode = (max_q * g <= kDecodeRows);
-    if (kv_int8 && (!decode || D != 128)) return FIA_ERR_UNSUPPORTED;
+    // int8 rows are one 128-byte TMA box row per key on both paths
+    if (kv_int8 && D != 128) return FIA_ERR_UNSUPPORTED;
 
     fia_op *o = new fia_op();
     o->q_dtype = query->dtype == FIA_BF16 ? 1 : 0;
@@ -700,9 +701,17 @@ fia_status fia_run(void *workspace, uint64_t workspaceSize, fia_op *op, void *st
         p.off_seq = (int32_t)op->off_seq;
         p.off_cta = (int32_t)op->off_cta;
         p.off_items = (int32_t)op->off_items;
+        p.k_scale = op->k_scale;
+        p.k_offset = op->k_offset;
+        p.v_scale = op->v_scale;
+        p.v_offset = op->v_offset;
+        p.k_tok_stride = op->k_tok_stride;
+        p.v_tok_stride = op->v_tok_stride;
+        p.k_mode = op->k_mode;
+        p.v_mode = op->v_mode;
         if (op->grid > 0)
-            e = launch_prefill(p, op->tq, op->tk, op->tv, op->tp, op->q_dtype, op->grid,
-                               op->inline_plan ? op->inline_plan->b : nullptr, s);
+            e = launch_prefill(p, op->tq, op->tk, op->tv, op->tp, op->q_dtype, op->kv_int8,
+                               op->grid, op->inline_plan ? op->inline_plan->b : nullptr, s);
     }
     if (e != cudaSuccess) {
         cudaGetLastError();

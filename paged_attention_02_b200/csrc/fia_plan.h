@@ -111,6 +111,12 @@ struct PrefillArgs {
     // kernel's inline plan parameter; offsets are bytes from the plan start.
     const uint8_t *plan;
     int32_t off_seq, off_cta, off_items;
+    // int8 cache: K and V tiles are dequantised, (x + offset) * scale, into
+    // the query dtype in shared memory before the MMAs read them
+    const float *k_scale, *k_offset;   // per channel [KVH, D] or per token [B, S]
+    const float *v_scale, *v_offset;
+    int64_t k_tok_stride, v_tok_stride;   // per-token mode: row stride S of [B, S]
+    int32_t k_mode, v_mode;  // 0 per (KV head, channel), 1 per (b, token)
 };
 
 // A plan of at most this many bytes travels as a kernel parameter (no
@@ -128,7 +134,7 @@ cudaError_t launch_combine(const CombineArgs &a, int q_dtype, bool kv_int8, int 
 // inline_plan: nullptr (plan in the workspace) or kInlinePlanBytes of host data.
 // tp: pse tensor map (used when a.c.pse_tma).
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tq, const CUtensorMap &tk,
-                           const CUtensorMap &tv, const CUtensorMap &tp, int q_dtype, int grid,
-                           const uint8_t *inline_plan, cudaStream_t s);
+                           const CUtensorMap &tv, const CUtensorMap &tp, int q_dtype, bool kv_int8,
+                           int grid, const uint8_t *inline_plan, cudaStream_t s);
 
 }  // namespace fia

@@ -29,6 +29,12 @@
 //              max grows by more than 2^8), P in the input dtype written back
 //              over S; at the end O / l, sink, lse (each lane writes half of
 //              its row).
+//   warps 18-19 (int8 cache only) converters: the producer lands raw int8 K
+//              and V tiles in rings of their own; each converter thread
+//              dequantises, (x + offset) * scale per channel or per token
+//              (V3 fake-quantization bullets), 16 values of 8 rows into the
+//              query dtype, written straight into the swizzled K / V stage
+//              the MMAs read, and the pair of warps then marks the stage full.
 // TMEM (512 columns): S_0 | S_1 | O_0 | O_1.  While one softmax group works on
 // its S, the tensor core runs the other tile's PV and QK^T.
 // Every mbarrier wait is bounded in time (see fia_device.cuh).
@@ -48,14 +54,17 @@ namespace fia {
 // bulk-copy engine over the V rows past kvSeqLen of a ragged last key tile.
 static __device__ __align__(128) uint8_t g_zero_rows[kPrefillBN * 128];
 
-template <int D, int MODE = kModePlain>
+template <int D, int MODE = kModePlain, bool I8 = false>
 struct PrefillCfg {
     static constexpr int kHalves = D / 64;                 // 128-byte column groups
     static constexpr int kTileBytes = 128 * D * 2;         // Q, K or V tile (128 rows)
     static constexpr int kGroupBytes = 128 * 128;          // one 128-row x 128-byte group
-    // pse mode gives one K and one V stage to the per-warp pse slots
+    static constexpr int kRawBytes = 128 * D;              // an int8 K or V tile
+    // pse mode gives one K and one V stage to the per-warp pse slots; an int8
+    // cache gives one V stage to its raw int8 rings (K and V, kRawStages each)
     static constexpr int kKStages = (MODE == kModePse) ? 1 : 2;
-    static constexpr int kVStages = (MODE == kModePse) ? 1 : 2;
+    static constexpr int kVStages = (MODE == kModePse || I8) ? 1 : 2;
+    static constexpr int kRawStages = !I8 ? 0 : (MODE == kModePse) ? 1 : 2;
     static constexpr int kOffQ = 0;                                    // Q[2]
     static constexpr int kOffK = kOffQ + 2 * kTileBytes;               // K[s]
     static constexpr int kOffV = kOffK + kKStages * kTileBytes;        // V[s]
@@ -63,18 +72,23 @@ struct PrefillCfg {
     // per softmax warp, fetched by that warp one key tile ahead
     static constexpr int kOffPse = kOffV + kVStages * kTileBytes;
     static constexpr int kPseBytes = (MODE == kModePse) ? 16 * 4096 : 0;
-    static constexpr int kOffBar = kOffPse + kPseBytes;
+    static constexpr int kOffRaw = kOffPse + kPseBytes;      // raw K[RS], raw V[RS]
+    static constexpr int kOffBar = kOffRaw + 2 * kRawStages * kRawBytes;
     // q_full, q_empty, k_full/k_empty[KS], v_full/v_empty[VS],
     // s_full[2], p_full[2], o_full[2], pse_full[16], vz_full,
-    // mma_drain (error exit), never (test hook: nothing arrives on it)
-    static constexpr int kNumBar = 2 + 2 * kKStages + 2 * kVStages + 6 + 16 + 1 + 2;
+    // mma_drain (error exit), never (test hook: nothing arrives on it),
+    // rk_full/rk_empty[RS], rv_full/rv_empty[RS] (int8 rings)
+    static constexpr int kNumBar = 2 + 2 * kKStages + 2 * kVStages + 6 + 16 + 1 + 2 + 4 * kRawStages;
     static constexpr int kUsed = kOffBar + kNumBar * 8 + 16;
     // Keep one CTA per SM (each CTA holds all 512 TMEM columns).
     static constexpr int kSmem = 1024 + (kUsed > 118 * 1024 ? kUsed : 118 * 1024);
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t col_s(int x) { return (uint32_t)x * 128u; }
     static constexpr uint32_t col_o(int x) { return 256u + (uint32_t)x * D; }
-    static constexpr int kThreads = 576;   // producer, UMMA, 2 x 8 softmax warps
+    // producer, UMMA, 2 x 8 softmax warps (+ 2 int8 converters: five warps on
+    // each SM sub-partition either way, so the register budget is unchanged)
+    static constexpr int kThreads = I8 ? 640 : 576;
+    static_assert(!I8 || D == 128, "int8 tiles are one 128-byte row per key");
 };
 
 // Bounded wait of a single-lane role (TMA producer, MMA issuer); on failure
@@ -104,20 +118,116 @@ struct PrefillCfg {
         }                                                                                 \
     } while (0)
 
-template <typename T, int D, int MODE, int PB, bool BAND>
-__global__ void __launch_bounds__(576, 1)
+// Dequantise one int8 tile (128 keys x 128 dims in 128-byte swizzled rows at
+// `raw`) into T at `dst`: two 64-column groups of 128-byte swizzled rows, the
+// layout TMA gives a 16-bit cache, so the MMAs read it unchanged.  The thread
+// (rl, c) converts dims 16c .. 16c + 15 of rows 8 it + rl; rows at or past
+// `valid` (past kvSeqLen, or never loaded) become zeros.  sc / of: TOK, the
+// tile's per-token rows (sc[r], of[r]); otherwise this thread's 16 channels
+// (sc[i], of[i]).  of may be null.
+//
+// value = (x + offset) * scale: the sign-flipped byte x + 128 placed at
+// mantissa bits 8..15 of 1.0 is the float v = 1 + (x + 128) / 2^15 (exact), and
+// value = v * (2^15 scale) + (offset - 2^15 - 128) * scale: one FMA per value,
+// rounded once, plus the rounding of the constant (about 0.004 scale, far
+// below the final rounding to T).
+template <typename T, bool TOK, bool FULL>
+__device__ __forceinline__ void dequant_tile(const uint8_t *__restrict__ raw,
+                                             uint8_t *__restrict__ dst, int rl, int c, int valid,
+                                             const float *sc, const float *of) {
+    float S[16], C[16];
+    if constexpr (!TOK) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float s = __ldg(sc + i);
+            const float o = of ? __ldg(of + i) : 0.f;
+            S[i] = s * 32768.f;
+            C[i] = (o - 32896.f) * s;
+        }
+    }
+    const uint32_t kOne = 0x3F800000u;
+    const int src_chunk = (c ^ rl) << 4;
+    const int lo_chunk = (((2 * c) & 7) ^ rl) << 4;
+    const int hi_chunk = (((2 * c + 1) & 7) ^ rl) << 4;
+    uint8_t *grp = dst + (c >> 2) * (128 * 128);
+#pragma unroll
+    for (int it = 0; it < 16; ++it) {
+        const int r = it * 8 + rl;
+        const uint4 w4 = *reinterpret_cast<const uint4 *>(raw + r * 128 + src_chunk);
+        const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+        float ts = 0.f, tc = 0.f;
+        if constexpr (TOK) {
+            // rows past the tile's keys read the last valid row's parameters
+            const int rr = FULL ? r : min(r, valid - 1);
+            const float s = __ldg(sc + rr);
+            const float o = of ? __ldg(of + rr) : 0.f;
+            ts = s * 32768.f;
+            tc = (o - 32896.f) * s;
+        }
+        uint32_t o8[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t x = w[i] ^ 0x80808080u;
+            float v[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                v[e] = __uint_as_float(prmt(x, kOne, 0x7604u | ((uint32_t)e << 4)));
+            uint64_t y01, y23;
+            if constexpr (TOK) {
+                const uint64_t S2 = f2pack(ts, ts), C2 = f2pack(tc, tc);
+                y01 = ffma2(f2pack(v[0], v[1]), S2, C2);
+                y23 = ffma2(f2pack(v[2], v[3]), S2, C2);
+            } else {
+                y01 = ffma2(f2pack(v[0], v[1]), f2pack(S[4 * i], S[4 * i + 1]),
+                            f2pack(C[4 * i], C[4 * i + 1]));
+                y23 = ffma2(f2pack(v[2], v[3]), f2pack(S[4 * i + 2], S[4 * i + 3]),
+                            f2pack(C[4 * i + 2], C[4 * i + 3]));
+            }
+            float a0, a1, a2, a3;
+            f2unpack(y01, a0, a1);
+            f2unpack(y23, a2, a3);
+            o8[2 * i] = pack2<T>(a0, a1);
+            o8[2 * i + 1] = pack2<T>(a2, a3);
+        }
+        if (!FULL && r >= valid) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) o8[k] = 0u;
+        }
+        uint8_t *row = grp + r * 128;
+        *reinterpret_cast<uint4 *>(row + lo_chunk) = make_uint4(o8[0], o8[1], o8[2], o8[3]);
+        *reinterpret_cast<uint4 *>(row + hi_chunk) = make_uint4(o8[4], o8[5], o8[6], o8[7]);
+    }
+}
+
+// Bounded wait of a converter warp (no TMEM state to settle): the warp leaves
+// together when any lane gave up.
+#define FIA_WAIT_C(bar, parity, where)                                                    \
+    do {                                                                                  \
+        const uint32_t _par = (parity);                                                   \
+        const bool _ok = mbar_wait((bar), _par, abort_flag, a.c.err, (where), a.c.wait_ns); \
+        if (!__all_sync(0xffffffffu, _ok)) {                                              \
+            if (lane == 0) fail_trail(a.c.err, (where), (uint32_t)idx, (uint32_t)dbg_j,   \
+                                      _par, (bar));                                       \
+            goto done;                                                                    \
+        }                                                                                 \
+    } while (0)
+
+template <typename T, int D, int MODE, int PB, bool BAND, bool I8>
+__global__ void __launch_bounds__(PrefillCfg<D, MODE, I8>::kThreads, 1)
 fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tq,
                    const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                    const __grid_constant__ CUtensorMap tp, const __grid_constant__ PlanBytes<PB> pl) {
-    using Cfg = PrefillCfg<D, MODE>;
-    constexpr int KS = Cfg::kKStages, VS = Cfg::kVStages;
+    using Cfg = PrefillCfg<D, MODE, I8>;
+    constexpr int KS = Cfg::kKStages, VS = Cfg::kVStages, RS = Cfg::kRawStages;
     constexpr bool BF = MmaType<T>::bf16;
     constexpr uint32_t IDESC_QK = umma_idesc_f16(BF, false, false, 128, kPrefillBN);
     constexpr uint32_t IDESC_PV = umma_idesc_f16(BF, false, true, 128, D);
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                ~uintptr_t(1023));
+    // 1024-byte aligned start, kept an offset of the shared array so that
+    // plain loads and stores through it stay shared-memory accesses
+    const uint32_t sm_raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((sm_raw + 1023u) & ~1023u) - sm_raw);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kOffBar);
     uint64_t *q_full = bars + 0;
     uint64_t *q_empty = bars + 1;
@@ -132,6 +242,10 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     uint64_t *vz_full = pse_full + 16;      // zero rows copied over a ragged V tile
     uint64_t *mma_drain = vz_full + 1;      // error exit: every MMA issued so far is done
     uint64_t *never = mma_drain + 1;        // test hook: nothing arrives on it
+    uint64_t *rk_full = never + 1;          // [RS] int8 rings (I8 only)
+    uint64_t *rk_empty = rk_full + RS;
+    uint64_t *rv_full = rk_empty + RS;
+    uint64_t *rv_empty = rv_full + RS;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + Cfg::kNumBar);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -148,8 +262,15 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     if (tid == 0) {
         mbar_init(q_full, 1);
         mbar_init(q_empty, 1);
-        for (int s = 0; s < KS; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
-        for (int s = 0; s < VS; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
+        // int8: the two converter warps fill the K / V stages
+        for (int s = 0; s < KS; ++s) { mbar_init(&k_full[s], I8 ? 2 : 1); mbar_init(&k_empty[s], 1); }
+        for (int s = 0; s < VS; ++s) { mbar_init(&v_full[s], I8 ? 2 : 1); mbar_init(&v_empty[s], 1); }
+        for (int s = 0; s < RS; ++s) {
+            mbar_init(&rk_full[s], 1);
+            mbar_init(&rk_empty[s], 2);
+            mbar_init(&rv_full[s], 1);
+            mbar_init(&rv_empty[s], 2);
+        }
         for (int x = 0; x < 2; ++x) {
             mbar_init(&s_full[x], 1);
             mbar_init(&p_full[x], 8);
@@ -215,6 +336,33 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                     const int t1 = min(t0 + kPrefillBN, gm.kvlen);
                     const int nbox = (t1 - t0 + br - 1) / br;
                     const uint32_t bytes = (uint32_t)(nbox * br * 128 * Cfg::kHalves);
+                    if constexpr (I8) {
+                        // raw int8 rows (one 128-byte box row per key) into the rings
+                        const uint32_t rbytes = (uint32_t)(nbox * br * 128);
+                        const int rks = req_k % RS;
+                        FIA_WAIT(&rk_empty[rks], ((req_k / RS) & 1) ^ 1, 11);
+                        uint8_t *kd = smem + Cfg::kOffRaw + rks * Cfg::kRawBytes;
+                        mbar_arrive_expect_tx(&rk_full[rks], rbytes);
+                        for (int bi = 0; bi < nbox; ++bi) {
+                            const int t = t0 + bi * br;
+                            int y, z;
+                            kv_box_yz(a.c, gm.kvh, bt_row[t / a.c.bs], t % a.c.bs, y, z);
+                            tma_load_3d(kd + bi * br * 128, &tk, &rk_full[rks], 0, y, z);
+                        }
+                        ++req_k;
+                        const int rvs = req_v % RS;
+                        FIA_WAIT(&rv_empty[rvs], ((req_v / RS) & 1) ^ 1, 12);
+                        uint8_t *vd = smem + Cfg::kOffRaw + (RS + rvs) * Cfg::kRawBytes;
+                        mbar_arrive_expect_tx(&rv_full[rvs], rbytes);
+                        for (int bi = 0; bi < nbox; ++bi) {
+                            const int t = t0 + bi * br;
+                            int y, z;
+                            kv_box_yz(a.c, gm.kvh, bt_row[t / a.c.bs], t % a.c.bs, y, z);
+                            tma_load_3d(vd + bi * br * 128, &tv, &rv_full[rvs], 0, y, z);
+                        }
+                        ++req_v;
+                        continue;
+                    }
                     const int ks = req_k % KS, vs = req_v % VS;
                     FIA_WAIT(&k_empty[ks], ((req_k / KS) & 1) ^ 1, 11);
                     uint8_t *kd = smem + Cfg::kOffK + ks * Cfg::kTileBytes;
@@ -324,7 +472,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 kmajor(k_lo + ksn * kTileStep, kd);
                 FIA_WAIT(&v_full[vs], (kvi / VS) & 1, 24);
                 const int valid = gm.kvlen - (gm.j0 + j) * kPrefillBN;
-                if (valid < kPrefillBN) {
+                if (!I8 && valid < kPrefillBN) {     // (int8: the converters write the zeros)
                     // rows past kvSeqLen: P is 0 there, but the slots may hold
                     // anything (NaN * 0 = NaN in the MMA): the bulk-copy engine
                     // writes zeros over them after the V tile has landed.
@@ -432,7 +580,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             }
             kv_it = kv_base + gm.nB;
         }
-    } else {
+    } else if (!I8 || warp < 18) {
         // ------------------------------------------------------------ softmax + epilogue
         // 8 warps per tile: warp (quadrant q, sub-block u) owns query rows
         // 32q + 16u .. +15 (TMEM lanes); lane t holds row 32q + 16u + (t & 15)
@@ -740,6 +888,72 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             tc_fence_before();
             __syncwarp();
         }
+    } else if constexpr (I8) {
+        // ------------------------------------------------------------ int8 converters
+        // Eight consecutive threads take eight consecutive rows of one 16-byte
+        // chunk, so the swizzled loads and stores of a quarter warp hit
+        // distinct banks.  K runs one tile ahead of V -- K(0), K(1), V(0),
+        // K(2), V(1), ... -- since the issuer wants V(j) and K(j + 1) together
+        // and the K stage frees a whole tile earlier than the single V stage.
+        const int u = tid - 18 * 32;
+        const int rl = u & 7;
+        const int c = u >> 3;
+        uint32_t rk_it = 0, rv_it = 0, k_it = 0, v_it = 0;
+        for (idx = it_begin; idx < it_end; ++idx) {
+            const PairGeom gm = pair_geom<BAND>(a, items, seqs, idx);
+            for (int s = 0; s <= gm.nB; ++s) {
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    const bool is_v = (h == 1);
+                    const int j = is_v ? s - 1 : s;
+                    if (j < 0 || j >= gm.nB) continue;
+                    dbg_j = j;
+                    const int t0 = (gm.j0 + j) * kPrefillBN;
+                    const int valid = min(kPrefillBN, gm.kvlen - t0);
+                    const uint32_t rit = is_v ? rv_it : rk_it;
+                    const uint32_t sit = is_v ? v_it : k_it;
+                    const int nst = is_v ? VS : KS;
+                    uint64_t *rfull = (is_v ? rv_full : rk_full) + rit % RS;
+                    uint64_t *rempty = (is_v ? rv_empty : rk_empty) + rit % RS;
+                    uint64_t *dfull = (is_v ? v_full : k_full) + sit % nst;
+                    uint64_t *dempty = (is_v ? v_empty : k_empty) + sit % nst;
+                    FIA_WAIT_C(dempty, ((sit / nst) & 1) ^ 1, is_v ? 43 : 41);
+                    FIA_WAIT_C(rfull, (rit / RS) & 1, is_v ? 42 : 40);
+                    const uint8_t *raw =
+                        smem + Cfg::kOffRaw + ((is_v ? RS : 0) + rit % RS) * Cfg::kRawBytes;
+                    uint8_t *dst = smem + (is_v ? Cfg::kOffV : Cfg::kOffK) + (sit % nst) * Cfg::kTileBytes;
+                    const bool tok = is_v ? a.v_mode != 0 : a.k_mode != 0;
+                    const float *sc = is_v ? a.v_scale : a.k_scale;
+                    const float *of = is_v ? a.v_offset : a.k_offset;
+                    if (tok) {
+                        const int64_t row0 = (int64_t)gm.b * (is_v ? a.v_tok_stride : a.k_tok_stride) + t0;
+                        if (valid == kPrefillBN)
+                            dequant_tile<T, true, true>(raw, dst, rl, c, valid, sc + row0,
+                                                        of ? of + row0 : nullptr);
+                        else
+                            dequant_tile<T, true, false>(raw, dst, rl, c, valid, sc + row0,
+                                                         of ? of + row0 : nullptr);
+                    } else {
+                        const int ch0 = gm.kvh * D + 16 * c;
+                        if (valid == kPrefillBN)
+                            dequant_tile<T, false, true>(raw, dst, rl, c, valid, sc + ch0,
+                                                         of ? of + ch0 : nullptr);
+                        else
+                            dequant_tile<T, false, false>(raw, dst, rl, c, valid, sc + ch0,
+                                                          of ? of + ch0 : nullptr);
+                    }
+                    // the MMAs (async proxy) read what was stored here, and TMA
+                    // refills the raw stage that was read here
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(dfull);
+                        mbar_arrive(rempty);
+                    }
+                    if (is_v) { ++rv_it; ++v_it; } else { ++rk_it; ++k_it; }
+                }
+            }
+        }
     }
 done:
     tc_fence_before();
@@ -752,10 +966,17 @@ done:
     if (*abort_flag) {
         if (warp == 0 && lane == 0) {
             if (req_q > 0) mbar_wait_drain(q_full, (req_q - 1) & 1);
-            for (uint32_t i = (req_k > KS ? req_k - KS : 0u); i < req_k; ++i)
-                mbar_wait_drain(&k_full[i % KS], (i / KS) & 1);
-            for (uint32_t i = (req_v > VS ? req_v - VS : 0u); i < req_v; ++i)
-                mbar_wait_drain(&v_full[i % VS], (i / VS) & 1);
+            if constexpr (I8) {
+                for (uint32_t i = (req_k > RS ? req_k - RS : 0u); i < req_k; ++i)
+                    mbar_wait_drain(&rk_full[i % RS], (i / RS) & 1);
+                for (uint32_t i = (req_v > RS ? req_v - RS : 0u); i < req_v; ++i)
+                    mbar_wait_drain(&rv_full[i % RS], (i / RS) & 1);
+            } else {
+                for (uint32_t i = (req_k > KS ? req_k - KS : 0u); i < req_k; ++i)
+                    mbar_wait_drain(&k_full[i % KS], (i / KS) & 1);
+                for (uint32_t i = (req_v > VS ? req_v - VS : 0u); i < req_v; ++i)
+                    mbar_wait_drain(&v_full[i % VS], (i / VS) & 1);
+            }
         } else if (warp == 1 && lane == 0) {
             umma_commit(mma_drain);
             mbar_wait_drain(mma_drain, 0);
@@ -773,30 +994,32 @@ done:
     }
 }
 
-template <typename T, int D, int MODE, bool BAND>
+template <typename T, int D, int MODE, bool BAND, bool I8>
 static cudaError_t launch_prefill_t(const PrefillArgs &a, const CUtensorMap &tq,
                                     const CUtensorMap &tk, const CUtensorMap &tv,
                                     const CUtensorMap &tp, int grid,
                                     const uint8_t *inline_plan, cudaStream_t s) {
-    const int smem = PrefillCfg<D, MODE>::kSmem;
+    using Cfg = PrefillCfg<D, MODE, I8>;
+    const int smem = Cfg::kSmem;
     if (inline_plan) {
-        auto kern = fia_prefill_kernel<T, D, MODE, kInlinePlanBytes, BAND>;
-        cudaError_t e = ensure_smem_attr<fia_prefill_kernel<T, D, MODE, kInlinePlanBytes, BAND>>(smem);
+        auto kern = fia_prefill_kernel<T, D, MODE, kInlinePlanBytes, BAND, I8>;
+        cudaError_t e =
+            ensure_smem_attr<fia_prefill_kernel<T, D, MODE, kInlinePlanBytes, BAND, I8>>(smem);
         if (e != cudaSuccess) return e;
         // inline_plan points at a full PlanBytes<kInlinePlanBytes> kept by the op
-        kern<<<grid, PrefillCfg<D, MODE>::kThreads, smem, s>>>(
+        kern<<<grid, Cfg::kThreads, smem, s>>>(
             a, tq, tk, tv, tp, *reinterpret_cast<const PlanBytes<kInlinePlanBytes> *>(inline_plan));
     } else {
-        auto kern = fia_prefill_kernel<T, D, MODE, 16, BAND>;
-        cudaError_t e = ensure_smem_attr<fia_prefill_kernel<T, D, MODE, 16, BAND>>(smem);
+        auto kern = fia_prefill_kernel<T, D, MODE, 16, BAND, I8>;
+        cudaError_t e = ensure_smem_attr<fia_prefill_kernel<T, D, MODE, 16, BAND, I8>>(smem);
         if (e != cudaSuccess) return e;
         PlanBytes<16> pl{};
-        kern<<<grid, PrefillCfg<D, MODE>::kThreads, smem, s>>>(a, tq, tk, tv, tp, pl);
+        kern<<<grid, Cfg::kThreads, smem, s>>>(a, tq, tk, tv, tp, pl);
     }
     return cudaGetLastError();
 }
 
-template <typename T, int D>
+template <typename T, int D, bool I8>
 static cudaError_t launch_prefill_mode(const PrefillArgs &a, const CUtensorMap &tq,
                                        const CUtensorMap &tk, const CUtensorMap &tv,
                                        const CUtensorMap &tp, int grid, const uint8_t *ip,
@@ -805,24 +1028,30 @@ static cudaError_t launch_prefill_mode(const PrefillArgs &a, const CUtensorMap &
     // keep the band's range checks out of the other kernels
     if (a.c.band) {
         if (a.c.mask_type != 0) return cudaErrorInvalidValue;
-        if (a.c.pse) return launch_prefill_t<T, D, kModePse, true>(a, tq, tk, tv, tp, grid, ip, s);
-        return launch_prefill_t<T, D, kModePlain, true>(a, tq, tk, tv, tp, grid, ip, s);
+        if (a.c.pse) return launch_prefill_t<T, D, kModePse, true, I8>(a, tq, tk, tv, tp, grid, ip, s);
+        return launch_prefill_t<T, D, kModePlain, true, I8>(a, tq, tk, tv, tp, grid, ip, s);
     }
-    if (a.c.pse) return launch_prefill_t<T, D, kModePse, false>(a, tq, tk, tv, tp, grid, ip, s);
-    if (a.c.mask_type == 3) return launch_prefill_t<T, D, kModeAlibi, false>(a, tq, tk, tv, tp, grid, ip, s);
-    return launch_prefill_t<T, D, kModePlain, false>(a, tq, tk, tv, tp, grid, ip, s);
+    if (a.c.pse) return launch_prefill_t<T, D, kModePse, false, I8>(a, tq, tk, tv, tp, grid, ip, s);
+    if (a.c.mask_type == 3)
+        return launch_prefill_t<T, D, kModeAlibi, false, I8>(a, tq, tk, tv, tp, grid, ip, s);
+    return launch_prefill_t<T, D, kModePlain, false, I8>(a, tq, tk, tv, tp, grid, ip, s);
 }
 
 cudaError_t launch_prefill(const PrefillArgs &a, const CUtensorMap &tq, const CUtensorMap &tk,
-                           const CUtensorMap &tv, const CUtensorMap &tp, int q_dtype, int grid,
-                           const uint8_t *inline_plan, cudaStream_t s) {
+                           const CUtensorMap &tv, const CUtensorMap &tp, int q_dtype, bool kv_int8,
+                           int grid, const uint8_t *inline_plan, cudaStream_t s) {
     const bool bf = (q_dtype == 1);
+    if (kv_int8) {
+        if (a.c.D != 128) return cudaErrorInvalidValue;
+        return bf ? launch_prefill_mode<__nv_bfloat16, 128, true>(a, tq, tk, tv, tp, grid, inline_plan, s)
+                  : launch_prefill_mode<__half, 128, true>(a, tq, tk, tv, tp, grid, inline_plan, s);
+    }
     if (a.c.D == 128)
-        return bf ? launch_prefill_mode<__nv_bfloat16, 128>(a, tq, tk, tv, tp, grid, inline_plan, s)
-                  : launch_prefill_mode<__half, 128>(a, tq, tk, tv, tp, grid, inline_plan, s);
+        return bf ? launch_prefill_mode<__nv_bfloat16, 128, false>(a, tq, tk, tv, tp, grid, inline_plan, s)
+                  : launch_prefill_mode<__half, 128, false>(a, tq, tk, tv, tp, grid, inline_plan, s);
     if (a.c.D == 64)
-        return bf ? launch_prefill_mode<__nv_bfloat16, 64>(a, tq, tk, tv, tp, grid, inline_plan, s)
-                  : launch_prefill_mode<__half, 64>(a, tq, tk, tv, tp, grid, inline_plan, s);
+        return bf ? launch_prefill_mode<__nv_bfloat16, 64, false>(a, tq, tk, tv, tp, grid, inline_plan, s)
+                  : launch_prefill_mode<__half, 64, false>(a, tq, tk, tv, tp, grid, inline_plan, s);
     return cudaErrorInvalidValue;
 }
 

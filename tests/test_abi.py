@@ -154,9 +154,17 @@ def test_phase1_int8_rules():
     ks = torch.ones(2, 128)
     # scales on a bf16 cache are a parameter error
     assert _call(ks=ks, vs=ks) == L.FIA_ERR_PARAM
-    # int8 needs the decode path (seqLen * g <= 16): 9 new tokens x g=2 is too many
+    # more than 16 rows per KV head (9 new tokens x g=2) takes the tensor-core
+    # path, which also reads an int8 cache
+    ok = (L.FIA_ERR_CUDA, L.FIA_OK)               # valid: no GPU here, phase 1 stops at encoding
     q = torch.zeros(10, 4, 128, dtype=torch.bfloat16)
-    assert _call(k=k8, v=k8, ks=ks, vs=ks, q=q, out=q.clone(), seq=[1, 9]) == L.FIA_ERR_UNSUPPORTED
+    assert _call(k=k8, v=k8, ks=ks, vs=ks, q=q, out=q.clone(), seq=[1, 9]) in ok
+    # an int8 cache needs headSize 128 (one 128-byte row per key) on both paths
+    k64 = torch.zeros(8, 16, 2, 64, dtype=torch.int8)
+    ks64 = torch.ones(2, 64)
+    for seq, n in (([1, 2], 3), ([1, 9], 10)):
+        q = torch.zeros(n, 4, 64, dtype=torch.bfloat16)
+        assert _call(k=k64, v=k64, ks=ks64, vs=ks64, q=q, out=q.clone(), seq=seq) == L.FIA_ERR_UNSUPPORTED
 
 
 def test_phase1_build_limits():

@@ -25,10 +25,12 @@ pytestmark = pytest.mark.gpu
 LIMIT_NS = 1_000_000          # 1 ms
 SITE_DECODE_STALL = 3         # decode kernels: the hook's wait
 SITE_PREFILL_STALL = 35       # prefill softmax warps: the hook's wait
-# Prefill wait sites: producer 10-12, issuer 20-27, softmax warps 30-35.  With
-# the softmax warps stalled, the issuer's wait for their P can run out first;
-# either is a time-out of a wait that nothing completed.
-PREFILL_SITES = set(range(10, 13)) | set(range(20, 28)) | set(range(30, 36))
+# Prefill wait sites: producer 10-12, issuer 20-27, softmax warps 30-35, int8
+# converters 40-43.  With the softmax warps stalled, the issuer's wait for
+# their P (or a wait further up the pipeline) can run out first; each is a
+# time-out of a wait that nothing completed.
+PREFILL_SITES = (set(range(10, 13)) | set(range(20, 28)) | set(range(30, 36)) |
+                 set(range(40, 44)))
 
 CASES = {
     "decode_bf16": (dict(seq_len=[1, 1, 1], kv_seq_len=[900, 70, 3000], head_num=16,
@@ -43,6 +45,11 @@ CASES = {
                                 kv_head_num=2, head_size=128, block_size=64,
                                 mask_type=W.MASK_CAUSAL),
                            2, SITE_PREFILL_STALL),
+    "prefill_int8_per_token": (dict(seq_len=[300, 130], kv_seq_len=[700, 130], head_num=8,
+                                    kv_head_num=2, head_size=128, block_size=64, kv_dtype="i8",
+                                    k_antiquant="token", v_antiquant="channel",
+                                    mask_type=W.MASK_CAUSAL),
+                               2, SITE_PREFILL_STALL),
     "prefill_pse_mha_f16": (dict(seq_len=[200], kv_seq_len=[264], head_num=4, kv_head_num=4,
                                  head_size=128, block_size=32, dtype="f16",
                                  mask_type=W.MASK_CAUSAL, pse=True),

@@ -119,6 +119,62 @@ PREFILL_CASES = {
 }
 
 
+# int8 cache with more than 16 query rows per KV head: prefix prefill over an
+# int8 cache and multi-token decode with seqLen * g > 16 take the tensor-core
+# kernel, which dequantises each K / V tile into the query dtype in shared
+# memory (V3 fake-quantization: per-channel and per-token scale / offset).
+INT8_PREFILL_CASES = {
+    "i8_prefix_causal_gqa_bs16_sink": dict(seq_len=[37, 130], kv_seq_len=[100, 300], head_num=8,
+                                           kv_head_num=2, head_size=128, block_size=16,
+                                           mask_type=W.MASK_CAUSAL, kv_dtype="i8", sink=True),
+    "i8_prefix_per_token_bs64": dict(seq_len=[200, 64], kv_seq_len=[500, 64], head_num=8,
+                                     kv_head_num=2, head_size=128, block_size=64,
+                                     mask_type=W.MASK_CAUSAL, kv_dtype="i8",
+                                     k_antiquant="token", v_antiquant="token"),
+    "i8_channel_k_token_v_alibi_f16": dict(seq_len=[150, 40], kv_seq_len=[150, 260], head_num=4,
+                                           kv_head_num=4, head_size=128, block_size=128,
+                                           dtype="f16", mask_type=W.MASK_ALIBI,
+                                           alibi_slopes=True, kv_dtype="i8",
+                                           k_antiquant="channel", v_antiquant="token"),
+    "i8_token_k_channel_v_symmetric": dict(seq_len=[130], kv_seq_len=[700], head_num=2,
+                                           kv_head_num=1, head_size=128, block_size=32,
+                                           kv_dtype="i8", k_antiquant="token",
+                                           v_antiquant="channel", int8_offsets=False),
+    "i8_pse_causal_f16": dict(seq_len=[150, 40], kv_seq_len=[150, 260], head_num=4,
+                              kv_head_num=2, head_size=128, block_size=64,
+                              mask_type=W.MASK_CAUSAL, pse=True, dtype="f16", kv_dtype="i8"),
+    "i8_pse_tma_rows_bs16": dict(seq_len=[200, 70], kv_seq_len=[264, 70], head_num=4,
+                                 kv_head_num=2, head_size=128, block_size=16,
+                                 mask_type=W.MASK_CAUSAL, pse=True, kv_dtype="i8"),
+    "i8_band_prefill": dict(seq_len=[300, 130], kv_seq_len=[700, 130], head_num=8,
+                            kv_head_num=2, head_size=128, block_size=64, band=(200, 0),
+                            kv_dtype="i8", sink=True),
+    "i8_mtp_g8_q3_causal_sink": dict(seq_len=[3, 3, 2], kv_seq_len=[700, 1500, 40], head_num=64,
+                                     kv_head_num=8, head_size=128, block_size=128,
+                                     mask_type=W.MASK_CAUSAL, kv_dtype="i8", sink=True),
+    "i8_g32_per_token_bs48": dict(seq_len=[1, 1], kv_seq_len=[513, 90], head_num=64,
+                                  kv_head_num=2, head_size=128, block_size=48, kv_dtype="i8",
+                                  k_antiquant="token", v_antiquant="token"),
+    "i8_bs80_odd_group_f16": dict(seq_len=[150, 20], kv_seq_len=[400, 20], head_num=6,
+                                  kv_head_num=2, head_size=128, block_size=80, dtype="f16",
+                                  mask_type=W.MASK_CAUSAL, kv_dtype="i8"),
+    "i8_bs256_mha_three_tiles": dict(seq_len=[300], kv_seq_len=[700], head_num=2, kv_head_num=2,
+                                     head_size=128, block_size=256, mask_type=W.MASK_CAUSAL,
+                                     kv_dtype="i8"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(INT8_PREFILL_CASES))
+def test_int8_prefill_small(name):
+    p = W.make_problem(name=name, seed=zlib.crc32(name.encode()) % 10000, spare_blocks=2,
+                       **INT8_PREFILL_CASES[name])
+    op, out, lse = run_gpu(p)
+    assert op.plan_info()["path"] == 2
+    ref_out, ref_lse = oracle.attention(p)
+    compare(out, lse, ref_out, ref_lse, name)
+    assert op.error_word() == 0
+
+
 @pytest.mark.parametrize("name", sorted(DECODE_CASES))
 def test_decode_small(name):
     p = W.make_problem(name=name, seed=zlib.crc32(name.encode()) % 10000, spare_blocks=2, **DECODE_CASES[name])
@@ -189,7 +245,7 @@ def test_dominant_key_bit_exact_gather(kind):
             assert np.array_equal(out[0, h], v), (target, h)
 
 
-@pytest.mark.parametrize("kind", ["decode", "prefill"])
+@pytest.mark.parametrize("kind", ["decode", "prefill", "prefill_int8"])
 def test_block_permutation_bitwise_invariant(kind):
     if kind == "decode":
         base = dict(seq_len=[1, 1, 1], kv_seq_len=[100, 513, 64], head_num=8, kv_head_num=2,
@@ -197,6 +253,8 @@ def test_block_permutation_bitwise_invariant(kind):
     else:
         base = dict(seq_len=[70, 128], kv_seq_len=[170, 128], head_num=4, kv_head_num=2,
                     head_size=128, block_size=16, mask_type=W.MASK_CAUSAL)
+        if kind == "prefill_int8":
+            base.update(kv_dtype="i8", k_antiquant="token")
     p = W.make_problem(seed=33, spare_blocks=5, **base)
     _, out, lse = run_gpu(p)
     _, out2, lse2 = run_gpu(W.permute_blocks(p, 7))
@@ -289,6 +347,16 @@ def test_config_int8_per_token_decode_full():
     _full_size(W.int8_per_token_decode())
 
 
+def test_int8_prefix_prefill_full():
+    op, _, _ = _full_size(W.int8_prefix_prefill())
+    assert op.plan_info()["path"] == 2
+
+
+def test_int8_mtp_decode_full():
+    op, _, _ = _full_size(W.int8_mtp_decode())
+    assert op.plan_info()["path"] == 2          # 3 tokens x g=8 = 24 rows per KV head
+
+
 def test_config_sliding_window_prefill_full():
     p = W.sliding_window_prefill()
     op, _, lse = _full_size(p)
@@ -313,6 +381,14 @@ KERNEL_AGREE_CASES = {
                                mask_type=W.MASK_ALIBI, alibi_slopes=True, sink=True),
     "band_d64_g16_q2": dict(seq_len=[2, 1], kv_seq_len=[400, 160], head_num=32, kv_head_num=2,
                             head_size=64, block_size=16, band=(100, 0)),
+    # int8 cache: the int8 decode kernel against the dequantising prefill kernel
+    "i8_decode_shape_g32_sink": dict(seq_len=[1, 1, 1], kv_seq_len=[300, 1000, 77], head_num=32,
+                                     kv_head_num=1, head_size=128, block_size=64, kv_dtype="i8",
+                                     sink=True),
+    "i8_per_token_g16_q2": dict(seq_len=[2, 1], kv_seq_len=[400, 160], head_num=32,
+                                kv_head_num=2, head_size=128, block_size=32, kv_dtype="i8",
+                                k_antiquant="token", v_antiquant="token",
+                                mask_type=W.MASK_CAUSAL),
 }
 
 
@@ -365,6 +441,10 @@ DETERMINISM_CASES = {
                                mask_type=W.MASK_CAUSAL),
     "band_prefill": dict(seq_len=[300, 130], kv_seq_len=[700, 130], head_num=8, kv_head_num=2,
                          head_size=128, block_size=64, band=(200, 0)),
+    "int8_prefill_mixed_modes": dict(seq_len=[300, 130], kv_seq_len=[700, 130], head_num=8,
+                                     kv_head_num=2, head_size=128, block_size=64, kv_dtype="i8",
+                                     k_antiquant="token", v_antiquant="channel",
+                                     mask_type=W.MASK_CAUSAL, sink=True),
     "band_decode": dict(seq_len=[1, 1], kv_seq_len=[4000, 1300], head_num=16, kv_head_num=4,
                         head_size=128, block_size=128, band=(255, 0)),
     "alibi_prefill_f16": dict(seq_len=[200, 64], kv_seq_len=[200, 300], head_num=4,

@@ -336,6 +336,30 @@ def sliding_window_prefill() -> Problem:
                         block_size=128, dtype="bf16", mask_type=MASK_NONE, band=(1023, 0))
 
 
+def int8_prefix_prefill() -> Problem:
+    """prefill_prefix (B=4, new=[128,256,512,1024] on prefixes
+    [0,512,1024,3072], H=32, KVH=8, D=128, bs=128, causal, bf16 query) over an
+    int8 cache with per-channel fp32 scale ~U(0.005,0.02) and offset
+    ~N(0,0.1), per-head learnable sink ~N(0,1)."""
+    new = [128, 256, 512, 1024]
+    prefix = [0, 512, 1024, 3072]
+    return make_problem(name="int8_prefix_prefill", seed=9, seq_len=new,
+                        kv_seq_len=[a + b for a, b in zip(new, prefix)],
+                        head_num=32, kv_head_num=8, head_size=128, block_size=128,
+                        dtype="bf16", kv_dtype="i8", mask_type=MASK_CAUSAL, sink=True)
+
+
+def int8_mtp_decode() -> Problem:
+    """Multi-token decode over the long int8 cache: 3 new tokens per sequence
+    (causal among themselves) on int8_long_decode's shapes (B=16,
+    kvSeqLen=32768, H=64, KVH=8, so 24 rows per KV head, D=128, bs=128, bf16
+    query, per-channel scale / offset, sink)."""
+    return make_problem(name="int8_mtp_decode", seed=10, seq_len=[3] * 16,
+                        kv_seq_len=[32768] * 16, head_num=64, kv_head_num=8, head_size=128,
+                        block_size=128, dtype="bf16", kv_dtype="i8", mask_type=MASK_CAUSAL,
+                        sink=True)
+
+
 NAMED = {
     "tiny_decode": tiny_decode,
     "prefill_prefix": prefill_prefix,
@@ -348,6 +372,8 @@ NAMED = {
     "mtp_decode": mtp_decode,
     "int8_per_token_decode": int8_per_token_decode,
     "sliding_window_prefill": sliding_window_prefill,
+    "int8_prefix_prefill": int8_prefix_prefill,
+    "int8_mtp_decode": int8_mtp_decode,
 }
 
 
