@@ -26,7 +26,10 @@
 //     the per-row constant, for V through a per-row sum of P from one extra
 //     MMA against ones).  The per-channel K scale is folded into q (with a
 //     power-of-two range fix), the K offset becomes one additive constant per
-//     row, and the V scale/offset are applied once in the combine.
+//     row, and the V scale/offset are applied once in the combine.  A fifth
+//     warp only requests tiles: a compute warp issuing the refills carried
+//     about a thousand cycles of barrier and TMA issue per tile (clock
+//     stamps) and, being the last to finish each tile, set every warp's pace.
 // Kernel 2, fia_combine_kernel: one CTA per (b, kvh, row); merges the unit
 //   partials in fixed logical order (deterministic), adds the learnable sink
 //   to the denominator, applies int8 V dequantisation, writes out and lse.
@@ -418,6 +421,10 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
 //   * V^T (A of O^T): M tile mt, row rho holds output dim
 //     64 (rho >> 3) + 8 (rho & 7) + mt, so a thread's dims of one key row are
 //     two runs of 8 contiguous bytes (two 8-byte shared loads).
+// int8 decode: warps 0-3 compute, warp 4 (from thread kI8Producer) requests
+// the tiles.  Four CTAs per SM for the per-channel single-column-tile kernel
+// (96 registers), three for the others (their extra state spills at 96).
+constexpr int kI8Producer = 128;
 struct DecodeI8Cfg {
     static constexpr int D = 128;
     static constexpr int kTileBytes = kDecodeTile * D;          // one of K or V
@@ -436,7 +443,7 @@ struct DecodeI8Cfg {
 };
 
 template <typename T, int NT, bool KTOK, bool VTOK>
-__global__ void __launch_bounds__(128, 4)
+__global__ void __launch_bounds__(160, (NT == 1 && !KTOK && !VTOK) ? 4 : 3)
 fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv) {
     using Cfg = DecodeI8Cfg;
@@ -498,8 +505,8 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
             tma_load_3d(vst + bi * br * 128, &tv, &full[s], 0, y, z);
         }
     };
-    int n_issued = 0;      // tiles requested (thread 0)
-    if (tid == 0) {
+    int n_issued = 0;      // tiles requested (producer thread)
+    if (tid == kI8Producer) {
         for (int j = 0; j < STAGES && j < n_tiles; ++j) issue(j);
         n_issued = min(STAGES, n_tiles);
     }
@@ -513,6 +520,23 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
             if (lane == 0) fail_trail(a.c.err, 3, (uint32_t)u.b, (uint32_t)u.kvh, 0u, never);
             n_run = 0;
         }
+    }
+    if (warp == 4) {
+        // producer: refill each stage as soon as the four compute warps are
+        // done with it.  A compute warp issuing the refills after its own
+        // share of a tile carried about a thousand cycles of barrier and TMA
+        // issue per tile (clock stamps), and its pace set every warp's data.
+        if (lane == 0 && n_run > 0) {
+            for (int j = 0; j + STAGES < n_tiles; ++j) {
+                if (!mbar_wait(&empty[j % STAGES], (j / STAGES) & 1, abort_flag, a.c.err, 2,
+                               a.c.wait_ns))
+                    break;
+                issue(j + STAGES);
+                ++n_issued;
+            }
+        }
+        __syncwarp();
+        n_run = 0;
     }
 
     // ---- Q'^T fragments: this thread holds query row nb = 8nt + r ----
@@ -635,7 +659,7 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
         else dst[32 + lane] = 0.f;
         cp_async_commit();
     };
-    if constexpr (KTOK || VTOK) tok_fetch(0);
+    if constexpr (KTOK || VTOK) { if (warp < 4) tok_fetch(0); }
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
         voff[nt][0] = voff[nt][1] = 0.f;
@@ -860,19 +884,6 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
 
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
-        bool stop = false;
-        if (tid == 0 && j + STAGES < n_tiles) {
-            if (mbar_wait(&empty[s], (j / STAGES) & 1, abort_flag, a.c.err, 2, a.c.wait_ns)) {
-                issue(j + STAGES);
-                ++n_issued;
-            } else {
-                stop = true;
-            }
-        }
-        __syncwarp();
-        // a failed wait ends the key loop for the whole warp at once (lane 0
-        // alone leaving would strand its siblings at a warp barrier)
-        if (__any_sync(0xffffffffu, stop)) { ok = false; break; }
     }
     (void)ok;
     if constexpr (KTOK || VTOK) cp_async_wait<0>();   // no copy outlives the loop
@@ -895,7 +906,7 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
     // the buffers are reused below and before the CTA ends.  Earlier tiles'
     // copies completed before their stage was requested again.
     if (*abort_flag) {
-        if (tid == 0)
+        if (tid == kI8Producer)
             for (int j = max(0, n_issued - STAGES); j < n_issued; ++j)
                 mbar_wait_drain(&full[j % STAGES], (j / STAGES) & 1);
         __syncthreads();
@@ -903,19 +914,21 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
     float *ow = reinterpret_cast<float *>(smem);                               // [4][16][D]
     float2 *mlw = reinterpret_cast<float2 *>(smem + 4 * kDecodeRows * D * 4);  // [4][16]
     float *oww = ow + warp * kDecodeRows * D;
+    if (warp < 4) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
+        for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int n = 8 * nt + 2 * c + e;
+            for (int e = 0; e < 2; ++e) {
+                const int n = 8 * nt + 2 * c + e;
 #pragma unroll
-            // per-token V: + sum_t p_t sV_t oV_t (exactly 0 otherwise)
-            for (int mt = 0; mt < MT; ++mt) {
-                oww[n * D + 8 * r + mt] = fmaf(-1152.0f, osum[nt][e], o[nt][mt][e]) + voff[nt][e];
-                oww[n * D + 64 + 8 * r + mt] =
-                    fmaf(-1152.0f, osum[nt][e], o[nt][mt][2 + e]) + voff[nt][e];
+                // per-token V: + sum_t p_t sV_t oV_t (exactly 0 otherwise)
+                for (int mt = 0; mt < MT; ++mt) {
+                    oww[n * D + 8 * r + mt] = fmaf(-1152.0f, osum[nt][e], o[nt][mt][e]) + voff[nt][e];
+                    oww[n * D + 64 + 8 * r + mt] =
+                        fmaf(-1152.0f, osum[nt][e], o[nt][mt][2 + e]) + voff[nt][e];
+                }
+                if (r == 0) mlw[warp * kDecodeRows + n] = make_float2(m[nt][e], l[nt][e]);
             }
-            if (r == 0) mlw[warp * kDecodeRows + n] = make_float2(m[nt][e], l[nt][e]);
         }
     }
     __syncthreads();
@@ -1011,7 +1024,7 @@ static cudaError_t launch_decode_i8_m(const DecodeArgs &a, const CUtensorMap &tk
     const int smem = DecodeI8Cfg::kSmem;
     cudaError_t e = ensure_smem_attr<fia_decode_i8_kernel<T, NT, KTOK, VTOK>>(smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, 128, smem, s>>>(a, tk, tv);
+    kern<<<grid, kI8Producer + 32, smem, s>>>(a, tk, tv);
     return cudaGetLastError();
 }
 

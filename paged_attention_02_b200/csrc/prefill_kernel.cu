@@ -74,6 +74,7 @@ struct PrefillCfg {
     static constexpr int kPseBytes = (MODE == kModePse) ? 16 * 4096 : 0;
     static constexpr int kOffRaw = kOffPse + kPseBytes;      // raw K[RS], raw V[RS]
     static constexpr int kOffBar = kOffRaw + 2 * kRawStages * kRawBytes;
+    static_assert(kOffRaw % 1024 == 0, "swizzled TMA destinations are 1024-byte aligned");
     // q_full, q_empty, k_full/k_empty[KS], v_full/v_empty[VS],
     // s_full[2], p_full[2], o_full[2], pse_full[16], vz_full,
     // mma_drain (error exit), never (test hook: nothing arrives on it),

@@ -336,6 +336,15 @@ def sliding_window_prefill() -> Problem:
                         block_size=128, dtype="bf16", mask_type=MASK_NONE, band=(1023, 0))
 
 
+def causal_mha_prefill() -> Problem:
+    """alibi_prefill's shapes with the plain causal mask and no bias (B=2,
+    seqLen=kvSeqLen=2048, H=KVH=32, D=128, bs=128, fp16): the cost of the
+    ALiBi bias is measured against it."""
+    return make_problem(name="causal_mha_prefill", seed=4, seq_len=[2048, 2048],
+                        kv_seq_len=[2048, 2048], head_num=32, kv_head_num=32, head_size=128,
+                        block_size=128, dtype="f16", mask_type=MASK_CAUSAL)
+
+
 def int8_prefix_prefill() -> Problem:
     """prefill_prefix (B=4, new=[128,256,512,1024] on prefixes
     [0,512,1024,3072], H=32, KVH=8, D=128, bs=128, causal, bf16 query) over an
@@ -372,6 +381,7 @@ NAMED = {
     "mtp_decode": mtp_decode,
     "int8_per_token_decode": int8_per_token_decode,
     "sliding_window_prefill": sliding_window_prefill,
+    "causal_mha_prefill": causal_mha_prefill,
     "int8_prefix_prefill": int8_prefix_prefill,
     "int8_mtp_decode": int8_mtp_decode,
 }
