@@ -103,6 +103,14 @@ typedef enum { FIA_ANTIQUANT_PER_CHANNEL = 0, FIA_ANTIQUANT_PER_TOKEN = 1 } fia_
 /* sparse modes (V3 sparseMode): 0 = mask from maskType, 4 = band */
 typedef enum { FIA_SPARSE_NONE = 0, FIA_SPARSE_BAND = 4 } fia_sparse_mode;
 
+/* kernel choice (fia_ext.path).  FIA_PATH_AUTO picks the split-KV decode
+   kernels when the rows per KV head (max seqLen * headNum / kvHeadNum) are at
+   most 16, or at most 128 with max seqLen < 64 (in 16-row chunks), and the
+   tensor-core prefill kernel otherwise.  FIA_PATH_DECODE / FIA_PATH_TENSOR
+   force one (the result agrees to rounding; FIA_PATH_DECODE with more than
+   128 rows per KV head is FIA_ERR_PARAM). */
+typedef enum { FIA_PATH_AUTO = 0, FIA_PATH_DECODE = 1, FIA_PATH_TENSOR = 2 } fia_path;
+
 typedef struct {
     /* pse-shift bias [batch, headNum, maxQ, maxKV], the query's dtype, added to
        the scaled scores: s += pse[b][h][i][t] for new token i and key position t
@@ -151,6 +159,8 @@ typedef struct {
     int32_t sparseMode;
     int64_t preTokens;
     int64_t nextTokens;
+    /* kernel choice, a fia_path value (0, the default, is automatic). */
+    int32_t path;
 } fia_ext;
 
 typedef struct fia_op fia_op;

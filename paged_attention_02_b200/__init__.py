@@ -18,10 +18,12 @@ import torch
 
 from . import _lib
 from ._lib import (FIA_KV_BNBSH, FIA_KV_BNNBSD, FIA_MASK_ALIBI, FIA_MASK_CAUSAL, FIA_MASK_NONE,
-                   FiaError, fia_ext, fia_plan_info, fia_tensor)
+                   FIA_PATH_AUTO, FIA_PATH_DECODE, FIA_PATH_TENSOR, FiaError, fia_ext,
+                   fia_plan_info, fia_tensor)
 
 __all__ = ["FiaOp", "fused_infer_attention", "FIA_MASK_NONE", "FIA_MASK_ALIBI",
-           "FIA_MASK_CAUSAL", "FIA_KV_BNBSH", "FIA_KV_BNNBSD", "FiaError", "tensor_desc",
+           "FIA_MASK_CAUSAL", "FIA_KV_BNBSH", "FIA_KV_BNNBSD", "FIA_PATH_AUTO",
+           "FIA_PATH_DECODE", "FIA_PATH_TENSOR", "FiaError", "tensor_desc",
            "validate_block_tables"]
 
 _DT = {torch.float16: _lib.FIA_F16, torch.bfloat16: _lib.FIA_BF16, torch.float32: _lib.FIA_F32,
@@ -89,6 +91,8 @@ class FiaOp:
     (``want_lse=False`` skips lse).  Tensors are referenced, not copied: keep
     them unchanged while runs are in flight.  ``check_block_tables=True``
     runs ``validate_block_tables`` on the table first (a host copy: debugging only).
+    ``path``: 0 automatic, ``FIA_PATH_DECODE`` (1) or ``FIA_PATH_TENSOR`` (2)
+    forces the split-KV decode kernels or the tensor-core kernel.
     """
 
     def __init__(self, query, key, value, block_tables, seq_len: Sequence[int],
@@ -97,7 +101,8 @@ class FiaOp:
                  k_offset=None, v_scale=None, v_offset=None, out=None, lse=None,
                  want_lse: bool = True, kv_layout: int = FIA_KV_BNBSH,
                  k_antiquant_mode: int = 0, v_antiquant_mode: int = 0,
-                 band: Optional[Tuple[int, int]] = None, check_block_tables: bool = False):
+                 band: Optional[Tuple[int, int]] = None, check_block_tables: bool = False,
+                 path: int = 0):
         dev = query.device
         if check_block_tables:
             bnnbsd = int(kv_layout) == FIA_KV_BNNBSD
@@ -117,7 +122,7 @@ class FiaOp:
                             _ptr(self._d["ko"]), _ptr(self._d["vs"]), _ptr(self._d["vo"]),
                             _ptr(self._d["lse"]), int(kv_layout), int(k_antiquant_mode),
                             int(v_antiquant_mode), _lib.FIA_SPARSE_BAND if band else 0,
-                            int(band[0]) if band else 0, int(band[1]) if band else 0)
+                            int(band[0]) if band else 0, int(band[1]) if band else 0, int(path))
         b = len(seq_len)
         self._sl = (ctypes.c_int32 * max(b, 1))(*[int(x) for x in seq_len])
         self._kl = (ctypes.c_int32 * max(b, 1))(*[int(x) for x in kv_seq_len])

@@ -23,6 +23,7 @@ FIA_ERR_CUDA = 7
 
 FIA_F16, FIA_BF16, FIA_F32, FIA_I8, FIA_I32 = 0, 1, 2, 3, 4
 FIA_MASK_NONE, FIA_MASK_ALIBI, FIA_MASK_CAUSAL = 0, 3, 9
+FIA_PATH_AUTO, FIA_PATH_DECODE, FIA_PATH_TENSOR = 0, 1, 2
 FIA_KV_BNBSH, FIA_KV_BNNBSD = 0, 1
 FIA_ANTIQUANT_PER_CHANNEL, FIA_ANTIQUANT_PER_TOKEN = 0, 1
 FIA_SPARSE_NONE, FIA_SPARSE_BAND = 0, 4
@@ -40,7 +41,7 @@ class fia_ext(ctypes.Structure):
                 ("lse", ctypes.POINTER(fia_tensor)), ("kvLayout", ctypes.c_int32),
                 ("kAntiquantMode", ctypes.c_int32), ("vAntiquantMode", ctypes.c_int32),
                 ("sparseMode", ctypes.c_int32), ("preTokens", ctypes.c_int64),
-                ("nextTokens", ctypes.c_int64)]
+                ("nextTokens", ctypes.c_int64), ("path", ctypes.c_int32)]
 
 
 class fia_plan_info(ctypes.Structure):

@@ -90,7 +90,7 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
     const DecodeUnit u = a.units[blockIdx.x];
     const SeqInfo si = a.c.seq[u.b];
     const int g = a.c.g;
-    const int R = si.qlen * g;
+    const int R = min(kDecodeRows, si.qlen * g - u.r0);   // rows of this unit's chunk
     const int n_tiles = (u.t_end - u.t_begin + kDecodeTile - 1) / kDecodeTile;
 
     if (tid == 0) {
@@ -149,8 +149,8 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
     const int ra = r, rb = r + 8;
     int head_a = 0, head_b = 0, qi_a = 0, qi_b = 0;
     const bool va = ra < R, vb = rb < R;
-    if (va) { qi_a = ra / g; head_a = u.kvh * g + ra % g; }
-    if (vb) { qi_b = rb / g; head_b = u.kvh * g + rb % g; }
+    if (va) { qi_a = (u.r0 + ra) / g; head_a = u.kvh * g + (u.r0 + ra) % g; }
+    if (vb) { qi_b = (u.r0 + rb) / g; head_b = u.kvh * g + (u.r0 + rb) % g; }
     const int qpos_a = si.kvlen - si.qlen + qi_a;
     const int qpos_b = si.kvlen - si.qlen + qi_b;
     const T *qp = reinterpret_cast<const T *>(a.c.q);
@@ -471,7 +471,7 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
     const DecodeUnit u = a.units[blockIdx.x];
     const SeqInfo si = a.c.seq[u.b];
     const int g = a.c.g;
-    const int R = si.qlen * g;
+    const int R = min(kDecodeRows, si.qlen * g - u.r0);   // rows of this unit's chunk
     const int n_tiles = (u.t_end - u.t_begin + kDecodeTile - 1) / kDecodeTile;
 
     if (tid == 0) {
@@ -558,8 +558,8 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
         for (int nt = 0; nt < NT; ++nt) {
             const int nb = 8 * nt + r;
             const bool vr = nb < R;
-            const int qi = vr ? nb / g : 0;
-            const int head = vr ? u.kvh * g + nb % g : 0;
+            const int qi = vr ? (u.r0 + nb) / g : 0;
+            const int head = vr ? u.kvh * g + (u.r0 + nb) % g : 0;
             const T *qrow = qp + ((int64_t)(si.cu_q + qi) * a.c.H + head) * D;
             float qv[KT][4];
             float mx = 0.f, cs = 0.f;
@@ -621,8 +621,8 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
             add[nt][e] = __shfl_sync(0xffffffffu, add_b[nt], 4 * (2 * c + e));
             qs[nt][e] = ktok ? __shfl_sync(0xffffffffu, qs_b[nt], 4 * (2 * c + e)) : 0.f;
             vrow[nt][e] = n < R;
-            const int qi = vrow[nt][e] ? n / g : 0;
-            const int head = vrow[nt][e] ? u.kvh * g + n % g : 0;
+            const int qi = vrow[nt][e] ? (u.r0 + n) / g : 0;
+            const int head = vrow[nt][e] ? u.kvh * g + (u.r0 + n) % g : 0;
             qpos[nt][e] = si.kvlen - si.qlen + qi;
             slope[nt][e] = (alibi && vrow[nt][e]) ? a.c.slopes[head] * kLog2e : 0.f;
             pse_row[nt][e] = nullptr;
@@ -958,15 +958,16 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
 template <typename T, int D, bool INT8>
 __global__ void __launch_bounds__(D)
 fia_combine_kernel(const __grid_constant__ CombineArgs a) {
-    // one CTA per (sequence, kv head, row); one thread per channel d
+    // one CTA per (sequence, kv head, row of a chunk); one thread per channel d
     const CombineItem it = a.items[blockIdx.x];
     const SeqInfo si = a.c.seq[it.b];
     const int g = a.c.g;
-    const int row = blockIdx.y;
-    if (row >= si.qlen * g) return;
+    const int row = blockIdx.y;                 // row within the chunk (partial slot row)
+    const int n = it.r0 + row;                  // row of the group
+    if (n >= si.qlen * g) return;
     const int d = threadIdx.x;
-    const int head = it.kvh * g + row % g;
-    const int token = si.cu_q + row / g;
+    const int head = it.kvh * g + n % g;
+    const int token = si.cu_q + n / g;
     T *out = reinterpret_cast<T *>(a.c.out);
     float M = -INFINITY;
     for (int s = 0; s < it.nsplit; ++s)

@@ -319,7 +319,21 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
     if (bs < 16 || bs > 256 || bs % 16 != 0) return FIA_ERR_UNSUPPORTED;
     if (nb * bs >= (int64_t(1) << 31) || n_tokens >= (int64_t(1) << 31)) return FIA_ERR_UNSUPPORTED;
     if (band && max_kv >= (int64_t(1) << 30)) return FIA_ERR_UNSUPPORTED;
-    const bool decode = (max_q * g <= kDecodeRows);
+    // Kernel choice.  The tensor-core kernel's 128-row tiles hold one query
+    // head's new tokens, so they are well filled only for long new-token
+    // runs; decode-shaped calls (up to 16 rows per KV head, or fewer than 64
+    // new tokens and at most 8 chunks of 16 rows) take the decode kernels,
+    // one unit per 16-row chunk, the chunks of one key range side by side so
+    // that the later reads of each K/V tile come from L2.
+    const int32_t path_hint = ext ? ext->path : (int32_t)FIA_PATH_AUTO;
+    if (path_hint != FIA_PATH_AUTO && path_hint != FIA_PATH_DECODE && path_hint != FIA_PATH_TENSOR)
+        return FIA_ERR_PARAM;
+    const int64_t rows_per_kvh = max_q * g;
+    const bool fits_decode = rows_per_kvh <= (int64_t)kDecodeRows * kDecodeMaxChunks;
+    if (path_hint == FIA_PATH_DECODE && !fits_decode) return FIA_ERR_PARAM;
+    const bool decode = path_hint == FIA_PATH_DECODE ||
+                        (path_hint == FIA_PATH_AUTO &&
+                         (rows_per_kvh <= kDecodeRows || (fits_decode && max_q < 64)));
     // int8 rows are one 128-byte TMA box row per key on both paths
     if (kv_int8 && D != 128) return FIA_ERR_UNSUPPORTED;
 
@@ -458,7 +472,7 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
     std::vector<uint8_t> host;
     if (decode) {
         o->path = 1;
-        o->max_rows = (int32_t)(max_q * g);
+        o->max_rows = (int32_t)std::min<int64_t>(max_q * g, kDecodeRows);   // per unit
         const bool causal = (maskType != FIA_MASK_NONE);
         (void)causal;
         // keys a sequence's rows can see: all of [0, kvSeqLen), or under a band
@@ -475,11 +489,13 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
                 *lo = (*lo / kDecodeTile) * kDecodeTile;
             }
         };
+        // 16-row chunks of sequence b's seqLen * g rows
+        auto chunks = [&](int b) { return (int)((int64_t(seqLen[b]) * g + kDecodeRows - 1) / kDecodeRows); };
         int64_t total = 0;
         for (int b = 0; b < batch; ++b) {
             int64_t lo, hi;
             key_range(b, &lo, &hi);
-            total += (hi - lo) * kvHeadNum;
+            total += (hi - lo) * kvHeadNum * chunks(b);
         }
         const int64_t target_units = (int64_t)nsm * 2 * 4;
         int64_t split = (total + target_units - 1) / std::max<int64_t>(target_units, 1);
@@ -493,18 +509,31 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
             int64_t lo, hi;
             key_range(b, &lo, &hi);
             const int ns = (int)std::max<int64_t>(1, (hi - lo + split - 1) / split);
+            const int nch = chunks(b);
             for (int kvh = 0; kvh < kvHeadNum; ++kvh) {
-                citems.push_back({slot, ns, b, kvh});
-                for (int s = 0; s < ns; ++s) {
-                    DecodeUnit u{};
-                    u.b = b;
-                    u.kvh = kvh;
-                    u.t_begin = (int32_t)std::min<int64_t>(hi, lo + s * split);
-                    u.t_end = (int32_t)std::min<int64_t>(hi, lo + (s + 1) * split);
-                    u.slot = slot + s;
-                    units.push_back(u);
+                // chunk c owns slots slot + c * ns .. + ns - 1 (one per split)
+                for (int ch = 0; ch < nch; ++ch) {
+                    CombineItem ci{};
+                    ci.slot0 = slot + ch * ns;
+                    ci.nsplit = ns;
+                    ci.b = b;
+                    ci.kvh = kvh;
+                    ci.r0 = ch * kDecodeRows;
+                    citems.push_back(ci);
                 }
-                slot += ns;
+                for (int s = 0; s < ns; ++s) {
+                    for (int ch = 0; ch < nch; ++ch) {
+                        DecodeUnit u{};
+                        u.b = b;
+                        u.kvh = kvh;
+                        u.t_begin = (int32_t)std::min<int64_t>(hi, lo + s * split);
+                        u.t_end = (int32_t)std::min<int64_t>(hi, lo + (s + 1) * split);
+                        u.slot = slot + ch * ns + s;
+                        u.r0 = ch * kDecodeRows;
+                        units.push_back(u);
+                    }
+                }
+                slot += nch * ns;
             }
         }
         std::stable_sort(units.begin(), units.end(), [](const DecodeUnit &x, const DecodeUnit &y) {

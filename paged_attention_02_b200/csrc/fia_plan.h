@@ -14,16 +14,21 @@ struct SeqInfo {
     int32_t pad;
 };
 
-// Decode work unit: one (sequence, kv head, key range) split.
+// Decode work unit: one (sequence, kv head, row chunk, key range) split.
+// Rows are the seqLen * g (new token, head-in-group) pairs of the group,
+// row n = token * g + head-in-group; a unit takes rows r0 .. r0 + 15.
 struct DecodeUnit {
     int32_t b, kvh, t_begin, t_end;
-    int32_t slot;    // partial-result slot (logical split order within (b, kvh))
-    int32_t pad[3];
+    int32_t slot;    // partial-result slot (logical split order within its chunk)
+    int32_t r0;      // first row of the chunk
+    int32_t pad[2];
 };
 
-// Decode combine item: the splits of one (sequence, kv head).
+// Decode combine item: the splits of one (sequence, kv head, row chunk).
 struct CombineItem {
     int32_t slot0, nsplit, b, kvh;
+    int32_t r0;      // first row of the chunk
+    int32_t pad[3];
 };
 
 // Prefill work item: a pair of 128-new-token tiles of one sequence that read
@@ -37,6 +42,7 @@ struct PrefillItem {
 };
 
 constexpr int kDecodeRows = 16;      // rows (new token x head-in-group) per decode unit
+constexpr int kDecodeMaxChunks = 8;  // row chunks per (sequence, KV head) on the decode path
 constexpr int kDecodeTile = 64;      // keys per decode pipeline stage
 constexpr int kPrefillBM = 128;      // new tokens per prefill item
 constexpr int kPrefillBN = 128;      // keys per prefill tile

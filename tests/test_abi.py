@@ -62,7 +62,8 @@ def _call(**kw):
     P = lambda x: ctypes.pointer(x) if x is not None else None
     ext = fia_ext(P(d["pse"]), P(d["sink"]), P(d["ks"]), None, P(d["vs"]), None, P(d["lse"]),
                   int(args.get("layout", 0)), int(args.get("kmode", 0)), int(args.get("vmode", 0)),
-                  int(args.get("sparse", 0)), int(args.get("pre", 0)), int(args.get("next", 0)))
+                  int(args.get("sparse", 0)), int(args.get("pre", 0)), int(args.get("next", 0)),
+                  int(args.get("path", 0)))
     if args["seq"] is None:                       # NULL host length arrays
         sl = kl = None
     else:
@@ -165,6 +166,24 @@ def test_phase1_int8_rules():
     for seq, n in (([1, 2], 3), ([1, 9], 10)):
         q = torch.zeros(n, 4, 64, dtype=torch.bfloat16)
         assert _call(k=k64, v=k64, ks=ks64, vs=ks64, q=q, out=q.clone(), seq=seq) == L.FIA_ERR_UNSUPPORTED
+
+
+def test_phase1_path_choice():
+    from paged_attention_02_b200 import _lib as L
+    ok = (L.FIA_ERR_CUDA, L.FIA_OK)               # valid: no GPU here, phase 1 stops at encoding
+    assert _call(path=3) == L.FIA_ERR_PARAM
+    assert _call(path=-1) == L.FIA_ERR_PARAM
+    for path in (0, 1, 2):
+        assert _call(path=path) in ok
+    # the decode kernels take at most 8 chunks of 16 rows per KV head: 65
+    # new tokens x g = 2 is 130 rows
+    q = torch.zeros(66, 4, 128, dtype=torch.bfloat16)
+    k = torch.zeros(16, 16, 2, 128, dtype=torch.bfloat16)
+    bt = torch.zeros(2, 8, dtype=torch.int32)
+    assert _call(q=q, out=q.clone(), k=k, v=k.clone(), bt=bt, seq=[1, 65], kv=[20, 100],
+                 path=1) == L.FIA_ERR_PARAM
+    assert _call(q=q, out=q.clone(), k=k, v=k.clone(), bt=bt, seq=[1, 65], kv=[20, 100],
+                 path=2) in ok
 
 
 def test_phase1_build_limits():

@@ -168,11 +168,49 @@ INT8_PREFILL_CASES = {
 def test_int8_prefill_small(name):
     p = W.make_problem(name=name, seed=zlib.crc32(name.encode()) % 10000, spare_blocks=2,
                        **INT8_PREFILL_CASES[name])
-    op, out, lse = run_gpu(p)
+    op, out, lse = run_gpu(p, path=2)
     assert op.plan_info()["path"] == 2
     ref_out, ref_lse = oracle.attention(p)
     compare(out, lse, ref_out, ref_lse, name)
     assert op.error_word() == 0
+
+
+# Decode-shaped calls with more than 16 rows per KV head (MTP with g * seqLen
+# > 16, wide GQA groups): the decode kernels in 16-row chunks per unit.
+DECODE_CHUNK_CASES = {
+    "chunk_mtp_g8_q3_causal_sink": dict(seq_len=[3, 3, 2], kv_seq_len=[700, 1500, 40], head_num=64,
+                                        kv_head_num=8, head_size=128, block_size=128,
+                                        mask_type=W.MASK_CAUSAL, sink=True),
+    "chunk_g32_decode_f16": dict(seq_len=[1, 1, 1], kv_seq_len=[300, 1000, 77], head_num=32,
+                                 kv_head_num=1, head_size=128, block_size=64, dtype="f16"),
+    "chunk_i8_mtp_g8_q3": dict(seq_len=[3, 2], kv_seq_len=[900, 300], head_num=16, kv_head_num=2,
+                               head_size=128, block_size=64, kv_dtype="i8",
+                               mask_type=W.MASK_CAUSAL, sink=True),
+    "chunk_i8_per_token_g16_q2": dict(seq_len=[2, 1], kv_seq_len=[400, 160], head_num=32,
+                                      kv_head_num=2, head_size=128, block_size=32, kv_dtype="i8",
+                                      k_antiquant="token", v_antiquant="channel",
+                                      mask_type=W.MASK_CAUSAL),
+    "chunk_alibi_g32_q2_f16": dict(seq_len=[1, 2], kv_seq_len=[513, 90], head_num=64,
+                                   kv_head_num=2, head_size=128, block_size=128, dtype="f16",
+                                   mask_type=W.MASK_ALIBI, alibi_slopes=True, sink=True),
+    "chunk_pse_q5_g4_d64": dict(seq_len=[5, 3], kv_seq_len=[90, 200], head_num=8, kv_head_num=2,
+                                head_size=64, block_size=16, mask_type=W.MASK_CAUSAL, pse=True,
+                                dtype="f16"),
+    "chunk_band_q6_g8_d64": dict(seq_len=[6, 2], kv_seq_len=[500, 64], head_num=16,
+                                 kv_head_num=2, head_size=64, block_size=16, band=(77, 1)),
+    "chunk_128_rows_bs48": dict(seq_len=[16, 1], kv_seq_len=[700, 33], head_num=16, kv_head_num=2,
+                                head_size=128, block_size=48, mask_type=W.MASK_CAUSAL),
+}
+
+
+@pytest.mark.parametrize("name", sorted(DECODE_CHUNK_CASES))
+def test_decode_row_chunks(name):
+    p = W.make_problem(name=name, seed=zlib.crc32(name.encode()) % 10000, spare_blocks=2,
+                       **DECODE_CHUNK_CASES[name])
+    op, out, lse = run_gpu(p)
+    assert op.plan_info()["path"] == 1
+    ref_out, ref_lse = oracle.attention(p)
+    compare(out, lse, ref_out, ref_lse, name)
 
 
 @pytest.mark.parametrize("name", sorted(DECODE_CASES))
@@ -187,7 +225,7 @@ def test_decode_small(name):
 @pytest.mark.parametrize("name", sorted(PREFILL_CASES))
 def test_prefill_small(name):
     p = W.make_problem(name=name, seed=zlib.crc32(name.encode()) % 10000, spare_blocks=2, **PREFILL_CASES[name])
-    op, out, lse = run_gpu(p)
+    op, out, lse = run_gpu(p, path=2)
     assert op.plan_info()["path"] == 2
     ref_out, ref_lse = oracle.attention(p)
     compare(out, lse, ref_out, ref_lse, name)
@@ -211,7 +249,7 @@ def test_single_key_returns_value_row_bitwise(kind):
     else:
         p = W.make_problem(seed=31, seq_len=[1, 1], kv_seq_len=[1, 1], head_num=32,
                            kv_head_num=1, head_size=128, block_size=16)
-    _, out, _ = run_gpu(p)
+    _, out, _ = run_gpu(p, path=2 if kind == "prefill" else 0)
     for b in range(2):
         blk = int(p.block_tables[b, 0])
         for h in range(p.head_num):
@@ -239,7 +277,7 @@ def test_dominant_key_bit_exact_gather(kind):
         blk = int(p.block_tables[0, target // 16])
         kc[blk, target % 16, 0] = (q * 200.0 / float(q.norm() ** 2)).to(torch.float16)
         pp = dataclasses.replace(p, key_cache=kc, query=qs)
-        _, out, _ = run_gpu(pp)
+        _, out, _ = run_gpu(pp, path=2 if kind == "prefill" else 0)
         v = p.value_cache[blk, target % 16, 0].double().numpy()
         for h in range(p.head_num):
             assert np.array_equal(out[0, h], v), (target, h)
@@ -354,7 +392,7 @@ def test_int8_prefix_prefill_full():
 
 def test_int8_mtp_decode_full():
     op, _, _ = _full_size(W.int8_mtp_decode())
-    assert op.plan_info()["path"] == 2          # 3 tokens x g=8 = 24 rows per KV head
+    assert op.plan_info()["path"] == 1          # 3 tokens x g=8 = 24 rows: two 16-row chunks
 
 
 def test_config_sliding_window_prefill_full():
@@ -395,9 +433,14 @@ KERNEL_AGREE_CASES = {
 @pytest.mark.parametrize("name", sorted(KERNEL_AGREE_CASES))
 def test_decode_and_prefill_kernels_agree(name):
     p = W.make_problem(name=name, seed=zlib.crc32(name.encode()) % 10000, **KERNEL_AGREE_CASES[name])
-    op, out, lse = run_gpu(p)
+    op, out, lse = run_gpu(p, path=2)
     assert op.plan_info()["path"] == 2
     compare_full(p, out, lse)
+    # the whole problem on the decode kernels, in 16-row chunks
+    dop, dout, dlse = run_gpu(p, path=1)
+    assert dop.plan_info()["path"] == 1
+    compare_full(p, dout, dlse)
+    assert float(np.abs(dout - out).max()) <= 2e-2
     g = p.head_num // p.kv_head_num
     qmax = int(max(p.seq_len))
     # heads per decode-sized group: the largest divisor of g with n * qmax <= 16
