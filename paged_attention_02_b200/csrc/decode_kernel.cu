@@ -46,6 +46,67 @@
 
 namespace fia {
 
+// The last step of a decode unit, once its 4 warps' (m, l, O) sit in shared
+// memory (ow [4][16][D], mlw [4][16]): merge them per row, then either write
+// the unit's partial for the combine kernel or, when every (sequence, KV
+// head, chunk) has a single split (a.direct), finish the rows here with the
+// combine's rules (sink in the denominator, int8 per-channel V, lse) and
+// save the combine launch.
+template <typename T, int D, bool INT8>
+__device__ __forceinline__ void finish_unit(const DecodeArgs &a, const DecodeUnit &u,
+                                            const SeqInfo &si, int R, const float *ow,
+                                            const float2 *mlw) {
+    const int g = a.c.g;
+    float *po = a.part_o + (int64_t)u.slot * kDecodeRows * D;
+    float2 *pml = a.part_ml + (int64_t)u.slot * kDecodeRows;
+    for (int idx = threadIdx.x; idx < R * D; idx += blockDim.x) {
+        const int row = idx / D, d = idx % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, mlw[w * kDecodeRows + row].x);
+        float acc = 0.f, L = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float2 ml = mlw[w * kDecodeRows + row];
+                const float f = ex2(ml.x - M);
+                acc = fmaf(ow[(w * kDecodeRows + row) * D + d], f, acc);
+                L = fmaf(ml.y, f, L);
+            }
+        }
+        if (!a.direct) {
+            po[row * D + d] = acc;
+            if (d == 0) pml[row] = make_float2(M, L);
+            continue;
+        }
+        const int n = u.r0 + row;                  // row of the group
+        const int head = u.kvh * g + n % g;
+        const int64_t o_idx = (int64_t)(si.cu_q + n / g) * a.c.H + head;
+        float val = 0.f, lse = INFINITY;
+        if (M != -INFINITY) {
+            const float sink2 = a.c.sink ? a.c.sink[head] * kLog2e : -INFINITY;
+            const float M2 = fmaxf(M, sink2);
+            const float f = ex2(M - M2);
+            L *= f;
+            acc *= f;
+            const float Lt = L + (a.c.sink ? ex2(sink2 - M2) : 0.f);
+            if constexpr (INT8) {
+                if (!a.v_mode) {      // per-channel V (per-token V is in acc already)
+                    const float vs = a.v_scale[u.kvh * D + d];
+                    const float vo = a.v_offset ? a.v_offset[u.kvh * D + d] : 0.f;
+                    acc = vs * fmaf(vo, L, acc);
+                }
+            }
+            val = acc / Lt;
+            lse = (M2 + log2f(Lt)) * kLn2;
+        }
+        T *out = reinterpret_cast<T *>(a.c.out);
+        if constexpr (MmaType<T>::bf16) out[o_idx * D + d] = __float2bfloat16_rn(val);
+        else out[o_idx * D + d] = __float2half_rn(val);
+        if (d == 0 && a.c.lse) a.c.lse[o_idx] = lse;
+    }
+}
+
 template <int D>
 struct DecodeCfg {
     static constexpr int kRowBytes = D * 2;
@@ -382,26 +443,7 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
         mlw[warp * kDecodeRows + rb] = make_float2(m_b, l_b);
     }
     __syncthreads();
-    float *po = a.part_o + (int64_t)u.slot * kDecodeRows * D;
-    float2 *pml = a.part_ml + (int64_t)u.slot * kDecodeRows;
-    for (int idx = tid; idx < R * D; idx += blockDim.x) {
-        const int row = idx / D, d = idx % D;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) M = fmaxf(M, mlw[w * kDecodeRows + row].x);
-        float acc = 0.f, L = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const float2 ml = mlw[w * kDecodeRows + row];
-                const float f = ex2(ml.x - M);
-                acc = fmaf(ow[(w * kDecodeRows + row) * D + d], f, acc);
-                L = fmaf(ml.y, f, L);
-            }
-        }
-        po[row * D + d] = acc;
-        if (d == 0) pml[row] = make_float2(M, L);
-    }
+    finish_unit<T, D, false>(a, u, si, R, ow, mlw);
 }
 
 // ---------------------------------------------------------------------------
@@ -932,26 +974,7 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
         }
     }
     __syncthreads();
-    float *po = a.part_o + (int64_t)u.slot * kDecodeRows * D;
-    float2 *pml = a.part_ml + (int64_t)u.slot * kDecodeRows;
-    for (int idx = tid; idx < R * D; idx += blockDim.x) {
-        const int row = idx / D, d = idx % D;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) M = fmaxf(M, mlw[w * kDecodeRows + row].x);
-        float acc = 0.f, L = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const float2 ml = mlw[w * kDecodeRows + row];
-                const float f = ex2(ml.x - M);
-                acc = fmaf(ow[(w * kDecodeRows + row) * D + d], f, acc);
-                L = fmaf(ml.y, f, L);
-            }
-        }
-        po[row * D + d] = acc;
-        if (d == 0) pml[row] = make_float2(M, L);
-    }
+    finish_unit<T, D, true>(a, u, si, R, ow, mlw);
 }
 
 // ---------------------------------------------------------------------------

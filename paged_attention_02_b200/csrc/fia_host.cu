@@ -60,6 +60,7 @@ struct fia_op {
     size_t off_part_ml = 0, off_part_o = 0;
     uint64_t ws_size = 0;
     int32_t grid = 0, grid2 = 0;
+    int32_t direct = 0;             // decode: no combine (every item has one split)
     int32_t max_rows = 0;           // decode: max seqLen * g
     int32_t k_mode = 0, v_mode = 0;     // int8 dequant modes (fia_antiquant_mode)
     int64_t k_tok_stride = 0, v_tok_stride = 0;
@@ -550,7 +551,12 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
         off = align_up(off + sizeof(float) * kDecodeRows * D * std::max(slot, 1), 256);
         o->ws_size = off;
         o->grid = (int32_t)units.size();
-        o->grid2 = (int32_t)citems.size();
+        // every (sequence, KV head, chunk) in one split: the decode units
+        // finish their rows themselves and the combine launch is skipped
+        bool one_split = true;
+        for (const CombineItem &ci : citems) one_split = one_split && ci.nsplit == 1;
+        o->direct = one_split ? 1 : 0;
+        o->grid2 = one_split ? 0 : (int32_t)citems.size();
         o->work_items = (int64_t)units.size();
         host.assign(o->plan_bytes, 0);
         std::memcpy(host.data() + o->off_seq, seq.data(), sizeof(SeqInfo) * batch);
@@ -710,6 +716,7 @@ fia_status fia_run(void *workspace, uint64_t workspaceSize, fia_op *op, void *st
         d.v_mode = op->v_mode;
         d.n_units = op->grid;
         d.max_rows = op->max_rows;
+        d.direct = op->direct;
         if (op->grid > 0) e = launch_decode(d, op->tk, op->tv, op->q_dtype, op->kv_int8, op->grid, s);
         if (e == cudaSuccess && op->grid2 > 0) {
             CombineArgs cb{};
@@ -817,6 +824,7 @@ fia_status fia_decode_run_static(fia_op *op, void *stream_ptr) {
     d.v_mode = op->v_mode;
     d.n_units = op->grid;
     d.max_rows = op->max_rows;
+    d.direct = op->direct;
     if (op->ev_start && cudaEventRecord(op->ev_start, s) != cudaSuccess) {
         cudaGetLastError();
         return FIA_ERR_CUDA;

@@ -99,6 +99,7 @@ struct DecodeArgs {
     int32_t k_mode, v_mode;  // int8 dequant: 0 per (KV head, channel), 1 per (b, token)
     int32_t n_units;
     int32_t max_rows;       // max over sequences of seqLen * g (<= kDecodeRows)
+    int32_t direct;         // every item has one split: units write the output (no combine)
 };
 
 struct CombineArgs {

@@ -213,6 +213,34 @@ def test_decode_row_chunks(name):
     compare(out, lse, ref_out, ref_lse, name)
 
 
+# Every (sequence, KV head) in a single split: the decode units finish their
+# rows (sink, int8 V dequantisation, lse) and the combine kernel is skipped.
+SINGLE_SPLIT_CASES = {
+    "one_split_bf16_sink": dict(seq_len=[1, 1, 1], kv_seq_len=[37, 100, 1], head_num=8,
+                                kv_head_num=2, head_size=128, block_size=16, sink=True),
+    "one_split_i8_channel_sink_f16": dict(seq_len=[1, 2], kv_seq_len=[120, 64], head_num=16,
+                                          kv_head_num=2, head_size=128, block_size=32,
+                                          dtype="f16", kv_dtype="i8", sink=True,
+                                          mask_type=W.MASK_CAUSAL),
+    "one_split_i8_per_token": dict(seq_len=[1, 1], kv_seq_len=[90, 128], head_num=8,
+                                   kv_head_num=1, head_size=128, block_size=64, kv_dtype="i8",
+                                   k_antiquant="token", v_antiquant="token"),
+    "one_split_d64_chunks": dict(seq_len=[3, 1], kv_seq_len=[70, 20], head_num=16, kv_head_num=2,
+                                 head_size=64, block_size=16, mask_type=W.MASK_CAUSAL),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SINGLE_SPLIT_CASES))
+def test_single_split_decode_skips_combine(name):
+    p = W.make_problem(name=name, seed=zlib.crc32(name.encode()) % 10000, spare_blocks=2,
+                       **SINGLE_SPLIT_CASES[name])
+    op, out, lse = run_gpu(p)
+    info = op.plan_info()
+    assert info["path"] == 1 and info["kernels_per_run"] == 1
+    ref_out, ref_lse = oracle.attention(p)
+    compare(out, lse, ref_out, ref_lse, name)
+
+
 @pytest.mark.parametrize("name", sorted(DECODE_CASES))
 def test_decode_small(name):
     p = W.make_problem(name=name, seed=zlib.crc32(name.encode()) % 10000, spare_blocks=2, **DECODE_CASES[name])
