@@ -151,7 +151,7 @@ fia_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ 
     const DecodeUnit u = a.units[blockIdx.x];
     const SeqInfo si = a.c.seq[u.b];
     const int g = a.c.g;
-    const int R = min(kDecodeRows, si.qlen * g - u.r0);   // rows of this unit's chunk
+    const int R = min(a.c.chunk_rows, si.qlen * g - u.r0);   // rows of this unit's chunk
     const int n_tiles = (u.t_end - u.t_begin + kDecodeTile - 1) / kDecodeTile;
 
     if (tid == 0) {
@@ -513,7 +513,7 @@ fia_decode_i8_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
     const DecodeUnit u = a.units[blockIdx.x];
     const SeqInfo si = a.c.seq[u.b];
     const int g = a.c.g;
-    const int R = min(kDecodeRows, si.qlen * g - u.r0);   // rows of this unit's chunk
+    const int R = min(a.c.chunk_rows, si.qlen * g - u.r0);   // rows of this unit's chunk
     const int n_tiles = (u.t_end - u.t_begin + kDecodeTile - 1) / kDecodeTile;
 
     if (tid == 0) {
@@ -987,7 +987,7 @@ fia_combine_kernel(const __grid_constant__ CombineArgs a) {
     const int g = a.c.g;
     const int row = blockIdx.y;                 // row within the chunk (partial slot row)
     const int n = it.r0 + row;                  // row of the group
-    if (n >= si.qlen * g) return;
+    if (row >= a.c.chunk_rows || n >= si.qlen * g) return;
     const int d = threadIdx.x;
     const int head = it.kvh * g + n % g;
     const int token = si.cu_q + n / g;

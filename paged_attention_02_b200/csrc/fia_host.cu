@@ -473,7 +473,13 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
     std::vector<uint8_t> host;
     if (decode) {
         o->path = 1;
-        o->max_rows = (int32_t)std::min<int64_t>(max_q * g, kDecodeRows);   // per unit
+        // Rows per unit: 16, or, for an int8 cache past 16 rows per KV head,
+        // 8, so that every unit runs the int8 kernel's single-column-tile
+        // instance (no spills, four CTAs per SM); the extra reads of each
+        // K/V tile by the other chunks of its key range come from L2.
+        const int chunk_rows = (kv_int8 && max_q * g > kDecodeRows) ? kDecodeRows / 2 : kDecodeRows;
+        c.chunk_rows = chunk_rows;
+        o->max_rows = (int32_t)std::min<int64_t>(max_q * g, chunk_rows);   // per unit
         const bool causal = (maskType != FIA_MASK_NONE);
         (void)causal;
         // keys a sequence's rows can see: all of [0, kvSeqLen), or under a band
@@ -491,7 +497,7 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
             }
         };
         // 16-row chunks of sequence b's seqLen * g rows
-        auto chunks = [&](int b) { return (int)((int64_t(seqLen[b]) * g + kDecodeRows - 1) / kDecodeRows); };
+        auto chunks = [&](int b) { return (int)((int64_t(seqLen[b]) * g + chunk_rows - 1) / chunk_rows); };
         int64_t total = 0;
         for (int b = 0; b < batch; ++b) {
             int64_t lo, hi;
@@ -519,7 +525,7 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
                     ci.nsplit = ns;
                     ci.b = b;
                     ci.kvh = kvh;
-                    ci.r0 = ch * kDecodeRows;
+                    ci.r0 = ch * chunk_rows;
                     citems.push_back(ci);
                 }
                 for (int s = 0; s < ns; ++s) {
@@ -530,7 +536,7 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
                         u.t_begin = (int32_t)std::min<int64_t>(hi, lo + s * split);
                         u.t_end = (int32_t)std::min<int64_t>(hi, lo + (s + 1) * split);
                         u.slot = slot + ch * ns + s;
-                        u.r0 = ch * kDecodeRows;
+                        u.r0 = ch * chunk_rows;
                         units.push_back(u);
                     }
                 }

@@ -66,6 +66,7 @@ struct CommonArgs {
     int32_t kv_layout;      // 0: [blocks, bs, KVH, D]; 1: [blocks, KVH, bs, D]
     int32_t band;           // band mask: keys qpos - pre .. qpos + next
     int32_t pre, next;      // band limits (clamped to +-2^30)
+    int32_t chunk_rows;     // decode: rows per unit chunk (16, or 8 for int8 past 16 rows)
     float scale_log2;       // qkScale * log2(e)
     // Failure detection: every bounded wait gives up after wait_ns.  With
     // stall set (a test hook), one role first waits on a barrier that nothing
