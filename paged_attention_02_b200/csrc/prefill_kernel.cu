@@ -30,11 +30,13 @@
 //              over S; at the end O / l, sink, lse (each lane writes half of
 //              its row).
 //   warps 18-19 (int8 cache only) converters: the producer lands raw int8 K
-//              and V tiles in rings of their own; each converter thread
-//              dequantises, (x + offset) * scale per channel or per token
-//              (V3 fake-quantization bullets), 16 values of 8 rows into the
-//              query dtype, written straight into the swizzled K / V stage
-//              the MMAs read, and the pair of warps then marks the stage full.
+//              and V tiles in rings of their own; the products then run in
+//              f16.  Per item the converters rewrite the Q tiles as f16(q *
+//              kScale) (per-channel keys) or f16(q); per tile each thread
+//              turns 16 values of 8 rows into f16 -- per channel x + offset,
+//              widened exactly (the V scale joins in the epilogue), per token
+//              (x + offset) * scale (V3 fake-quantization bullets) -- written
+//              straight into the swizzled K / V stage the MMAs read.
 // TMEM (512 columns): S_0 | S_1 | O_0 | O_1.  While one softmax group works on
 // its S, the tensor core runs the other tile's PV and QK^T.
 // Every mbarrier wait is bounded in time (see fia_device.cuh).
@@ -43,6 +45,8 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <math.h>
+
+#include <type_traits>
 
 #include "fia_device.cuh"
 #include "fia_plan.h"
@@ -78,8 +82,9 @@ struct PrefillCfg {
     // q_full, q_empty, k_full/k_empty[KS], v_full/v_empty[VS],
     // s_full[2], p_full[2], o_full[2], pse_full[16], vz_full,
     // mma_drain (error exit), never (test hook: nothing arrives on it),
-    // rk_full/rk_empty[RS], rv_full/rv_empty[RS] (int8 rings)
-    static constexpr int kNumBar = 2 + 2 * kKStages + 2 * kVStages + 6 + 16 + 1 + 2 + 4 * kRawStages;
+    // rk_full/rk_empty[RS], rv_full/rv_empty[RS] (int8 rings), q_conv (int8:
+    // the converted Q tiles are ready)
+    static constexpr int kNumBar = 2 + 2 * kKStages + 2 * kVStages + 6 + 16 + 1 + 2 + 4 * kRawStages + 1;
     static constexpr int kUsed = kOffBar + kNumBar * 8 + 16;
     // Keep one CTA per SM (each CTA holds all 512 TMEM columns).
     static constexpr int kSmem = 1024 + (kUsed > 118 * 1024 ? kUsed : 118 * 1024);
@@ -200,6 +205,93 @@ __device__ __forceinline__ void dequant_tile(const uint8_t *__restrict__ raw,
     }
 }
 
+// int8 cache, per-channel mode: one tile's bytes widened exactly to f16,
+// x + 128 placed under the f16 exponent pattern of 1024 (the value 1152 + x)
+// minus 1152, with OFS plus the channel's offset (one f16 rounding); the
+// scale is applied elsewhere (folded into Q for K, in the epilogue for V).
+// Same layout and thread mapping as
+// dequant_tile; rows at or past `valid` become zeros.  of: this thread's 16
+// channels' offsets (OFS).
+template <bool FULL, bool OFS>
+__device__ __forceinline__ void widen_tile(const uint8_t *__restrict__ raw,
+                                           uint8_t *__restrict__ dst, int rl, int c, int valid,
+                                           const float *of) {
+    __half2 o2[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        o2[k] = (OFS && of) ? __floats2half2_rn(__ldg(of + 2 * k), __ldg(of + 2 * k + 1))
+                            : __floats2half2_rn(0.f, 0.f);
+    const __half2 k1152 = __floats2half2_rn(1152.f, 1152.f);
+    const uint32_t kF = 0x64646464u;
+    const int src_chunk = (c ^ rl) << 4;
+    const int lo_chunk = (((2 * c) & 7) ^ rl) << 4;
+    const int hi_chunk = (((2 * c + 1) & 7) ^ rl) << 4;
+    uint8_t *grp = dst + (c >> 2) * (128 * 128);
+#pragma unroll
+    for (int it = 0; it < 16; ++it) {
+        const int r = it * 8 + rl;
+        const uint4 w4 = *reinterpret_cast<const uint4 *>(raw + r * 128 + src_chunk);
+        const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+        uint32_t o8[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t x = w[i] ^ 0x80808080u;
+            const uint32_t h01 = prmt(x, kF, 0x4140u), h23 = prmt(x, kF, 0x4342u);
+            __half2 y01 = __hsub2(*reinterpret_cast<const __half2 *>(&h01), k1152);
+            __half2 y23 = __hsub2(*reinterpret_cast<const __half2 *>(&h23), k1152);
+            if constexpr (OFS) {
+                y01 = __hadd2(y01, o2[2 * i]);
+                y23 = __hadd2(y23, o2[2 * i + 1]);
+            }
+            o8[2 * i] = *reinterpret_cast<uint32_t *>(&y01);
+            o8[2 * i + 1] = *reinterpret_cast<uint32_t *>(&y23);
+        }
+        if (!FULL && r >= valid) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) o8[k] = 0u;
+        }
+        uint8_t *row = grp + r * 128;
+        *reinterpret_cast<uint4 *>(row + lo_chunk) = make_uint4(o8[0], o8[1], o8[2], o8[3]);
+        *reinterpret_cast<uint4 *>(row + hi_chunk) = make_uint4(o8[4], o8[5], o8[6], o8[7]);
+    }
+}
+
+// int8 cache: a Q tile (128 rows x 128 dims of T in two 64-column groups of
+// 128-byte swizzled rows) rewritten in place as f16(q * scale_d), so the
+// products run in f16 against the widened keys.  Thread u of 64 takes chunk
+// position p = u & 15 (group p >> 3, chunk p & 7) of rows (u >> 4) + 4 i; the
+// eight threads of a quarter warp cover one row's eight chunks.  sc: the
+// per-channel K scale of the KV head, or null (per-token keys: scale 1).
+template <typename T>
+__device__ __forceinline__ void q_to_f16(uint8_t *__restrict__ q, int u, const float *sc) {
+    const int p = u & 15, hv = p >> 3, cl = p & 7;
+    float s8[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s8[e] = sc ? __ldg(sc + hv * 64 + cl * 8 + e) : 1.f;
+    uint8_t *grp = q + hv * (128 * 128);
+#pragma unroll 4
+    for (int r = u >> 4; r < 128; r += 4) {
+        uint4 *ptr = reinterpret_cast<uint4 *>(grp + r * 128 + ((cl ^ (r & 7)) << 4));
+        const uint4 w4 = *ptr;
+        const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+        uint32_t o4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float f0, f1;
+            if constexpr (MmaType<T>::bf16) {
+                f0 = __uint_as_float(w[i] << 16);
+                f1 = __uint_as_float(w[i] & 0xffff0000u);
+            } else {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
+                f0 = f.x;
+                f1 = f.y;
+            }
+            o4[i] = pack2<__half>(f0 * s8[2 * i], f1 * s8[2 * i + 1]);
+        }
+        *ptr = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+    }
+}
+
 // Bounded wait of a converter warp (no TMEM state to settle): the warp leaves
 // together when any lane gave up.
 #define FIA_WAIT_C(bar, parity, where)                                                    \
@@ -220,7 +312,9 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                    const __grid_constant__ CUtensorMap tp, const __grid_constant__ PlanBytes<PB> pl) {
     using Cfg = PrefillCfg<D, MODE, I8>;
     constexpr int KS = Cfg::kKStages, VS = Cfg::kVStages, RS = Cfg::kRawStages;
-    constexpr bool BF = MmaType<T>::bf16;
+    // int8 cache: the products run in f16 (Q, the widened K / V and P)
+    using MT = std::conditional_t<I8, __half, T>;
+    constexpr bool BF = MmaType<MT>::bf16;
     constexpr uint32_t IDESC_QK = umma_idesc_f16(BF, false, false, 128, kPrefillBN);
     constexpr uint32_t IDESC_PV = umma_idesc_f16(BF, false, true, 128, D);
 
@@ -247,6 +341,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     uint64_t *rk_empty = rk_full + RS;
     uint64_t *rv_full = rk_empty + RS;
     uint64_t *rv_empty = rv_full + RS;
+    uint64_t *q_conv = rv_empty + RS;       // int8: Q in f16 (2 converter warps)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + Cfg::kNumBar);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -281,6 +376,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         mbar_init(vz_full, 1);
         mbar_init(mma_drain, 1);
         mbar_init(never, 1);
+        mbar_init(q_conv, 2);
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tq);
@@ -442,7 +538,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             // registers are scarce (96 per thread) and the softmax roles need them
             uint64_t qd[NKQ], kd[NKQ], vd[8];
             uint32_t pa[8];
-            FIA_WAIT(q_full, q_it & 1, 20);
+            FIA_WAIT(I8 ? q_conv : q_full, q_it & 1, 20);
             ++q_it;
             const uint32_t kv_base = kv_it;
             {
@@ -810,7 +906,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                         acc2[x & 3] = fadd2(acc2[x & 3], pp);
                         float p0, p1;
                         f2unpack(pp, p0, p1);
-                        pk[x] = pack2<T>(p0, p1);
+                        pk[x] = pack2<MT>(p0, p1);
                     }
                     // packed P columns 32h + 16cc .. +15 (keys 64h + 32cc ..)
                     tmem_st16x2_16<32>(scol + cc * 16, pk);
@@ -874,10 +970,21 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 reg_fence32(orr);
                 if (valid) {
                     uint32_t pk[16];
+                    if (I8 && a.v_mode == 0) {
+                        // per-channel V: the widened values carry the offset; the
+                        // scale multiplies each output channel here
+                        const float *vsc = a.v_scale + gm.kvh * D + DH * half + cc * 32;
 #pragma unroll
-                    for (int x = 0; x < 16; ++x)
-                        pk[x] = pack2<T>(__uint_as_float(orr[2 * x]) * oscale,
-                                         __uint_as_float(orr[2 * x + 1]) * oscale);
+                        for (int x = 0; x < 16; ++x)
+                            pk[x] = pack2<T>(__uint_as_float(orr[2 * x]) * (oscale * __ldg(vsc + 2 * x)),
+                                             __uint_as_float(orr[2 * x + 1]) *
+                                                 (oscale * __ldg(vsc + 2 * x + 1)));
+                    } else {
+#pragma unroll
+                        for (int x = 0; x < 16; ++x)
+                            pk[x] = pack2<T>(__uint_as_float(orr[2 * x]) * oscale,
+                                             __uint_as_float(orr[2 * x + 1]) * oscale);
+                    }
                     uint4 *dst = reinterpret_cast<uint4 *>(outp + orow * D + DH * half + cc * 32);
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
@@ -899,9 +1006,23 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         const int u = tid - 18 * 32;
         const int rl = u & 7;
         const int c = u >> 3;
-        uint32_t rk_it = 0, rv_it = 0, k_it = 0, v_it = 0;
+        uint32_t rk_it = 0, rv_it = 0, k_it = 0, v_it = 0, q_it = 0;
         for (idx = it_begin; idx < it_end; ++idx) {
             const PairGeom gm = pair_geom<BAND>(a, items, seqs, idx);
+            if (gm.nB > 0) {
+                // the pair's Q tiles, in place, to f16 (times the per-channel
+                // K scale); each warp converts half of the rows
+                dbg_j = -1;
+                FIA_WAIT_C(q_full, q_it & 1, 44);
+                ++q_it;
+                const float *ksc = a.k_mode == 0 ? a.k_scale + gm.kvh * D : nullptr;
+#pragma unroll 1
+                for (int x = 0; x < 2; ++x)
+                    if (gm.t[x].valid) q_to_f16<T>(smem + Cfg::kOffQ + x * Cfg::kTileBytes, u, ksc);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(q_conv);
+            }
             for (int s = 0; s <= gm.nB; ++s) {
 #pragma unroll 1
                 for (int h = 0; h < 2; ++h) {
@@ -927,21 +1048,22 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                     const float *sc = is_v ? a.v_scale : a.k_scale;
                     const float *of = is_v ? a.v_offset : a.k_offset;
                     if (tok) {
+                        // per token: (x + offset) * scale in f16
                         const int64_t row0 = (int64_t)gm.b * (is_v ? a.v_tok_stride : a.k_tok_stride) + t0;
                         if (valid == kPrefillBN)
-                            dequant_tile<T, true, true>(raw, dst, rl, c, valid, sc + row0,
-                                                        of ? of + row0 : nullptr);
-                        else
-                            dequant_tile<T, true, false>(raw, dst, rl, c, valid, sc + row0,
+                            dequant_tile<MT, true, true>(raw, dst, rl, c, valid, sc + row0,
                                                          of ? of + row0 : nullptr);
-                    } else {
-                        const int ch0 = gm.kvh * D + 16 * c;
-                        if (valid == kPrefillBN)
-                            dequant_tile<T, false, true>(raw, dst, rl, c, valid, sc + ch0,
-                                                         of ? of + ch0 : nullptr);
                         else
-                            dequant_tile<T, false, false>(raw, dst, rl, c, valid, sc + ch0,
-                                                          of ? of + ch0 : nullptr);
+                            dequant_tile<MT, true, false>(raw, dst, rl, c, valid, sc + row0,
+                                                          of ? of + row0 : nullptr);
+                    } else {
+                        // per channel: x + offset exactly widened; the scale is
+                        // folded into Q (keys) or applied in the epilogue (values)
+                        const int ch0 = gm.kvh * D + 16 * c;
+                        // (one instance per tile shape: a null offset adds zeros)
+                        const float *ofc = of ? of + ch0 : nullptr;
+                        if (valid == kPrefillBN) widen_tile<true, true>(raw, dst, rl, c, valid, ofc);
+                        else widen_tile<false, true>(raw, dst, rl, c, valid, ofc);
                     }
                     // the MMAs (async proxy) read what was stored here, and TMA
                     // refills the raw stage that was read here

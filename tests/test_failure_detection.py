@@ -26,11 +26,11 @@ LIMIT_NS = 1_000_000          # 1 ms
 SITE_DECODE_STALL = 3         # decode kernels: the hook's wait
 SITE_PREFILL_STALL = 35       # prefill softmax warps: the hook's wait
 # Prefill wait sites: producer 10-12, issuer 20-27, softmax warps 30-35, int8
-# converters 40-43.  With the softmax warps stalled, the issuer's wait for
+# converters 40-44.  With the softmax warps stalled, the issuer's wait for
 # their P (or a wait further up the pipeline) can run out first; each is a
 # time-out of a wait that nothing completed.
 PREFILL_SITES = (set(range(10, 13)) | set(range(20, 28)) | set(range(30, 36)) |
-                 set(range(40, 44)))
+                 set(range(40, 45)))
 
 CASES = {
     "decode_bf16": (dict(seq_len=[1, 1, 1], kv_seq_len=[900, 70, 3000], head_num=16,
