@@ -197,9 +197,9 @@ typedef struct fia_op fia_op;
  * Supported build limits: headSize in {64, 128} (128 with an int8 cache);
  * blockSize a multiple of 16, 16 <= blockSize <= 256; headNum <= 1024.
  * Everything else the pages allow returns FIA_ERR_UNSUPPORTED.  With an int8
- * cache and more than 16 query rows per KV head (seqLen * headNum / kvHeadNum)
- * the tensor-core path dequantises each K/V tile into the query dtype before
- * the products, so a dequantised value must lie in that dtype's range.
+ * cache on the tensor-core path (fia_path, below) the products run in f16:
+ * q * kScale (per-channel keys), the cache values plus their offsets, and
+ * per-token dequantised values must lie within f16 range (|v| < 65504).
  * nTokens == 0 returns FIA_OK with workspaceSize 0 and an op whose run is a no-op.
  */
 FIA_API fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key,
