@@ -8,7 +8,7 @@
 // (O, m, l), and a second kernel merges the splits with the lse rule of the
 // V3 "lse" bullet (max, rescaled exponent sums, log of the sum added back).
 //
-// Kernel 1 (one CTA per split unit (b, kvh, [t0, t1))).  K/V rows of the unit
+// Kernel 1 (one CTA per split unit (b, kvh, 16-row chunk, [t0, t1))).  K/V rows of the unit
 // stream through a ring of shared-memory tiles (64 keys each) filled by TMA:
 // one 3-D box per (block run, 128-byte column group), the physical row coming
 // from the block table, so every cached byte is fetched once, 128-byte
@@ -33,6 +33,8 @@
 // Kernel 2, fia_combine_kernel: one CTA per (b, kvh, row); merges the unit
 //   partials in fixed logical order (deterministic), adds the learnable sink
 //   to the denominator, applies int8 V dequantisation, writes out and lse.
+//   When every (b, kvh, chunk) has a single split the units apply the same
+//   rules themselves (finish_unit) and this kernel is not launched.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>

@@ -4,11 +4,15 @@
 // Phase 1 (fia_get_workspace_size) mirrors the first-phase call of the aclnn
 // FusedInferAttentionScore API and the ATB PrefixEncoder
 // GetWorkspaceSize call: it verifies the inputs and sizes the workspace.
-// seqLen / kvSeqLen are host arrays (PrefixEncoder table: "Host side"), so the
-// whole work decomposition is planned here, on the host:
-//   * decode path (max seqLen * g <= 16): split-KV units of whole 64-key
-//     tiles, sized so the grid fills the SMs several times, ordered longest
-//     first; one combine item per (sequence, kv head);
+// seqLen / kvSeqLen are host arrays (the PrefixEncoder parameter table puts
+// them on the host), so the whole work decomposition is planned here:
+//   * decode path (up to 16 rows -- new token x head of the group -- per KV
+//     head, or up to 128 with fewer than 64 new tokens; fia_ext.path may
+//     force either path): split-KV units of whole 64-key tiles and 16-row
+//     chunks (8 over an int8 cache past 16 rows), sized so the grid fills the
+//     SMs several times, ordered longest first; one combine item per
+//     (sequence, kv head, chunk), and no combine launch when every item has
+//     a single split;
 //   * prefill path: (sequence, 128-token tile, head) items, costed by the
 //     number of 128-key tiles they read, assigned longest-processing-time
 //     first to one persistent CTA per SM.
