@@ -325,6 +325,54 @@ __device__ __forceinline__ void umma_pv_qk(uint32_t o_col, uint32_t p_col, uint6
         : "memory");
 }
 
+// umma_pv_qk with one more QK^T K-step (descriptors qx / kx, accumulating)
+// before the commit: the ALiBi bias step.
+__device__ __forceinline__ void umma_pv_qk_x(uint32_t o_col, uint32_t p_col, uint64_t v0,
+                                             uint32_t idesc_pv, uint32_t acc, uint32_t s_col,
+                                             uint64_t q0, uint64_t k0, uint32_t idesc_qk,
+                                             uint64_t qx, uint64_t kx, uint64_t *bar) {
+    asm volatile(
+        "{\n\t.reg .pred p, t, z;\n\t.reg .b64 v, q, k;\n\t.reg .b32 pa;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.b32 t, %4, %4;\n\t"
+        "setp.ne.b32 z, %4, %4;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+        "add.s32 pa, %1, 8;\n\tadd.s64 v, %2, 128;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [pa], v, %3, t;\n\t"
+        "add.s32 pa, %1, 16;\n\tadd.s64 v, %2, 256;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [pa], v, %3, t;\n\t"
+        "add.s32 pa, %1, 24;\n\tadd.s64 v, %2, 384;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [pa], v, %3, t;\n\t"
+        "add.s32 pa, %1, 32;\n\tadd.s64 v, %2, 512;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [pa], v, %3, t;\n\t"
+        "add.s32 pa, %1, 40;\n\tadd.s64 v, %2, 640;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [pa], v, %3, t;\n\t"
+        "add.s32 pa, %1, 48;\n\tadd.s64 v, %2, 768;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [pa], v, %3, t;\n\t"
+        "add.s32 pa, %1, 56;\n\tadd.s64 v, %2, 896;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [pa], v, %3, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%5], %6, %7, %8, z;\n\t"
+        "add.s64 q, %6, 2;\n\tadd.s64 k, %7, 2;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%5], q, k, %8, t;\n\t"
+        "add.s64 q, %6, 4;\n\tadd.s64 k, %7, 4;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%5], q, k, %8, t;\n\t"
+        "add.s64 q, %6, 6;\n\tadd.s64 k, %7, 6;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%5], q, k, %8, t;\n\t"
+        "add.s64 q, %6, 1024;\n\tadd.s64 k, %7, 1024;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%5], q, k, %8, t;\n\t"
+        "add.s64 q, %6, 1026;\n\tadd.s64 k, %7, 1026;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%5], q, k, %8, t;\n\t"
+        "add.s64 q, %6, 1028;\n\tadd.s64 k, %7, 1028;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%5], q, k, %8, t;\n\t"
+        "add.s64 q, %6, 1030;\n\tadd.s64 k, %7, 1030;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%5], q, k, %8, t;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%5], %10, %11, %8, t;\n\t"
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%9];\n\t}"
+        ::"r"(o_col), "r"(p_col), "l"(v0), "r"(idesc_pv), "r"(acc), "r"(s_col), "l"(q0), "l"(k0),
+          "r"(idesc_qk), "r"(smem_u32(bar)), "l"(qx), "l"(kx)
+        : "memory");
+}
+
 // Arrive (once) on `bar` when every tcgen05 op this thread issued so far is done.
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -418,6 +466,13 @@ __host__ __device__ __forceinline__ constexpr uint32_t umma_desc_lo(uint32_t sme
 }
 __host__ __device__ __forceinline__ constexpr uint32_t umma_desc_hi_sw128(uint32_t sbo_bytes) {
     return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+}
+// High word for an unswizzled K-major operand (layout type 0): 8-row x
+// 16-byte core matrices, `sbo_bytes` between 8-row groups along M / N; the
+// low word's leading byte offset is the step between the two core matrices
+// of a 16-wide K-step.
+__host__ __device__ __forceinline__ constexpr uint32_t umma_desc_hi_none(uint32_t sbo_bytes) {
+    return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14);
 }
 static_assert(umma_desc_sw128(0x2A400u + 0x460u, 16384u, 1024u) ==
                   (((uint64_t)umma_desc_hi_sw128(1024u) << 32) |
@@ -591,6 +646,15 @@ template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16
     return __bfloat162float(v);
 }
 template <> __device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
+
+// v rounded (to nearest even) to T and back
+template <typename T> __device__ __forceinline__ float round_to(float v);
+template <> __device__ __forceinline__ float round_to<__nv_bfloat16>(float v) {
+    return __bfloat162float(__float2bfloat16_rn(v));
+}
+template <> __device__ __forceinline__ float round_to<__half>(float v) {
+    return __half2float(__float2half_rn(v));
+}
 
 // 128-byte swizzle (16-byte chunk index XOR row-in-8) for a 1024-aligned region
 // of 128-byte rows.

@@ -5,7 +5,10 @@
 
 namespace fia {
 
-enum { kModePlain = 0, kModeAlibi = 1, kModePse = 2 };
+// kModeAlibiMma: the ALiBi bias inside a key tile added by one extra K-step
+// of the QK^T MMA (16-bit cache, positive qkScale); kModeAlibi adds it in
+// the softmax (int8 cache, or any scale)
+enum { kModePlain = 0, kModeAlibi = 1, kModePse = 2, kModeAlibiMma = 3 };
 
 struct SubGeom {
     bool valid;

@@ -77,7 +77,14 @@ struct PrefillCfg {
     static constexpr int kOffPse = kOffV + kVStages * kTileBytes;
     static constexpr int kPseBytes = (MODE == kModePse) ? 16 * 4096 : 0;
     static constexpr int kOffRaw = kOffPse + kPseBytes;      // raw K[RS], raw V[RS]
-    static constexpr int kOffBar = kOffRaw + 2 * kRawStages * kRawBytes;
+    // kModeAlibiMma: the bias operands of the extra QK^T K-step, unswizzled
+    // K-major 8-row x 16-byte core matrices: per tile of the pair the Q side
+    // (one core matrix shared by all 16 row groups, then a zero one for K
+    // columns 8..15), then the K side (16 groups of 8 key rows, each group's
+    // core matrix followed by its zero one)
+    static constexpr int kOffExt = kOffRaw + 2 * kRawStages * kRawBytes;
+    static constexpr int kExtBytes = (MODE == kModeAlibiMma) ? 2 * 256 + 2 * 2048 : 0;
+    static constexpr int kOffBar = kOffExt + kExtBytes;
     static_assert(kOffRaw % 1024 == 0, "swizzled TMA destinations are 1024-byte aligned");
     // q_full, q_empty, k_full/k_empty[KS], v_full/v_empty[VS],
     // s_full[2], p_full[2], o_full[2], pse_full[16], vz_full,
@@ -315,6 +322,10 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     // int8 cache: the products run in f16 (Q, the widened K / V and P)
     using MT = std::conditional_t<I8, __half, T>;
     constexpr bool BF = MmaType<MT>::bf16;
+    // ALiBi through the MMA: S gains slope / qkScale * (t - t0) for key t of a
+    // tile starting at key t0, the rest of the bias is one constant per row
+    constexpr bool XB = (MODE == kModeAlibiMma);
+    static_assert(!XB || !I8, "the bias K-step is for 16-bit caches");
     constexpr uint32_t IDESC_QK = umma_idesc_f16(BF, false, false, 128, kPrefillBN);
     constexpr uint32_t IDESC_PV = umma_idesc_f16(BF, false, true, 128, D);
 
@@ -388,6 +399,25 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         tmem_alloc(tmem_slot, Cfg::kTmemCols);
         tmem_relinquish();
     }
+    if constexpr (XB) {
+        // bias operands (16-byte rows): [0, 8) / [16, 24) Q side of tiles 0 / 1
+        // (written per item by the producer), [8, 16) / [24, 32) zeros; then
+        // per group of 8 keys 8 rows x = (x, x, x, 0 ...) -- the column offset
+        // inside the key tile, exact in 16 bits, meeting the three parts of the
+        // slope -- and 8 zero rows
+        uint4 *ext = reinterpret_cast<uint4 *>(smem + Cfg::kOffExt);
+        for (int r16 = tid; r16 < 288; r16 += Cfg::kThreads) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            const int L = r16 - 32;
+            if (L >= 0 && (L & 15) < 8) {
+                const float xv = (float)((L >> 4) * 8 + (L & 15));
+                v.x = pack2<MT>(xv, xv);
+                v.y = pack2<MT>(xv, 0.f);
+            }
+            ext[r16] = v;
+        }
+        fence_proxy_async_smem();
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -417,6 +447,24 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 const PairGeom gm = pair_geom<BAND>(a, items, seqs, idx);
                 if (gm.nB == 0) continue;
                 FIA_WAIT(q_empty, (req_q & 1) ^ 1, 10);
+                if constexpr (XB) {
+                    // Q side of the bias step: slope / qkScale (log2 units over
+                    // the scale folded into the exponent) as the sum of three
+                    // 16-bit parts, in each of the 8 rows of the shared core matrix
+#pragma unroll
+                    for (int x = 0; x < 2; ++x) {
+                        if (!gm.t[x].valid) continue;
+                        const float sv = a.c.slopes[gm.t[x].h] * kLog2e / a.c.scale_log2;
+                        const float s0 = round_to<MT>(sv);
+                        const float s1 = round_to<MT>(sv - s0);
+                        const float s2 = sv - s0 - s1;
+                        const uint32_t w0 = pack2<MT>(s0, s1), w1 = pack2<MT>(s2, 0.f);
+                        const uint32_t qx = smem_u32(smem + Cfg::kOffExt + x * 256);
+#pragma unroll
+                        for (int r8 = 0; r8 < 8; ++r8) sts128(qx + r8 * 16, w0, w1, 0u, 0u);
+                    }
+                    fence_proxy_async_smem();
+                }
                 mbar_arrive_expect_tx(q_full, (gm.t[0].valid ? 2 : 1) * Cfg::kTileBytes);
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
@@ -524,9 +572,20 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) d[kk] = tmem + Cfg::col_s(x) + kk * 8;
         };
+        // bias step operands: tile x's Q side (every 8-row group reads the
+        // same core matrix: stride 0), the key-column side (8-key groups 256
+        // bytes apart); each K-step's second core matrix 128 bytes on
+        const uint32_t sm_ext = smem_u32(smem + Cfg::kOffExt);
+        auto qxd = [&](int x) {
+            return ((uint64_t)umma_desc_hi_none(0) << 32) | umma_desc_lo(sm_ext + x * 256, 128);
+        };
+        auto kxd = [&]() {
+            return ((uint64_t)umma_desc_hi_none(256) << 32) | umma_desc_lo(sm_ext + 512, 128);
+        };
         auto qk = [&](int x, const uint64_t (&qd)[NKQ], const uint64_t (&kd)[NKQ]) {
             if constexpr (NKQ == 8) umma_ss_x8(tmem + Cfg::col_s(x), qd, kd, IDESC_QK, 0u);
             else umma_ss_x4(tmem + Cfg::col_s(x), qd, kd, IDESC_QK, 0u);
+            if constexpr (XB) umma_ss(tmem + Cfg::col_s(x), qxd(x), kxd(), IDESC_QK, 1u);
         };
         static_assert(kPrefillBN / 16 == 8, "PV issue assumes 8 key steps per tile");
         static_assert(NKQ == 4 || NKQ == 8, "QK issue assumes D = 64 or 128");
@@ -596,9 +655,14 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                         tc_fence_after();
                         if constexpr (NKQ == 8) {
                             if (j + 1 < gm.nA) {
-                                umma_pv_qk(tmem + Cfg::col_o(0), tmem + Cfg::col_s(0), vd[0],
-                                           IDESC_PV, j > 0 ? 1u : 0u, tmem + Cfg::col_s(0), q0d,
-                                           kd[0], IDESC_QK, &s_full[0]);
+                                if constexpr (XB)
+                                    umma_pv_qk_x(tmem + Cfg::col_o(0), tmem + Cfg::col_s(0), vd[0],
+                                                 IDESC_PV, j > 0 ? 1u : 0u, tmem + Cfg::col_s(0),
+                                                 q0d, kd[0], IDESC_QK, qxd(0), kxd(), &s_full[0]);
+                                else
+                                    umma_pv_qk(tmem + Cfg::col_o(0), tmem + Cfg::col_s(0), vd[0],
+                                               IDESC_PV, j > 0 ? 1u : 0u, tmem + Cfg::col_s(0), q0d,
+                                               kd[0], IDESC_QK, &s_full[0]);
                             } else {
                                 ptmem(0, pa);
                                 umma_ts_x8(tmem + Cfg::col_o(0), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
@@ -620,9 +684,14 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                     ++p_it[1];
                     tc_fence_after();
                     if (NKQ == 8 && more) {
-                        umma_pv_qk(tmem + Cfg::col_o(1), tmem + Cfg::col_s(1), vd[0], IDESC_PV,
-                                   j > 0 ? 1u : 0u, tmem + Cfg::col_s(1), q1d, kd[0], IDESC_QK,
-                                   &s_full[1]);
+                        if constexpr (XB)
+                            umma_pv_qk_x(tmem + Cfg::col_o(1), tmem + Cfg::col_s(1), vd[0], IDESC_PV,
+                                         j > 0 ? 1u : 0u, tmem + Cfg::col_s(1), q1d, kd[0], IDESC_QK,
+                                         qxd(1), kxd(), &s_full[1]);
+                        else
+                            umma_pv_qk(tmem + Cfg::col_o(1), tmem + Cfg::col_s(1), vd[0], IDESC_PV,
+                                       j > 0 ? 1u : 0u, tmem + Cfg::col_s(1), q1d, kd[0], IDESC_QK,
+                                       &s_full[1]);
                     } else {
                         ptmem(1, pa);
                         kmajor(q_lo + kTileStep, qd);
@@ -696,7 +765,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         const float sl2 = a.c.scale_log2;
         // plain mode with a positive scale: mask raw scores and fold the scale
         // into the exponent (one FFMA per element)
-        const bool fold = (MODE == kModePlain) && (sl2 > 0.f);
+        const bool fold = (MODE == kModePlain || XB) && (sl2 > 0.f);
         uint32_t s_it = 0, p_it = 0, o_it = 0;
         T *outp = reinterpret_cast<T *>(a.c.out);
         const bool pse_tma = (MODE == kModePse) && a.c.pse_tma;
@@ -742,7 +811,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 continue;
             }
             float slope2 = 0.f;
-            if constexpr (MODE == kModeAlibi) slope2 = a.c.slopes[sg.h] * kLog2e;
+            if constexpr (MODE == kModeAlibi || XB) slope2 = a.c.slopes[sg.h] * kLog2e;
             const T *pse_row = nullptr;
             if constexpr (MODE == kModePse) {
                 // rows past seqLen read row 0 of the sequence (their output is dropped)
@@ -880,6 +949,13 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 float mx = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
                 if (fold) mx = (mx == -INFINITY) ? -INFINITY : mx * sl2;
+                // bias step mode: S holds slope * (t - t0) of the tile's first key
+                // t0; slope * (t0 - qpos) is the same for the whole row of the tile
+                float cb = 0.f;
+                if constexpr (XB) {
+                    cb = slope2 * (float)((gm.j0 + j) * kPrefillBN - qpos);
+                    mx += cb;
+                }
 
                 // running max: exact on the first tile, afterwards raised only
                 // when it grows by more than 2^8 (O and l stay consistent with m)
@@ -897,7 +973,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 const float mu = (m == -INFINITY) ? 0.f : m;
 
                 // P = 2^(s - m) in the input dtype over this lane's half row
-                const uint64_t negmu2 = f2pack(-mu, -mu);
+                const uint64_t negmu2 = f2pack(cb - mu, cb - mu);
                 const uint64_t sl2x2 = f2pack(sl2, sl2);
                 uint64_t acc2[4];
 #pragma unroll
@@ -1165,8 +1241,13 @@ static cudaError_t launch_prefill_mode(const PrefillArgs &a, const CUtensorMap &
         return launch_prefill_t<T, D, kModePlain, true, I8>(a, tq, tk, tv, tp, grid, ip, s);
     }
     if (a.c.pse) return launch_prefill_t<T, D, kModePse, false, I8>(a, tq, tk, tv, tp, grid, ip, s);
-    if (a.c.mask_type == 3)
+    if (a.c.mask_type == 3) {
+        if constexpr (!I8) {
+            if (a.c.scale_log2 > 0.f)
+                return launch_prefill_t<T, D, kModeAlibiMma, false, I8>(a, tq, tk, tv, tp, grid, ip, s);
+        }
         return launch_prefill_t<T, D, kModeAlibi, false, I8>(a, tq, tk, tv, tp, grid, ip, s);
+    }
     return launch_prefill_t<T, D, kModePlain, false, I8>(a, tq, tk, tv, tp, grid, ip, s);
 }
 

@@ -116,6 +116,18 @@ PREFILL_CASES = {
                             mask_type=W.MASK_ALIBI, alibi_slopes=True),
     "bs48_pse_causal": dict(seq_len=[150], kv_seq_len=[200], head_num=4, kv_head_num=2,
                             head_size=128, block_size=48, mask_type=W.MASK_CAUSAL, pse=True),
+    # ALiBi with the in-tile bias as an extra QK^T K-step: GQA pairs whose two
+    # tiles carry different heads' slopes, a long prefix (biases in the
+    # hundreds), D = 64; a negative qkScale takes the softmax-side bias instead
+    "alibi_gqa_long_prefix_bf16": dict(seq_len=[200, 64], kv_seq_len=[2300, 64], head_num=8,
+                                       kv_head_num=2, head_size=128, block_size=64,
+                                       mask_type=W.MASK_ALIBI, alibi_slopes=True),
+    "alibi_d64_gqa_f16": dict(seq_len=[130, 260], kv_seq_len=[400, 260], head_num=8,
+                              kv_head_num=4, head_size=64, block_size=32, dtype="f16",
+                              mask_type=W.MASK_ALIBI, alibi_slopes=True),
+    "alibi_negative_scale_f16": dict(seq_len=[150], kv_seq_len=[300], head_num=4, kv_head_num=4,
+                                     head_size=128, block_size=64, dtype="f16", qk_scale=-0.05,
+                                     mask_type=W.MASK_ALIBI, alibi_slopes=True),
 }
 
 
