@@ -642,6 +642,15 @@ fia_status fia_get_workspace_size(const fia_tensor *query, const fia_tensor *key
             per[l.second].push_back(cd.it);
             heap.push({l.first + cd.cost, l.second});
         }
+        // A CTA's total, hence the makespan, does not depend on the order of its
+        // items.  Ordered by (sequence, KV head), every CTA sweeps the KV heads
+        // at about the same pace, so the K/V tiles in use at any moment are
+        // those of a few heads and stay in L2 between their items (longest
+        // first, the items of all heads run at once and K/V is re-read).
+        for (auto &v : per)
+            std::stable_sort(v.begin(), v.end(), [](const PrefillItem &x, const PrefillItem &y) {
+                return x.b != y.b ? x.b < y.b : x.kvh < y.kvh;
+            });
         std::vector<int32_t> cta_off(grid + 1, 0);
         std::vector<PrefillItem> flat;
         flat.reserve(items.size());
