@@ -477,7 +477,8 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 const int32_t *bt_row = a.c.bt + (int64_t)gm.b * a.c.bt_stride;
                 for (int j = 0; j < gm.nB; ++j) {
                     dbg_j = j;
-                    const int t0 = (gm.j0 + j) * kPrefillBN;
+                    // key tiles last to first in the ALiBi-through-MMA mode
+                    const int t0 = (XB ? gm.j0 + gm.nB - 1 - j : gm.j0 + j) * kPrefillBN;
                     const int t1 = min(t0 + kPrefillBN, gm.kvlen);
                     const int nbox = (t1 - t0 + br - 1) / br;
                     const uint32_t bytes = (uint32_t)(nbox * br * 128 * Cfg::kHalves);
@@ -600,13 +601,20 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             FIA_WAIT(I8 ? q_conv : q_full, q_it & 1, 20);
             ++q_it;
             const uint32_t kv_base = kv_it;
+            // Tile 0 takes part in iterations [a0, a0 + nA).  Key tiles run
+            // first to last (a0 = 0), or in the ALiBi-through-MMA mode last to
+            // first, where tile 0's fewer key tiles are the last iterations:
+            // the diagonal tile, whose bias is the largest, then fixes the
+            // running maximum and the lazy O rescale is rarely needed.
+            const int a0 = XB ? gm.nB - gm.nA : 0;
+            auto t0_on = [&](int jj) { return jj >= a0 && jj < a0 + gm.nA; };
             {
                 // QK for key tile 0 (both tiles)
                 const int ks = kv_base % KS;
                 kmajor(k_lo + ks * kTileStep, kd);
                 FIA_WAIT(&k_full[ks], (kv_base / KS) & 1, 21);
                 tc_fence_after();
-                if (gm.nA > 0) {
+                if (gm.nA > 0 && a0 == 0) {
                     kmajor(q_lo, qd);
                     qk(0, qd, kd);
                     umma_commit(&s_full[0]);
@@ -627,7 +635,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 vmajor(v_lo + vs * kTileStep, vd);
                 kmajor(k_lo + ksn * kTileStep, kd);
                 FIA_WAIT(&v_full[vs], (kvi / VS) & 1, 24);
-                const int valid = gm.kvlen - (gm.j0 + j) * kPrefillBN;
+                const int valid = gm.kvlen - (XB ? gm.j0 + gm.nB - 1 - j : gm.j0 + j) * kPrefillBN;
                 if (!I8 && valid < kPrefillBN) {     // (int8: the converters write the zeros)
                     // rows past kvSeqLen: P is 0 there, but the slots may hold
                     // anything (NaN * 0 = NaN in the MMA): the bulk-copy engine
@@ -649,36 +657,43 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                     // QK_X(j+1) is issued after PV_X(j), so its S-ready commit also
                     // tells the softmax warps that PV_X(j) is done with O.
                     if (more) FIA_WAIT(&k_full[ksn], (kn / KS) & 1, 22);
-                    if (j < gm.nA) {
+                    if (t0_on(j)) {
                         FIA_WAIT(&p_full[0], p_it[0] & 1, 23);
                         ++p_it[0];
                         tc_fence_after();
+                        const uint32_t acc0 = j > a0 ? 1u : 0u;
                         if constexpr (NKQ == 8) {
-                            if (j + 1 < gm.nA) {
+                            if (t0_on(j + 1)) {
                                 if constexpr (XB)
                                     umma_pv_qk_x(tmem + Cfg::col_o(0), tmem + Cfg::col_s(0), vd[0],
-                                                 IDESC_PV, j > 0 ? 1u : 0u, tmem + Cfg::col_s(0),
+                                                 IDESC_PV, acc0, tmem + Cfg::col_s(0),
                                                  q0d, kd[0], IDESC_QK, qxd(0), kxd(), &s_full[0]);
                                 else
                                     umma_pv_qk(tmem + Cfg::col_o(0), tmem + Cfg::col_s(0), vd[0],
-                                               IDESC_PV, j > 0 ? 1u : 0u, tmem + Cfg::col_s(0), q0d,
+                                               IDESC_PV, acc0, tmem + Cfg::col_s(0), q0d,
                                                kd[0], IDESC_QK, &s_full[0]);
                             } else {
                                 ptmem(0, pa);
-                                umma_ts_x8(tmem + Cfg::col_o(0), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
+                                umma_ts_x8(tmem + Cfg::col_o(0), pa, vd, IDESC_PV, acc0);
                                 umma_commit(&o_full[0]);
                             }
                         } else {
                             ptmem(0, pa);
                             kmajor(q_lo, qd);
-                            umma_ts_x8(tmem + Cfg::col_o(0), pa, vd, IDESC_PV, j > 0 ? 1u : 0u);
-                            if (j + 1 < gm.nA) {
+                            umma_ts_x8(tmem + Cfg::col_o(0), pa, vd, IDESC_PV, acc0);
+                            if (t0_on(j + 1)) {
                                 qk(0, qd, kd);
                                 umma_commit(&s_full[0]);
                             } else {
                                 umma_commit(&o_full[0]);
                             }
                         }
+                    } else if (t0_on(j + 1)) {
+                        // tile 0's first key tile is the next one (reverse order)
+                        tc_fence_after();
+                        kmajor(q_lo, qd);
+                        qk(0, qd, kd);
+                        umma_commit(&s_full[0]);
                     }
                     FIA_WAIT(&p_full[1], p_it[1] & 1, 25);
                     ++p_it[1];
@@ -822,7 +837,9 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             if (pse_tma) pse_fetch(gm, sg, 0);
             for (int j = 0; j < sg.n; ++j) {
                 dbg_j = j;
-                const int tb = (gm.j0 + j) * kPrefillBN + 64 * half;   // first key of this lane
+                // this tile's key tile (last to first in the ALiBi-through-MMA mode)
+                const int kt = XB ? gm.j0 + sg.n - 1 - j : gm.j0 + j;
+                const int tb = kt * kPrefillBN + 64 * half;            // first key of this lane
                 FIA_WAIT_W(&s_full[X], s_it & 1, 30);
                 ++s_it;
                 __syncwarp();          // tcgen05.ld/st below are warp-collective (.aligned)
@@ -953,7 +970,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 // t0; slope * (t0 - qpos) is the same for the whole row of the tile
                 float cb = 0.f;
                 if constexpr (XB) {
-                    cb = slope2 * (float)((gm.j0 + j) * kPrefillBN - qpos);
+                    cb = slope2 * (float)(kt * kPrefillBN - qpos);
                     mx += cb;
                 }
 
@@ -962,7 +979,8 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 const float m_new = fmaxf(m, mx);
                 bool need = false;
                 float alpha = 1.0f;
-                if (j == 0) {
+                if (j == 0 || m == -INFINITY) {
+                    // (no key seen yet: O and l are exact zeros, nothing to rescale)
                     m = m_new;
                 } else if (m_new > m + 8.0f) {
                     need = true;
