@@ -326,6 +326,13 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     // tile starting at key t0, the rest of the bias is one constant per row
     constexpr bool XB = (MODE == kModeAlibiMma);
     static_assert(!XB || !I8, "the bias K-step is for 16-bit caches");
+    // Instances whose pairs end both tiles on the same key tile (band: GQA
+    // pairs or single tiles; ALiBi through the MMA: key tiles last to first)
+    // run an item's epilogue inside the next item's first key tile and send
+    // that item's first QK_0 early.  Elsewhere (first-to-last MHA pairs, whose
+    // tile 0 ends a key tile early and hides its epilogue there; pse and int8,
+    // short of registers) the epilogue follows the item at once.
+    constexpr bool DEFER = (BAND || XB) && !I8 && MODE != kModePse;
     constexpr uint32_t IDESC_QK = umma_idesc_f16(BF, false, false, 128, kPrefillBN);
     constexpr uint32_t IDESC_PV = umma_idesc_f16(BF, false, true, 128, D);
 
@@ -547,6 +554,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         // precedes it.
         if (lane != 0) goto done;
         uint32_t q_it = 0, kv_it = 0, p_it[2] = {0, 0};
+        bool qk0_early = false;     // the next item's first QK_0 went out already
         constexpr int NKQ = D / 16;                     // K-steps of QK^T
         constexpr uint32_t kHi = umma_desc_hi_sw128(1024);
         constexpr uint32_t kTileStep = Cfg::kTileBytes >> 4;
@@ -588,6 +596,33 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             else umma_ss_x4(tmem + Cfg::col_s(x), qd, kd, IDESC_QK, 0u);
             if constexpr (XB) umma_ss(tmem + Cfg::col_s(x), qxd(x), kxd(), IDESC_QK, 1u);
         };
+        // At the last key tile of an item whose two tiles end together, the
+        // next item's first QK_0 goes out right after PV_0 instead of after
+        // tile 1's last P, so tile 0's softmax warps can start the next item
+        // (its epilogue follows that item's first tile).  Its inputs cannot
+        // wait on anything issued later: the next Q was requested once this
+        // item's last QK finished, and the next K tile takes the stage of
+        // K(nB - 2), freed before that.  (int8: the converted Q has its own
+        // barrier; not done there.)  Returns false if a wait gave up.
+        auto qk0_next = [&](const PairGeom &g0, uint64_t (&qd)[NKQ], uint64_t (&kd)[NKQ]) -> bool {
+            if constexpr (!DEFER) return true;
+            if (idx + 1 >= it_end) return true;
+            const PairGeom gn = pair_geom<BAND>(a, items, seqs, idx + 1);
+            if (gn.nB == 0 || gn.nA == 0) return true;
+            if (XB && gn.nA != gn.nB) return true;      // its tile 0 starts later
+            const uint32_t k0 = kv_it + g0.nB;
+            const int ks0 = k0 % KS;
+            kmajor(k_lo + ks0 * kTileStep, kd);
+            if (!mbar_wait(q_full, q_it & 1, abort_flag, a.c.err, 20, a.c.wait_ns)) return false;
+            if (!mbar_wait(&k_full[ks0], (k0 / KS) & 1, abort_flag, a.c.err, 21, a.c.wait_ns))
+                return false;
+            tc_fence_after();
+            kmajor(q_lo, qd);
+            qk(0, qd, kd);
+            umma_commit(&s_full[0]);
+            qk0_early = true;
+            return true;
+        };
         static_assert(kPrefillBN / 16 == 8, "PV issue assumes 8 key steps per tile");
         static_assert(NKQ == 4 || NKQ == 8, "QK issue assumes D = 64 or 128");
         for (idx = it_begin; idx < it_end; ++idx) {
@@ -614,11 +649,12 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 kmajor(k_lo + ks * kTileStep, kd);
                 FIA_WAIT(&k_full[ks], (kv_base / KS) & 1, 21);
                 tc_fence_after();
-                if (gm.nA > 0 && a0 == 0) {
+                if (gm.nA > 0 && a0 == 0 && !qk0_early) {
                     kmajor(q_lo, qd);
                     qk(0, qd, kd);
                     umma_commit(&s_full[0]);
                 }
+                qk0_early = false;
                 kmajor(q_lo + kTileStep, qd);
                 qk(1, qd, kd);
                 umma_commit(&s_full[1]);
@@ -676,6 +712,10 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                                 ptmem(0, pa);
                                 umma_ts_x8(tmem + Cfg::col_o(0), pa, vd, IDESC_PV, acc0);
                                 umma_commit(&o_full[0]);
+                                if (!more && !qk0_next(gm, qd, kd)) {
+                                    fail_trail(a.c.err, 20, (uint32_t)idx, (uint32_t)dbg_j, q_it & 1, q_full);
+                                    goto done;
+                                }
                             }
                         } else {
                             ptmem(0, pa);
@@ -686,6 +726,10 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                                 umma_commit(&s_full[0]);
                             } else {
                                 umma_commit(&o_full[0]);
+                                if (!more && !qk0_next(gm, qd, kd)) {
+                                    fail_trail(a.c.err, 20, (uint32_t)idx, (uint32_t)dbg_j, q_it & 1, q_full);
+                                    goto done;
+                                }
                             }
                         }
                     } else if (t0_on(j + 1)) {
@@ -797,6 +841,75 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                     tma_load_3d(pslot + hh * 2048, &tp, pbar, (g2.j0 + jt) * kPrefillBN + 64 * hh,
                                 s2.q0 + 32 * quad + 16 * sub, g2.b * a.c.H + s2.h);
             }
+        };
+
+        // Epilogue of a finished item -- O / l (+ sink), lse; each lane writes
+        // D/2 columns -- from the state the item left (ep_h < 0: none pending).
+        // DEFER: it runs after the next item's first P is in TMEM and before
+        // that P is signalled: the PV that overwrites O waits for the signal,
+        // and the softmax of the new item's first tile overlaps the wait for
+        // the old item's last PV instead of following the epilogue.  Returns
+        // false if the wait for that PV gave up (the caller takes the error exit).
+        float ep_m = 0.f, ep_l = 0.f;
+        int ep_row = -1, ep_h = -1, ep_kvh = 0;
+        auto epilogue = [&]() -> bool {
+            const bool got = mbar_wait(&o_full[X], o_it & 1, abort_flag, a.c.err, 32, a.c.wait_ns);
+            if (!__all_sync(0xffffffffu, got)) {
+                if (lane == 0) fail_trail(a.c.err, 32, (uint32_t)idx, (uint32_t)dbg_j, o_it & 1, &o_full[X]);
+                tmem_st_wait();
+                return false;
+            }
+            ++o_it;
+            __syncwarp();
+            tc_fence_after();
+            const float mu = (ep_m == -INFINITY) ? 0.f : ep_m;
+            float M = mu, lt = ep_l;
+            if (a.c.sink) {
+                const float s2 = a.c.sink[ep_h] * kLog2e;
+                M = fmaxf(mu, s2);
+                lt = ep_l * ex2(mu - M) + ex2(s2 - M);
+            }
+            // a row with no visible key (possible under a band mask): out 0,
+            // lse +inf, with or without a sink
+            const bool no_key = BAND && (ep_m == -INFINITY);
+            const float oscale = no_key ? 0.f : ex2(mu - M) / lt;
+            const int64_t orow = (int64_t)ep_row * a.c.H + ep_h;
+#pragma unroll
+            for (int cc = 0; cc < DH / 32; ++cc) {
+                uint32_t orr[32];
+                tmem_ld16x2_32<DH>(ocol + cc * 32, orr);
+                tmem_ld_wait();
+                reg_fence32(orr);
+                if (ep_row >= 0) {
+                    uint32_t pk[16];
+                    if (I8 && a.v_mode == 0) {
+                        // per-channel V: the widened values carry the offset; the
+                        // scale multiplies each output channel here
+                        const float *vsc = a.v_scale + ep_kvh * D + DH * half + cc * 32;
+#pragma unroll
+                        for (int x = 0; x < 16; ++x)
+                            pk[x] = pack2<T>(__uint_as_float(orr[2 * x]) * (oscale * __ldg(vsc + 2 * x)),
+                                             __uint_as_float(orr[2 * x + 1]) *
+                                                 (oscale * __ldg(vsc + 2 * x + 1)));
+                    } else {
+#pragma unroll
+                        for (int x = 0; x < 16; ++x)
+                            pk[x] = pack2<T>(__uint_as_float(orr[2 * x]) * oscale,
+                                             __uint_as_float(orr[2 * x + 1]) * oscale);
+                    }
+                    uint4 *dst = reinterpret_cast<uint4 *>(outp + orow * D + DH * half + cc * 32);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                }
+                __syncwarp();
+            }
+            if (ep_row >= 0 && a.c.lse && half == 0)
+                a.c.lse[orow] = no_key ? INFINITY : (M + log2f(lt)) * kLn2;
+            tc_fence_before();
+            __syncwarp();
+            ep_h = -1;
+            return true;
         };
 
         // test hook: wait on a barrier nothing signals, so the bounded wait
@@ -1044,62 +1157,25 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
+                if (DEFER && j == 0 && ep_h >= 0 && !epilogue()) goto done;
                 if (lane == 0) mbar_arrive(&p_full[X]);
                 ++p_it;
             }
 
-            // ---- epilogue: O / l (+ sink), lse; each lane writes D/2 columns ----
+            // DEFER: the item's epilogue runs inside the next item's first key
+            // tile (or after the last item); its state waits here
             dbg_j = sg.n;
             l += __shfl_xor_sync(0xffffffffu, l, 16);
-            FIA_WAIT_W(&o_full[X], o_it & 1, 32);
-            ++o_it;
-            __syncwarp();
-            tc_fence_after();
-            const float mu = (m == -INFINITY) ? 0.f : m;
-            float M = mu, lt = l;
-            if (a.c.sink) {
-                const float s2 = a.c.sink[sg.h] * kLog2e;
-                M = fmaxf(mu, s2);
-                lt = l * ex2(mu - M) + ex2(s2 - M);
+            ep_m = m;
+            ep_l = l;
+            ep_row = valid ? gm.cu_q + i : -1;
+            ep_h = sg.h;
+            ep_kvh = gm.kvh;
+            if constexpr (!DEFER) {
+                if (!epilogue()) goto done;
             }
-            // a row with no visible key (possible under a band mask): out 0,
-            // lse +inf, with or without a sink
-            const bool no_key = BAND && (m == -INFINITY);
-            const float oscale = no_key ? 0.f : ex2(mu - M) / lt;
-#pragma unroll
-            for (int cc = 0; cc < DH / 32; ++cc) {
-                uint32_t orr[32];
-                tmem_ld16x2_32<DH>(ocol + cc * 32, orr);
-                tmem_ld_wait();
-                reg_fence32(orr);
-                if (valid) {
-                    uint32_t pk[16];
-                    if (I8 && a.v_mode == 0) {
-                        // per-channel V: the widened values carry the offset; the
-                        // scale multiplies each output channel here
-                        const float *vsc = a.v_scale + gm.kvh * D + DH * half + cc * 32;
-#pragma unroll
-                        for (int x = 0; x < 16; ++x)
-                            pk[x] = pack2<T>(__uint_as_float(orr[2 * x]) * (oscale * __ldg(vsc + 2 * x)),
-                                             __uint_as_float(orr[2 * x + 1]) *
-                                                 (oscale * __ldg(vsc + 2 * x + 1)));
-                    } else {
-#pragma unroll
-                        for (int x = 0; x < 16; ++x)
-                            pk[x] = pack2<T>(__uint_as_float(orr[2 * x]) * oscale,
-                                             __uint_as_float(orr[2 * x + 1]) * oscale);
-                    }
-                    uint4 *dst = reinterpret_cast<uint4 *>(outp + orow * D + DH * half + cc * 32);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-                }
-                __syncwarp();
-            }
-            if (valid && a.c.lse && half == 0) a.c.lse[orow] = no_key ? INFINITY : (M + log2f(lt)) * kLn2;
-            tc_fence_before();
-            __syncwarp();
         }
+        if (DEFER && ep_h >= 0 && !epilogue()) goto done;
     } else if constexpr (I8) {
         // ------------------------------------------------------------ int8 converters
         // Eight consecutive threads take eight consecutive rows of one 16-byte
