@@ -7,8 +7,10 @@ namespace fia {
 
 // kModeAlibiMma: the ALiBi bias inside a key tile added by one extra K-step
 // of the QK^T MMA (16-bit cache, positive qkScale); kModeAlibi adds it in
-// the softmax (int8 cache, or any scale)
-enum { kModePlain = 0, kModeAlibi = 1, kModePse = 2, kModeAlibiMma = 3 };
+// the softmax (int8 cache, or any scale).  kModePlainGqa: kModePlain for GQA
+// (g >= 2) over a 16-bit cache, whose pairs end both tiles on the same key
+// tile.
+enum { kModePlain = 0, kModeAlibi = 1, kModePse = 2, kModeAlibiMma = 3, kModePlainGqa = 4 };
 
 struct SubGeom {
     bool valid;

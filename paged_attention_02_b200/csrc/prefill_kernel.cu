@@ -326,13 +326,13 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
     // tile starting at key t0, the rest of the bias is one constant per row
     constexpr bool XB = (MODE == kModeAlibiMma);
     static_assert(!XB || !I8, "the bias K-step is for 16-bit caches");
-    // Instances whose pairs end both tiles on the same key tile (band: GQA
-    // pairs or single tiles; ALiBi through the MMA: key tiles last to first)
-    // run an item's epilogue inside the next item's first key tile and send
-    // that item's first QK_0 early.  Elsewhere (first-to-last MHA pairs, whose
-    // tile 0 ends a key tile early and hides its epilogue there; pse and int8,
-    // short of registers) the epilogue follows the item at once.
-    constexpr bool DEFER = (BAND || XB) && !I8 && MODE != kModePse;
+    // Instances whose pairs end both tiles on the same key tile (GQA pairs,
+    // band: GQA pairs or single tiles; ALiBi through the MMA: key tiles last
+    // to first) run an item's epilogue inside the next item's first key tile
+    // and send that item's first QK_0 early.  Elsewhere (first-to-last MHA
+    // pairs, whose tile 0 ends a key tile early and hides its epilogue there;
+    // pse and int8, short of registers) the epilogue follows the item at once.
+    constexpr bool DEFER = (BAND || XB || MODE == kModePlainGqa) && !I8 && MODE != kModePse;
     constexpr uint32_t IDESC_QK = umma_idesc_f16(BF, false, false, 128, kPrefillBN);
     constexpr uint32_t IDESC_PV = umma_idesc_f16(BF, false, true, 128, D);
 
@@ -824,7 +824,7 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
         const float sl2 = a.c.scale_log2;
         // plain mode with a positive scale: mask raw scores and fold the scale
         // into the exponent (one FFMA per element)
-        const bool fold = (MODE == kModePlain || XB) && (sl2 > 0.f);
+        const bool fold = (MODE == kModePlain || MODE == kModePlainGqa || XB) && (sl2 > 0.f);
         uint32_t s_it = 0, p_it = 0, o_it = 0;
         T *outp = reinterpret_cast<T *>(a.c.out);
         const bool pse_tma = (MODE == kModePse) && a.c.pse_tma;
@@ -1171,7 +1171,9 @@ fia_prefill_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant_
             ep_row = valid ? gm.cu_q + i : -1;
             ep_h = sg.h;
             ep_kvh = gm.kvh;
-            if constexpr (!DEFER) {
+            // (pairs that do not end both tiles together -- never in the
+            // deferring instances' plans -- take the epilogue at once)
+            if (!DEFER || (!BAND && !XB && gm.nA != gm.nB)) {
                 if (!epilogue()) goto done;
             }
         }
@@ -1341,6 +1343,9 @@ static cudaError_t launch_prefill_mode(const PrefillArgs &a, const CUtensorMap &
                 return launch_prefill_t<T, D, kModeAlibiMma, false, I8>(a, tq, tk, tv, tp, grid, ip, s);
         }
         return launch_prefill_t<T, D, kModeAlibi, false, I8>(a, tq, tk, tv, tp, grid, ip, s);
+    }
+    if constexpr (!I8) {
+        if (a.c.g >= 2) return launch_prefill_t<T, D, kModePlainGqa, false, I8>(a, tq, tk, tv, tp, grid, ip, s);
     }
     return launch_prefill_t<T, D, kModePlain, false, I8>(a, tq, tk, tv, tp, grid, ip, s);
 }
