@@ -8,7 +8,7 @@
 // generated internally, maskType 3 ALiBi from per-head slopes; V4 alibi
 // fullmask = pse tensor; V4 learnable sink; V3 lse bullet).
 //
-// One persistent CTA per SM walks a host-planned, longest-first list of tile
+// One persistent CTA per SM walks a host-planned (longest-first) list of tile
 // PAIRS: two 128-token tiles that read the same KV head (two heads of one GQA
 // group, or two consecutive tiles of one head), so every K/V tile fetched
 // serves 2 x 128 query rows.  Warp roles (18 warps):
@@ -39,6 +39,16 @@
 //              straight into the swizzled K / V stage the MMAs read.
 // TMEM (512 columns): S_0 | S_1 | O_0 | O_1.  While one softmax group works on
 // its S, the tensor core runs the other tile's PV and QK^T.
+// Modes (template MODE): plain (causal or none), plain GQA (the same for
+// g >= 2 over a 16-bit cache), ALiBi with the bias in the softmax (int8 cache
+// or qkScale <= 0), ALiBi through the MMA (16-bit cache, qkScale > 0: the
+// in-tile part of the bias is one more K-step of each QK^T block, the rest a
+// per-row constant; key tiles run last to first), pse.  In the plain GQA,
+// band and ALiBi-through-MMA instances an item's epilogue runs inside the
+// next item's first key tile, and the issuer sends that item's first QK of
+// tile 0 right after this item's last PV of tile 0.
+// Each CTA's items are ordered by (sequence, KV head) on the host, so the
+// CTAs sweep the KV heads together and K/V stays in L2 between items.
 // Every mbarrier wait is bounded in time (see fia_device.cuh).
 #include <cuda.h>
 #include <cuda_bf16.h>
